@@ -1,0 +1,256 @@
+"""Float64 CPU oracle for the NVFP4 paged KV path.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` use it; the product library never does.
+It shares no code with the CUDA path: the arithmetic lives in
+``nvkv_oracle.c`` (plain C, IEEE double), and this module only builds it
+with gcc and marshals numpy arrays into it.
+
+Sources (page titles and sections of the pages this path is built from):
+  * "gzenz/ninfer" README, "Fork changes vs upstream" -> "Context and model",
+    NVFP4 KV cache bullet: 4-bit E2M1 codes plus one E4M3 scale per group
+    of 16, here groups along head_dim.
+  * "knoopx/ninfer" README, "Capabilities and limits": chunked prefill,
+    batched decode, MTP verify with one to five drafts, one shared KV pool.
+
+Parity of every function here is pinned by ``tests/test_oracle_pins.py``
+(format tables, exhaustive rounding sweeps against an independent
+table-scan formulation and torch's float8 conversion, round-trip
+invariants, closed-form attention cases and pure-Python brute force).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "nvkv_oracle.c")
+_LIB = os.path.join(_HERE, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile nvkv_oracle.c into liboracle.so next to it (gcc -O2)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fPIC", "-shared", "-fno-fast-math",
+             "-ffp-contract=off", "-o", tmp, _SRC, "-lm", "-lpthread"])
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def lib():
+    global _lib
+    with _lock:
+        if _lib is None:
+            L = ctypes.CDLL(build())
+            d, i32, u8, u16 = ctypes.c_double, ctypes.c_int, ctypes.c_uint8, ctypes.c_uint16
+            vp = ctypes.c_void_p
+            L.oracle_bf16_value.restype = d
+            L.oracle_bf16_value.argtypes = [u16]
+            L.oracle_e2m1_value.restype = d
+            L.oracle_e2m1_value.argtypes = [i32]
+            L.oracle_e4m3_value.restype = d
+            L.oracle_e4m3_value.argtypes = [i32]
+            L.oracle_e4m3_round.restype = u8
+            L.oracle_e4m3_round.argtypes = [d]
+            L.oracle_e2m1_round_index.restype = i32
+            L.oracle_e2m1_round_index.argtypes = [d]
+            L.oracle_quantize_group.restype = None
+            L.oracle_quantize_group.argtypes = [vp, vp, vp]
+            L.oracle_quantize_groups.restype = None
+            L.oracle_quantize_groups.argtypes = [vp, ctypes.c_long, vp, vp]
+            L.oracle_dequant.restype = d
+            L.oracle_dequant.argtypes = [i32, i32]
+            L.oracle_qdq_row.restype = None
+            L.oracle_qdq_row.argtypes = [vp, i32, vp]
+            L.oracle_page_bytes.restype = ctypes.c_size_t
+            L.oracle_page_bytes.argtypes = [i32, i32]
+            L.oracle_append.restype = None
+            L.oracle_append.argtypes = [vp, i32, i32, vp, i32, vp, i32, vp, vp, vp]
+            L.oracle_pool_read_row.restype = None
+            L.oracle_pool_read_row.argtypes = [vp, i32, i32, vp, i32, i32, i32, vp]
+            L.oracle_attention_rows.restype = None
+            L.oracle_attention_rows.argtypes = [i32, vp, vp, i32, i32, vp, vp, vp, d, vp, vp, vp, i32]
+            L.oracle_attention_pool.restype = None
+            L.oracle_attention_pool.argtypes = [i32, vp, i32, i32, vp, vp, vp, vp, d, vp, vp, vp, i32]
+            _lib = L
+    return _lib
+
+
+def _ptr(a: np.ndarray) -> int:
+    assert a.flags["C_CONTIGUOUS"]
+    return a.ctypes.data
+
+
+def _u16(a) -> np.ndarray:
+    a = np.asarray(a)
+    if a.dtype != np.uint16:
+        raise TypeError("bf16 inputs are passed as their raw uint16 bits")
+    return np.ascontiguousarray(a)
+
+
+# --------------------------------------------------------------------------
+# formats
+# --------------------------------------------------------------------------
+def bf16_value(bits: int) -> float:
+    return lib().oracle_bf16_value(int(bits))
+
+
+def e2m1_value(code: int) -> float:
+    return lib().oracle_e2m1_value(int(code))
+
+
+def e4m3_value(byte: int) -> float:
+    return lib().oracle_e4m3_value(int(byte))
+
+
+def e4m3_round(x: float) -> int:
+    return int(lib().oracle_e4m3_round(float(x)))
+
+
+def e2m1_round_index(r: float) -> int:
+    return int(lib().oracle_e2m1_round_index(float(r)))
+
+
+def dequant(code: int, scale_byte: int) -> float:
+    return lib().oracle_dequant(int(code), int(scale_byte))
+
+
+def quantize_group(x_bits) -> tuple[np.ndarray, int]:
+    """16 bf16 values (uint16 bits) -> (16 E2M1 codes as uint8, E4M3 scale byte)."""
+    x = _u16(x_bits).reshape(16)
+    codes = np.zeros(16, np.uint8)
+    sb = np.zeros(1, np.uint8)
+    lib().oracle_quantize_group(_ptr(x), _ptr(codes), _ptr(sb))
+    return codes, int(sb[0])
+
+
+def quantize_rows(x_bits) -> tuple[np.ndarray, np.ndarray]:
+    """[..., D] bf16 bits -> codes [..., D] (uint8, one per element) and
+    scales [..., D/16] (uint8)."""
+    x = _u16(x_bits)
+    D = x.shape[-1]
+    flat = np.ascontiguousarray(x.reshape(-1, 16))
+    codes = np.zeros(flat.shape, np.uint8)
+    scales = np.zeros(flat.shape[0], np.uint8)
+    lib().oracle_quantize_groups(_ptr(flat), flat.shape[0], _ptr(codes), _ptr(scales))
+    return codes.reshape(x.shape), scales.reshape(x.shape[:-1] + (D // 16,))
+
+
+def qdq_rows(x_bits) -> np.ndarray:
+    """Quantise and dequantise rows of bf16 bits ([..., D]) -> float64."""
+    x = _u16(x_bits)
+    D = x.shape[-1]
+    flat = np.ascontiguousarray(x.reshape(-1, D))
+    out = np.zeros(flat.shape, np.float64)
+    L = lib()
+    for i in range(flat.shape[0]):
+        L.oracle_qdq_row(flat[i].ctypes.data, D, out[i].ctypes.data)
+    return out.reshape(x.shape)
+
+
+# --------------------------------------------------------------------------
+# pool
+# --------------------------------------------------------------------------
+def page_bytes(num_kv_heads: int, head_dim: int) -> int:
+    return int(lib().oracle_page_bytes(num_kv_heads, head_dim))
+
+
+def append(pool: np.ndarray, num_kv_heads: int, head_dim: int, page_table: np.ndarray,
+           kv_lens: np.ndarray, k_new, v_new, cu_new: np.ndarray) -> None:
+    """Quantise k_new / v_new ([rows][Hkv][D] bf16 bits) into the pool image
+    in place; see oracle_append in nvkv_oracle.c for the position rule."""
+    assert pool.dtype == np.uint8 and pool.flags["C_CONTIGUOUS"]
+    pt = np.ascontiguousarray(page_table, np.int32)
+    kl = np.ascontiguousarray(kv_lens, np.int32)
+    cu = np.ascontiguousarray(cu_new, np.int32)
+    k = _u16(k_new)
+    v = _u16(v_new)
+    lib().oracle_append(_ptr(pool), num_kv_heads, head_dim, _ptr(pt), pt.shape[1], _ptr(kl),
+                        kl.shape[0], _ptr(k), _ptr(v), _ptr(cu))
+
+
+def pool_read_row(pool: np.ndarray, num_kv_heads: int, head_dim: int, page_row: np.ndarray,
+                  pos: int, h: int, is_v: bool) -> np.ndarray:
+    pr = np.ascontiguousarray(page_row, np.int32)
+    out = np.zeros(head_dim, np.float64)
+    lib().oracle_pool_read_row(_ptr(pool), num_kv_heads, head_dim, _ptr(pr), int(pos), int(h),
+                               int(bool(is_v)), _ptr(out))
+    return out
+
+
+# --------------------------------------------------------------------------
+# attention
+# --------------------------------------------------------------------------
+def _ptr_array(arrs) -> np.ndarray:
+    return np.array([a.ctypes.data for a in arrs], dtype=np.uint64)
+
+
+def attention_rows(jobs, num_kv_heads: int, head_dim: int, sm_scale: float,
+                   nthreads: int | None = None):
+    """Exact softmax attention for a list of output rows over a logical cache.
+
+    jobs: iterable of (k_rows, v_rows, h, n_visible, q) with k_rows / v_rows
+    the sequence's bf16 bits [rows][Hkv][D] in position order, h the kv-head,
+    n_visible the number of visible keys (position + 1) and q the [D] bf16
+    bits of the query row.  Returns (out [n][D] f64, lse [n], psum [n])."""
+    jobs = list(jobs)
+    n = len(jobs)
+    keep = []
+    ks, vs, qs = [], [], []
+    hs = np.zeros(n, np.int32)
+    nv = np.zeros(n, np.int32)
+    for i, (k, v, h, nvis, q) in enumerate(jobs):
+        k = _u16(k)
+        v = _u16(v)
+        q = _u16(q).reshape(head_dim)
+        keep += [k, v, q]
+        ks.append(k)
+        vs.append(v)
+        qs.append(q)
+        hs[i] = h
+        nv[i] = nvis
+    kp, vp_, qp = _ptr_array(ks), _ptr_array(vs), _ptr_array(qs)
+    out = np.zeros((n, head_dim), np.float64)
+    lse = np.zeros(n, np.float64)
+    psum = np.zeros(n, np.float64)
+    lib().oracle_attention_rows(n, _ptr(kp), _ptr(vp_), num_kv_heads, head_dim, _ptr(hs),
+                                _ptr(nv), _ptr(qp), float(sm_scale), _ptr(out), _ptr(lse),
+                                _ptr(psum), int(nthreads or os.cpu_count() or 1))
+    del keep
+    return out, lse, psum
+
+
+def attention_pool(pool: np.ndarray, num_kv_heads: int, head_dim: int, jobs, sm_scale: float,
+                   nthreads: int | None = None):
+    """As attention_rows, but the cache is a pool image; jobs are
+    (page_row, h, n_visible, q)."""
+    jobs = list(jobs)
+    n = len(jobs)
+    keep, prs, qs = [], [], []
+    hs = np.zeros(n, np.int32)
+    nv = np.zeros(n, np.int32)
+    for i, (pr, h, nvis, q) in enumerate(jobs):
+        pr = np.ascontiguousarray(pr, np.int32)
+        q = _u16(q).reshape(head_dim)
+        keep += [pr, q]
+        prs.append(pr)
+        qs.append(q)
+        hs[i] = h
+        nv[i] = nvis
+    pp, qp = _ptr_array(prs), _ptr_array(qs)
+    out = np.zeros((n, head_dim), np.float64)
+    lse = np.zeros(n, np.float64)
+    psum = np.zeros(n, np.float64)
+    lib().oracle_attention_pool(n, _ptr(pool), num_kv_heads, head_dim, _ptr(pp), _ptr(hs),
+                                _ptr(nv), _ptr(qp), float(sm_scale), _ptr(out), _ptr(lse),
+                                _ptr(psum), int(nthreads or os.cpu_count() or 1))
+    del keep
+    return out, lse, psum
