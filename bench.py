@@ -1,0 +1,317 @@
+"""Benchmark of the NVFP4 paged-KV hot path on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--T 1|6] [--impl native|reference]
+
+Workload: the long-context agentic batch -- 3 sequences with 330000,
+420000 and 470000 cached tokens, 24 query / 4 KV heads, head_dim 256, NVFP4
+KV in random page order -- decoding T=1 token each (T=6 for MTP verify).
+One step = quantise-append this step's K/V rows + split-K decode attention +
+combine, i.e. one attention layer of one decode iteration.  Inputs are
+synthetic (seeded N(0,1) bf16, four K channels x10) and resident in HBM;
+the 1.4 GB pool is larger than L2, so no flush is needed between steps.
+
+Metric: NVFP4 KV-read GB/s = algorithmic KV bytes of the step (every
+visible cached token, K and V, every kv-head, read once) / step time, with
+decode tokens/s (B*T query tokens per layer-call / step time) beside it.
+
+Launched with torchrun for N > 1: every rank runs its own replica of the
+workload (the path has no cross-GPU exchange); the reported value is the
+bytes of all ranks over the max-over-ranks time.
+
+--impl reference runs the float64 CPU oracle on a bounded sample of the
+same workload on this machine's host cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "NVFP4 KV-read GB/s (% of HBM peak) and decode tokens/s at 3x~470k ctx"
+FALLBACK_HBM_GBS = 6650.0
+
+
+def hbm_peak():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM_GBS, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks and throttle reasons sampled during the timed region."""
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.proc = None
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-i", str(gpu_index), "-lms", "200"], stdout=subprocess.PIPE,
+                stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in out.strip().splitlines():
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, parts[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+def oracle_sample(wl, rows_max=6, ctx_cap=None):
+    """Time the float64 oracle on one (sequence 0, kv-head 0) pair: all its
+    query rows over its whole visible cache.  Returns (GB/s in the metric's
+    unit, seconds, threads, description)."""
+    import oracle
+    b, h = 0, 0
+    kv_len = int(wl.kv_lens[b]) if ctx_cap is None else min(int(wl.kv_lens[b]), ctx_cap)
+    k, v = wl.kv_rows(b, 0, kv_len)
+    q = wl.queries()
+    G = wl.group
+    jobs = []
+    for t in range(wl.T):
+        for g in range(G):
+            n_vis = min(wl.query_position(b, t) + 1, kv_len)
+            jobs.append((k, v, h, n_vis, q[b * wl.T + t, h * G + g]))
+    jobs = jobs[:rows_max]
+    threads = os.cpu_count() or 1
+    oracle.lib()  # build / load outside the timed region
+    t0 = time.perf_counter()
+    oracle.attention_rows(jobs, wl.num_kv_heads, wl.head_dim, wl.sm_scale, threads)
+    dt = time.perf_counter() - t0
+    kv_bytes = kv_len * wl.head_dim * 2 * (1 / 2 + 1 / 16)  # one kv-head, K and V, NVFP4
+    desc = (f"sequence 0 ({kv_len} tokens), kv-head 0, {len(jobs)} query rows (all rows of that "
+            f"pair), float64 oracle, {min(threads, len(jobs))} threads busy")
+    return kv_bytes / dt / 1e9, dt, min(threads, len(jobs)), desc
+
+
+def run_reference(args):
+    from nvfp4_quantized_kv_b200 import workload as W
+    if int(os.environ.get("RANK", "0")) != 0:
+        return
+    wl = W.long_context(T=args.T)
+    cap = args.ref_ctx
+    vals = []
+    for _ in range(args.warmup):
+        oracle_sample(wl, ctx_cap=cap)
+    secs = 0.0
+    for _ in range(args.steps):
+        v, dt, threads, desc = oracle_sample(wl, ctx_cap=cap)
+        vals.append(v)
+        secs += dt
+    value = statistics.mean(vals)
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1000 * secs / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": wl.name, "sample": desc},
+        "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                         "sample": desc},
+        "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--T", type=int, default=1, help="queries per sequence: 1 decode, 6 MTP verify")
+    ap.add_argument("--impl", choices=["native", "reference"], default="native")
+    ap.add_argument("--num-splits", type=int, default=0)
+    ap.add_argument("--ref-ctx", type=int, default=None,
+                    help="reference arm: cap the sampled context (default: whole sequence 0)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        raise SystemExit("--warmup must be >= 3")
+    if args.impl == "reference":
+        run_reference(args)
+        return
+
+    import torch
+    import torch.distributed as dist
+    import nvfp4_quantized_kv_b200 as nv
+    from nvfp4_quantized_kv_b200 import workload as W
+    from nvfp4_quantized_kv_b200.harness import DeviceWorkload
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
+
+    wl = W.long_context(T=args.T)
+    dw = DeviceWorkload(wl, dev, fill=None, num_splits=args.num_splits)
+    dw.fill_context()
+    dw.load_step_inputs()
+    S = dw.num_splits or nv.nvkv_default_num_splits()
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        dw.append(stream)
+        dw.attend(stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+
+    # ---- timed region: K steps, events around every kernel ----
+    K = args.steps
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K)]
+    clocks = ClockSampler(local)
+    time.sleep(0.3)
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_end = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    t_start.record(stream)
+    for i in range(K):
+        e = ev[i]
+        e[0].record(stream)
+        nv.nvkv_append(dw.cache, dw.seqs, dw.k_new, dw.v_new, dw.cu_new, wl.batch * wl.T, wl.T, stream)
+        e[1].record(stream)
+        nv.nvkv_decode_attn(dw.cache, dw.seqs, dw.q, wl.T, wl.num_q_heads, wl.sm_scale, S,
+                            dw.workspace, stream)
+        e[2].record(stream)
+        nv.nvkv_combine(dw.seqs, dw.workspace, wl.T, wl.num_q_heads, wl.num_kv_heads, wl.head_dim,
+                        S, dw.out, stream)
+        e[3].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    ms = t_start.elapsed_time(t_end) / K
+    t_append = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    t_decode = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    t_combine = statistics.mean(e[2].elapsed_time(e[3]) for e in ev)
+    if world > 1:
+        tt = torch.tensor([ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    err = dw.err_bits()
+
+    kv_bytes = wl.kv_bytes_per_step()
+    value = world * kv_bytes / (ms * 1e-3) / 1e9
+    tokens_per_s = world * wl.batch * wl.T / (ms * 1e-3)
+    peak, peak_kind = hbm_peak()
+    decode_gbs = kv_bytes / (t_decode * 1e-3) / 1e9
+
+    # ---- end to end through the public API with host buffers ----
+    pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
+    h_k = pin(dw.k_new_np.view(np.int16))
+    h_v = pin(dw.v_new_np.view(np.int16))
+    h_q = pin(dw.q_np.view(np.int16))
+    h_out = torch.empty(dw.out.shape, dtype=torch.bfloat16).pin_memory()
+    d_k, d_v, d_q = (torch.empty(t.shape, dtype=torch.int16, device=dev) for t in (h_k, h_v, h_q))
+
+    def e2e_step():
+        d_k.copy_(h_k, non_blocking=True)
+        d_v.copy_(h_v, non_blocking=True)
+        d_q.copy_(h_q, non_blocking=True)
+        nv.nvkv_append(dw.cache, dw.seqs, d_k.view(torch.bfloat16), d_v.view(torch.bfloat16),
+                       dw.cu_new, wl.batch * wl.T, wl.T, stream)
+        nv.nvkv_decode_attn(dw.cache, dw.seqs, d_q.view(torch.bfloat16), wl.T, wl.num_q_heads,
+                            wl.sm_scale, S, dw.workspace, stream)
+        nv.nvkv_combine(dw.seqs, dw.workspace, wl.T, wl.num_q_heads, wl.num_kv_heads, wl.head_dim,
+                        S, dw.out, stream)
+        h_out.copy_(dw.out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        dist.barrier()
+    e0 = torch.cuda.Event(enable_timing=True)
+    e1 = torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(args.e2e_steps):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
+    if world > 1:
+        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        e2e_ms = float(tt.item())
+    h2d = h_k.numel() * 2 + h_v.numel() * 2 + h_q.numel() * 2
+    d2h = h_out.numel() * 2
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, dt, threads, desc = oracle_sample(wl)
+        cpu = {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc,
+               "seconds": dt}
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
+            "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": wl.name, "batch": wl.batch, "context": list(wl.ctx),
+                       "T": wl.T, "q_heads": wl.num_q_heads, "kv_heads": wl.num_kv_heads,
+                       "head_dim": wl.head_dim, "page_tokens": 16, "num_splits": S,
+                       "kv_bytes_per_step": kv_bytes, "l2": "inputs larger than L2 (1.4 GB pool)",
+                       "parallelism": f"replicas{world}" if world > 1 else "single-gpu"},
+            "hbm_frac": value / world / peak,
+            "decode_tokens_per_s": tokens_per_s,
+            "kernel_ms": {"append": t_append, "decode_attn": t_decode, "combine": t_combine},
+            "roofline": {"bound": "hbm", "achieved": decode_gbs, "peak": peak, "unit": "GB/s",
+                         "frac": decode_gbs / peak, "traffic": None,
+                         "kernel": "decode_attn", "peak_kind": peak_kind},
+            "e2e": {"value": world * kv_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
+                    "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
+            "gpu_launches": 3 * K,
+            "clocks": clk,
+            "device_errors": err,
+            "cpu_baseline": cpu,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,176 @@
+/*
+ * nvkv.h -- C ABI of libnvkv: attention over an NVFP4-quantised paged KV
+ * cache on NVIDIA B200 (sm_100a).
+ *
+ * The storage format is the one stated in the "gzenz/ninfer" README, section
+ * "Fork changes vs upstream", subsection "Context and model", NVFP4 KV cache
+ * bullet: every KV element is a 4-bit E2M1 code and each group of 16
+ * elements (here: 16 consecutive head_dim elements of one token and one
+ * kv-head) shares one E4M3 scale.  The serving features the calls follow are
+ * those listed in the "knoopx/ninfer" README, section "Capabilities and
+ * limits": one shared, startup-fixed KV pool serving every active request,
+ * batched decode replayed from CUDA Graphs, MTP speculative verify with one
+ * to five draft tokens (T = drafts + 1 causal queries per sequence), and
+ * chunked prefill; one GPU.
+ *
+ * Conventions for every call
+ *  - Every pointer named "device" is GPU memory owned by the caller; the
+ *    library never allocates, frees, synchronises or reads device memory
+ *    from the host.  Each call only enqueues kernels on `stream` (NULL = the
+ *    legacy default stream) and returns, so every call can be captured in a
+ *    CUDA Graph.
+ *  - Host-checkable argument errors return NVKV_ERR_INVALID_ARG or
+ *    NVKV_ERR_UNSUPPORTED before anything is launched; a failed launch
+ *    returns NVKV_ERR_CUDA.
+ *  - Device-resident metadata (page ids, lengths) is checked by the kernels:
+ *    an out-of-range page id or length is skipped (nothing is read or
+ *    written through it) and, when `err_word` is non-NULL, the matching
+ *    NVKV_DEVERR_* bit is OR-ed into *err_word.  Kernels never trap.
+ *  - bf16 tensors are row-major and contiguous, 16-byte aligned.
+ *
+ * Pool layout (this library's own; the pages do not fix one).  A page holds
+ * 16 consecutive token slots of one sequence for every kv-head.  Page p starts
+ * at pool + p * nvkv_page_bytes(Hkv, D); inside it, kv-head h owns the
+ * 18*D-byte block at offset h*18*D:
+ *   [0,     8D)  K codes  [16 slots][D/2]: byte i of a slot holds element 2i
+ *                in its low nibble and element 2i+1 in its high nibble
+ *   [8D,    9D)  K scales [16 slots][D/16]: byte g scales elements 16g..16g+15
+ *   [9D,   17D)  V codes  [D][8]: byte (d, i) holds slot 2i in its low nibble
+ *                and slot 2i+1 in its high nibble (V is stored transposed so a
+ *                head_dim row of 16 tokens is 8 contiguous bytes)
+ *   [17D,  18D)  V scales [D/16][16 slots]
+ * A code is sign<<3 | magnitude index, magnitudes {0,.5,1,1.5,2,3,4,6};
+ * value = E2M1(code) * E4M3(scale).  Quantisation of a group: scale = E4M3
+ * nearest to amax/6 (ties to even, saturating at 448); code = E2M1 nearest
+ * to x/scale (ties to even, saturating at 6); a scale of 0 gives all codes 0;
+ * a magnitude that rounds to 0 is stored as code 0.
+ */
+#ifndef NVKV_H
+#define NVKV_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same object as cudaStream_t. */
+typedef struct CUstream_st *nvkv_stream_t;
+
+typedef enum nvkv_status {
+    NVKV_OK = 0,
+    NVKV_ERR_INVALID_ARG = 1,  /* null pointer, negative size, inconsistent shape */
+    NVKV_ERR_UNSUPPORTED = 2,  /* valid but outside what the kernels implement */
+    NVKV_ERR_WORKSPACE = 3,    /* workspace missing, too small or misaligned */
+    NVKV_ERR_CUDA = 4          /* a kernel launch failed (cudaGetLastError) */
+} nvkv_status;
+
+/* Bits OR-ed into *err_word by the kernels. */
+#define NVKV_DEVERR_PAGE_ID 1u   /* a page-table entry outside [0, num_pages) */
+#define NVKV_DEVERR_LENGTH 2u    /* kv_len outside [rows or queries, max_kv_len] or
+                                    beyond max_pages_per_seq * 16 */
+#define NVKV_DEVERR_TIMEOUT 4u   /* a bounded wait inside a kernel gave up */
+
+/* The paged pool. */
+typedef struct nvkv_cache {
+    uint8_t *pool;          /* device, num_pages * nvkv_page_bytes() bytes, 16-B aligned */
+    int32_t num_pages;
+    int32_t num_kv_heads;   /* Hkv >= 1 */
+    int32_t head_dim;       /* D: 128 or 256 */
+} nvkv_cache;
+
+/* The batch of sequences a call works on. */
+typedef struct nvkv_seqs {
+    const int32_t *page_table;  /* device [batch][max_pages_per_seq]; entry i of
+                                   row b is the page holding positions 16i..16i+15 */
+    int32_t max_pages_per_seq;  /* row stride of page_table */
+    const int32_t *kv_lens;     /* device [batch]: tokens in the cache of each
+                                   sequence, INCLUDING the rows of this step */
+    int32_t batch;              /* B >= 1 */
+    int32_t max_kv_len;         /* host upper bound of kv_lens (sizes grids) */
+    int32_t *err_word;          /* device int32 or NULL (see NVKV_DEVERR_*) */
+} nvkv_seqs;
+
+/* Bytes of one page: 18 * num_kv_heads * head_dim (4.5 bits per element).
+ * Returns 0 for non-positive arguments. */
+size_t nvkv_page_bytes(int32_t num_kv_heads, int32_t head_dim);
+
+/* Quantise new K and V rows into the pool (the NVFP4 KV cache bullet above).
+ *   k_new, v_new: device bf16 [total_new][Hkv][D].
+ *   cu_new:       device int32 [batch+1], cu_new[0] = 0, non-decreasing;
+ *                 rows cu_new[b] .. cu_new[b+1]-1 belong to sequence b and are
+ *                 written to positions kv_lens[b]-n_b .. kv_lens[b]-1,
+ *                 n_b = cu_new[b+1]-cu_new[b].
+ *   total_new:    cu_new[batch] (host copy); max_new >= every n_b (host bound).
+ * Writes exactly the code nibbles and scale bytes of those positions; every
+ * other pool byte, including the other nibble of a shared V code byte, is
+ * left as it was.  Sequences must not share pages written by the same call. */
+nvkv_status nvkv_append(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *k_new,
+                        const void *v_new, const int32_t *cu_new, int32_t total_new,
+                        int32_t max_new, nvkv_stream_t stream);
+
+/* Split-K ("flash-decoding") plan used by nvkv_decode_attn / nvkv_combine.
+ *
+ * The KV of every (sequence, kv-head) pair is cut into 128-token units; the
+ * units of all pairs, ordered by (b, h, unit), are dealt to num_splits
+ * contiguous, equal-sized (+-1 unit) ranges.  Range c writes one partial
+ * result per pair it touches, into workspace slot c + b*Hkv + h, so a
+ * workspace holds num_splits + batch*Hkv - 1 slots.  num_splits = 0 picks
+ * the default for this GPU (a multiple of its SM count).
+ *
+ * nvkv_decode_workspace_bytes: bytes of workspace for T queries per
+ * sequence (rows = T * Hq/Hkv per pair); 0 on invalid arguments. */
+int32_t nvkv_default_num_splits(void);
+size_t nvkv_decode_workspace_bytes(int32_t batch, int32_t T, int32_t num_q_heads,
+                                   int32_t num_kv_heads, int32_t head_dim, int32_t num_splits);
+
+/* Host-side copy of the split plan, for inspection and tests: given host
+ * kv_lens[batch], writes for every pair bh = b*Hkv + h the first and last
+ * split touching it (first_split[bh] > last_split[bh] when the pair has no
+ * KV).  Launches nothing. */
+nvkv_status nvkv_split_plan(const int32_t *kv_lens_host, int32_t batch, int32_t num_kv_heads,
+                            int32_t num_splits, int32_t *first_split, int32_t *last_split);
+
+/* Decode / MTP-verify attention, first half: partial results per split.
+ *   q: device bf16 [batch*T][Hq][D]; row b*T + t is query t of sequence b,
+ *      at position kv_lens[b] - T + t, which sees keys 0 .. that position
+ *      (causal).  Query head hq reads kv-head hq / (Hq/Hkv).
+ *   T: 1 .. 16 queries per sequence; Hq a multiple of Hkv with T*Hq/Hkv <= 128.
+ *   sm_scale: scores are sm_scale * q.k (typically 1/sqrt(D)).
+ *   workspace: device, >= nvkv_decode_workspace_bytes(...), 16-B aligned.
+ * The scores, softmax and value sums run in fp32 on dequantised values;
+ * nvkv_combine must follow with the same T, heads and num_splits. */
+nvkv_status nvkv_decode_attn(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *q,
+                             int32_t T, int32_t num_q_heads, float sm_scale, int32_t num_splits,
+                             void *workspace, size_t workspace_bytes, nvkv_stream_t stream);
+
+/* Decode / MTP-verify attention, second half: merges the per-split partial
+ * results (log-sum-exp weighting) into out, device bf16 [batch*T][Hq][D].
+ * A query row that sees no key (kv_len < T - t) gets zeros. */
+nvkv_status nvkv_combine(const nvkv_seqs *seqs, const void *workspace, int32_t T,
+                         int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                         int32_t num_splits, void *out, nvkv_stream_t stream);
+
+/* Chunked-prefill attention ("knoopx/ninfer" README, "Capabilities and
+ * limits": chunked prefill): causal attention of a chunk of new queries
+ * against the whole cache of their sequence, whose K/V rows (including the
+ * chunk's own) have already been appended.
+ *   q:    device bf16 [total_q][Hq][D]; cu_q device int32 [batch+1]; rows
+ *         cu_q[b] .. cu_q[b+1]-1 are the n_b newest positions of sequence b
+ *         (kv_lens[b]-n_b .. kv_lens[b]-1).
+ *   total_q = cu_q[batch] (host), max_q >= every n_b (host bound).
+ *   out:  device bf16 [total_q][Hq][D]. */
+nvkv_status nvkv_prefill_attn(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *q,
+                              const int32_t *cu_q, int32_t total_q, int32_t max_q,
+                              int32_t num_q_heads, float sm_scale, void *out,
+                              nvkv_stream_t stream);
+
+/* Static description of a status code. */
+const char *nvkv_status_string(nvkv_status status);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NVKV_H */

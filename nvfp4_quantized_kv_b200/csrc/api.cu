@@ -1,0 +1,200 @@
+// api.cu -- the extern "C" boundary of libnvkv (declared in include/nvkv.h):
+// host-side argument checks, workspace carving and kernel dispatch.  Nothing
+// here allocates, synchronises or reads device memory.
+#include <cmath>
+
+#include "nvkv_common.cuh"
+
+namespace nvkv {
+cudaError_t launch_append(const nvkv_cache &, const nvkv_seqs &, const void *, const void *,
+                          const int32_t *, int, int, cudaStream_t);
+cudaError_t launch_decode_simt(const nvkv_cache &, const nvkv_seqs &, const void *, int, int,
+                               float, int, float *, float *, cudaStream_t);
+cudaError_t launch_combine(const nvkv_seqs &, const void *, const void *, int, int, int, int, int,
+                           void *, cudaStream_t);
+cudaError_t launch_prefill_simt(const nvkv_cache &, const nvkv_seqs &, const void *,
+                                const int32_t *, int, int, float, void *, cudaStream_t);
+}  // namespace nvkv
+
+using namespace nvkv;
+
+namespace {
+
+constexpr int kMaxT = 16;
+constexpr int kMaxRows = 128;  // T * Hq / Hkv per (sequence, kv-head)
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+nvkv_status check_cache(const nvkv_cache *c) {
+  if (!c || !c->pool || !aligned16(c->pool)) return NVKV_ERR_INVALID_ARG;
+  if (c->num_pages <= 0 || c->num_kv_heads <= 0) return NVKV_ERR_INVALID_ARG;
+  if (c->head_dim != 128 && c->head_dim != 256) return NVKV_ERR_UNSUPPORTED;
+  return NVKV_OK;
+}
+
+nvkv_status check_seqs(const nvkv_seqs *s) {
+  if (!s || !s->page_table || !s->kv_lens) return NVKV_ERR_INVALID_ARG;
+  if (s->batch <= 0 || s->max_pages_per_seq <= 0 || s->max_kv_len < 0) return NVKV_ERR_INVALID_ARG;
+  if ((int64_t)s->max_kv_len > (int64_t)s->max_pages_per_seq * kPageTokens)
+    return NVKV_ERR_INVALID_ARG;
+  return NVKV_OK;
+}
+
+nvkv_status check_heads(int Hq, int Hkv, int D, int T) {
+  if (Hq <= 0 || Hkv <= 0 || Hq % Hkv != 0) return NVKV_ERR_INVALID_ARG;
+  if (D != 128 && D != 256) return NVKV_ERR_UNSUPPORTED;
+  if (T <= 0) return NVKV_ERR_INVALID_ARG;
+  if (T > kMaxT || (int64_t)T * (Hq / Hkv) > kMaxRows) return NVKV_ERR_UNSUPPORTED;
+  return NVKV_OK;
+}
+
+int resolve_splits(int num_splits) {
+  return num_splits > 0 ? num_splits : nvkv_default_num_splits();
+}
+
+struct WorkspaceLayout {
+  size_t o_bytes, lse_off, total;
+};
+
+WorkspaceLayout layout(int batch, int T, int Hq, int Hkv, int D, int S) {
+  const size_t R = (size_t)T * (Hq / Hkv);
+  const size_t slots = (size_t)S + (size_t)batch * Hkv - 1;
+  WorkspaceLayout w;
+  w.o_bytes = align256(slots * R * D * sizeof(float));
+  w.lse_off = w.o_bytes;
+  w.total = w.o_bytes + align256(slots * R * sizeof(float));
+  return w;
+}
+
+nvkv_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NVKV_OK : NVKV_ERR_CUDA; }
+
+}  // namespace
+
+extern "C" {
+
+size_t nvkv_page_bytes(int32_t num_kv_heads, int32_t head_dim) {
+  if (num_kv_heads <= 0 || head_dim <= 0) return 0;
+  return (size_t)18 * num_kv_heads * head_dim;
+}
+
+int32_t nvkv_default_num_splits(void) {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+    cudaGetLastError();  // the failed query leaves a (non-sticky) error; clear it
+    sms = 148;           // B200
+  }
+  return 2 * sms;
+}
+
+size_t nvkv_decode_workspace_bytes(int32_t batch, int32_t T, int32_t num_q_heads,
+                                   int32_t num_kv_heads, int32_t head_dim, int32_t num_splits) {
+  if (batch <= 0 || num_splits < 0) return 0;
+  if (check_heads(num_q_heads, num_kv_heads, head_dim, T) != NVKV_OK) return 0;
+  return layout(batch, T, num_q_heads, num_kv_heads, head_dim, resolve_splits(num_splits)).total;
+}
+
+nvkv_status nvkv_split_plan(const int32_t *kv_lens_host, int32_t batch, int32_t num_kv_heads,
+                            int32_t num_splits, int32_t *first_split, int32_t *last_split) {
+  if (!kv_lens_host || !first_split || !last_split || batch <= 0 || num_kv_heads <= 0 ||
+      num_splits < 0)
+    return NVKV_ERR_INVALID_ARG;
+  const int64_t S = resolve_splits(num_splits);
+  int64_t U = 0;
+  for (int b = 0; b < batch; ++b) {
+    if (kv_lens_host[b] < 0) return NVKV_ERR_INVALID_ARG;
+    U += (int64_t)units_of_len(kv_lens_host[b]) * num_kv_heads;
+  }
+  int64_t start = 0;
+  for (int b = 0; b < batch; ++b) {
+    const int ub = units_of_len(kv_lens_host[b]);
+    for (int h = 0; h < num_kv_heads; ++h) {
+      const int bh = b * num_kv_heads + h;
+      if (ub == 0) {
+        first_split[bh] = 0;
+        last_split[bh] = -1;
+      } else {
+        first_split[bh] = (int32_t)range_of_unit(start, U, S);
+        last_split[bh] = (int32_t)range_of_unit(start + ub - 1, U, S);
+      }
+      start += ub;
+    }
+  }
+  return NVKV_OK;
+}
+
+nvkv_status nvkv_append(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *k_new,
+                        const void *v_new, const int32_t *cu_new, int32_t total_new,
+                        int32_t max_new, nvkv_stream_t stream) {
+  nvkv_status st = check_cache(cache);
+  if (st != NVKV_OK) return st;
+  if ((st = check_seqs(seqs)) != NVKV_OK) return st;
+  if (total_new < 0 || max_new < 0) return NVKV_ERR_INVALID_ARG;
+  if (total_new == 0 || max_new == 0) return NVKV_OK;
+  if (!k_new || !v_new || !cu_new || !aligned16(k_new) || !aligned16(v_new))
+    return NVKV_ERR_INVALID_ARG;
+  return cuda_status(launch_append(*cache, *seqs, k_new, v_new, cu_new, total_new, max_new,
+                                   reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvkv_status nvkv_decode_attn(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *q,
+                             int32_t T, int32_t num_q_heads, float sm_scale, int32_t num_splits,
+                             void *workspace, size_t workspace_bytes, nvkv_stream_t stream) {
+  nvkv_status st = check_cache(cache);
+  if (st != NVKV_OK) return st;
+  if ((st = check_seqs(seqs)) != NVKV_OK) return st;
+  if ((st = check_heads(num_q_heads, cache->num_kv_heads, cache->head_dim, T)) != NVKV_OK) return st;
+  if (!q || !aligned16(q) || !std::isfinite(sm_scale) || num_splits < 0) return NVKV_ERR_INVALID_ARG;
+  const int S = resolve_splits(num_splits);
+  const WorkspaceLayout w = layout(seqs->batch, T, num_q_heads, cache->num_kv_heads,
+                                   cache->head_dim, S);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < w.total) return NVKV_ERR_WORKSPACE;
+  float *ws_o = static_cast<float *>(workspace);
+  float *ws_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) + w.lse_off);
+  return cuda_status(launch_decode_simt(*cache, *seqs, q, T, num_q_heads, sm_scale, S, ws_o,
+                                        ws_lse, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvkv_status nvkv_combine(const nvkv_seqs *seqs, const void *workspace, int32_t T,
+                         int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
+                         int32_t num_splits, void *out, nvkv_stream_t stream) {
+  nvkv_status st = check_seqs(seqs);
+  if (st != NVKV_OK) return st;
+  if ((st = check_heads(num_q_heads, num_kv_heads, head_dim, T)) != NVKV_OK) return st;
+  if (!out || !aligned16(out) || num_splits < 0) return NVKV_ERR_INVALID_ARG;
+  if (!workspace || !aligned16(workspace)) return NVKV_ERR_WORKSPACE;
+  const int S = resolve_splits(num_splits);
+  const WorkspaceLayout w = layout(seqs->batch, T, num_q_heads, num_kv_heads, head_dim, S);
+  const void *ws_lse = static_cast<const char *>(workspace) + w.lse_off;
+  return cuda_status(launch_combine(*seqs, workspace, ws_lse, T, num_q_heads, num_kv_heads,
+                                    head_dim, S, out, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvkv_status nvkv_prefill_attn(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *q,
+                              const int32_t *cu_q, int32_t total_q, int32_t max_q,
+                              int32_t num_q_heads, float sm_scale, void *out,
+                              nvkv_stream_t stream) {
+  nvkv_status st = check_cache(cache);
+  if (st != NVKV_OK) return st;
+  if ((st = check_seqs(seqs)) != NVKV_OK) return st;
+  if (num_q_heads <= 0 || num_q_heads % cache->num_kv_heads != 0) return NVKV_ERR_INVALID_ARG;
+  if (total_q < 0 || max_q < 0 || !std::isfinite(sm_scale)) return NVKV_ERR_INVALID_ARG;
+  if (total_q == 0) return NVKV_OK;
+  if (!q || !cu_q || !out || !aligned16(q) || !aligned16(out)) return NVKV_ERR_INVALID_ARG;
+  return cuda_status(launch_prefill_simt(*cache, *seqs, q, cu_q, total_q, num_q_heads, sm_scale,
+                                         out, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+const char *nvkv_status_string(nvkv_status status) {
+  switch (status) {
+    case NVKV_OK: return "ok";
+    case NVKV_ERR_INVALID_ARG: return "invalid argument";
+    case NVKV_ERR_UNSUPPORTED: return "unsupported shape";
+    case NVKV_ERR_WORKSPACE: return "workspace missing, misaligned or too small";
+    case NVKV_ERR_CUDA: return "CUDA launch error";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

@@ -1,0 +1,122 @@
+// nvkv_common.cuh -- shared device helpers of the NVFP4 paged-KV kernels.
+//
+// Storage format: "gzenz/ninfer" README, "Fork changes vs upstream" ->
+// "Context and model", NVFP4 KV cache bullet (4-bit E2M1 codes, one E4M3
+// scale per 16 elements).  The page layout is documented in include/nvkv.h.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+#include <cuda_fp8.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/nvkv.h"
+
+namespace nvkv {
+
+constexpr int kPageTokens = 16;   // token slots per page
+constexpr int kGroup = 16;        // elements per E4M3 scale
+constexpr int kUnitTokens = 128;  // split-plan unit (8 pages)
+
+// Byte offsets inside one kv-head block of a page (18*D bytes).
+__host__ __device__ constexpr int kc_off(int) { return 0; }
+__host__ __device__ constexpr int ks_off(int D) { return 8 * D; }
+__host__ __device__ constexpr int vc_off(int D) { return 9 * D; }
+__host__ __device__ constexpr int vs_off(int D) { return 17 * D; }
+__host__ __device__ constexpr int head_bytes(int D) { return 18 * D; }
+
+// ---------------------------------------------------------------------------
+// Split plan (see nvkv_decode_workspace_bytes in nvkv.h).  Units of 128
+// tokens of every (b, h) pair, in (b, h, unit) order, are dealt to S ranges:
+// range c owns units [c*U/S, (c+1)*U/S).
+// ---------------------------------------------------------------------------
+__host__ __device__ inline int64_t range_begin(int64_t c, int64_t U, int64_t S) {
+  return (c * U) / S;
+}
+// The range holding unit u (0 <= u < U): the largest c with range_begin(c) <= u.
+__host__ __device__ inline int64_t range_of_unit(int64_t u, int64_t U, int64_t S) {
+  return ((u + 1) * S - 1) / U;
+}
+__host__ __device__ inline int units_of_len(int kv_len) {
+  return kv_len > 0 ? (kv_len + kUnitTokens - 1) / kUnitTokens : 0;
+}
+
+// ---------------------------------------------------------------------------
+// Error reporting: never trap, OR a bit into the caller's word.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ void report(int32_t *err, unsigned bit) {
+  if (err) atomicOr(reinterpret_cast<unsigned *>(err), bit);
+}
+
+// ---------------------------------------------------------------------------
+// Number formats.
+// ---------------------------------------------------------------------------
+// E4M3 byte -> fp32 (exact), through the hardware fp8 -> f16 conversion.
+__device__ __forceinline__ float e4m3_to_float(uint8_t b) {
+  __half_raw h = __nv_cvt_fp8_to_halfraw(static_cast<__nv_fp8_storage_t>(b), __NV_E4M3);
+  return __half2float(__half(h));
+}
+
+// Scale byte for a group with max |x| = amax: E4M3 round-to-nearest-even of
+// amax/6, saturating to 448.  amax/6 is the IEEE-rounded fp32 quotient; it
+// can only equal an E4M3 rounding midpoint when the exact quotient does
+// (the dividend has 8 significant bits, a midpoint times 6 at most 7), so
+// the decision is that of exact arithmetic.
+__device__ __forceinline__ uint8_t scale_byte_of_amax(float amax) {
+  float t = __fdiv_rn(amax, 6.0f);
+  return static_cast<uint8_t>(__nv_cvt_float_to_fp8(t, __NV_SATFINITE, __NV_E4M3));
+}
+
+// E2M1 code of x under scale s (> 0): the magnitude index is the number of
+// rounding midpoints m*s that |x| passes, with ties going to the even index
+// (strict comparison where the lower neighbour is even, >= where the upper
+// one is).  Every m*s is exact in fp32 (s has 4 significant bits, m at most
+// 3), so the comparisons are exact.  A zero magnitude gives code 0.
+__device__ __forceinline__ uint32_t e2m1_code(float x, float s) {
+  float a = fabsf(x);
+  uint32_t idx = (a > 0.25f * s) + (a >= 0.75f * s) + (a > 1.25f * s) + (a >= 1.75f * s) +
+                 (a > 2.5f * s) + (a >= 3.5f * s) + (a > 5.0f * s);
+  uint32_t sign = (__float_as_uint(x) >> 31) & 1u;
+  return idx ? (idx | (sign << 3)) : 0u;
+}
+
+// Two E2M1 codes (low nibble = first element) -> f16x2, exact.
+__device__ __forceinline__ uint32_t e2m1x2_to_f16x2(uint32_t byte) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 t;\n\tcvt.u8.u32 t, %1;\n\tcvt.rn.f16x2.e2m1x2 %0, t;\n\t}"
+      : "=r"(out)
+      : "r"(byte));
+  return out;
+}
+
+// Two E4M3 bytes (low byte = first element) -> f16x2, exact.
+__device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
+  uint32_t out;
+  uint16_t in = static_cast<uint16_t>(two_bytes);
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(out) : "h"(in));
+  return out;
+}
+
+__device__ __forceinline__ uint32_t hmul2_u32(uint32_t a, uint32_t b) {
+  __half2 r = __hmul2(*reinterpret_cast<__half2 *>(&a), *reinterpret_cast<__half2 *>(&b));
+  return *reinterpret_cast<uint32_t *>(&r);
+}
+
+__device__ __forceinline__ float2 f16x2_to_float2(uint32_t v) {
+  return __half22float2(*reinterpret_cast<__half2 *>(&v));
+}
+
+// Warp reductions.
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+}  // namespace nvkv

@@ -1,0 +1,64 @@
+"""Helpers shared by the GPU parity tests: oracle references for sampled
+output rows of a synthetic workload, and the attention tolerance."""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+import oracle
+from nvfp4_quantized_kv_b200.workload import Workload
+
+# Attention output tolerance against the float64 oracle computed on the same
+# dequantised values: |gpu - ref| <= ATOL + RTOL * |ref| element-wise.
+ATOL = 8e-3
+RTOL = 8e-3
+
+
+def oracle_outputs(wl: Workload, rows, nthreads=None):
+    """rows: list of (b, t, hq).  Returns float64 [len(rows)][D]: the exact
+    attention of query t of sequence b, head hq, over the sequence's keys
+    0 .. ctx_b + t (all rows of the workload, quantised by the oracle)."""
+    q = wl.queries()
+    G = wl.group
+    kv = {}
+    for b in sorted({r[0] for r in rows}):
+        kv[b] = wl.kv_rows(b, 0, int(wl.kv_lens[b]))
+    jobs = []
+    for b, t, hq in rows:
+        k, v = kv[b]
+        jobs.append((k, v, hq // G, wl.query_position(b, t) + 1, q[b * wl.T + t, hq]))
+    out, _, psum = oracle.attention_rows(jobs, wl.num_kv_heads, wl.head_dim, wl.sm_scale, nthreads)
+    assert np.all(np.abs(psum - 1) < 1e-9)
+    return out
+
+
+def gpu_rows(out: torch.Tensor, wl: Workload, rows) -> np.ndarray:
+    o = out.float().cpu().numpy()
+    return np.stack([o[b * wl.T + t, hq] for b, t, hq in rows]).astype(np.float64)
+
+
+def assert_close(got: np.ndarray, ref: np.ndarray, what: str):
+    err = np.abs(got - ref)
+    bound = ATOL + RTOL * np.abs(ref)
+    bad = err > bound
+    assert np.isfinite(got).all(), f"{what}: non-finite output"
+    assert not bad.any(), (f"{what}: {bad.sum()} of {bad.size} elements out of tolerance; "
+                           f"max err {err.max():.3e}, worst ratio {(err / bound).max():.2f}")
+    return float((err / bound).max())
+
+
+def all_rows(wl: Workload):
+    return [(b, t, hq) for b in range(wl.batch) for t in range(wl.T) for hq in range(wl.num_q_heads)]
+
+
+def sample_rows(wl: Workload, n: int, seed: int = 0):
+    rng = np.random.default_rng(seed)
+    rows = set()
+    # always the last query of every sequence and the first and last head
+    for b in range(wl.batch):
+        rows.add((b, wl.T - 1, 0))
+        rows.add((b, 0, wl.num_q_heads - 1))
+    while len(rows) < n:
+        rows.add((int(rng.integers(wl.batch)), int(rng.integers(wl.T)),
+                  int(rng.integers(wl.num_q_heads))))
+    return sorted(rows)

@@ -1,0 +1,148 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+include/nvkv.h declares, rejects bad arguments before launching anything,
+and its split plan covers every unit exactly once."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+import nvfp4_quantized_kv_b200 as nv
+from nvfp4_quantized_kv_b200 import build as nvbuild
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def lib():
+    nvbuild.build()
+    return nv.library()
+
+
+def declared_functions():
+    src = open(os.path.join(ROOT, "include", "nvkv.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(nvkv_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_every_declared_symbol_is_exported(lib):
+    names = declared_functions()
+    assert {"nvkv_append", "nvkv_decode_attn", "nvkv_combine", "nvkv_prefill_attn"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_page_bytes(lib):
+    assert nv.nvkv_page_bytes(4, 256) == 18432
+    assert nv.nvkv_page_bytes(2, 128) == 4608
+    assert lib.nvkv_page_bytes(0, 128) == 0 and lib.nvkv_page_bytes(2, -1) == 0
+
+
+def test_status_strings(lib):
+    for s in range(5):
+        assert nv.nvkv_status_string(s)
+    assert "unknown" in nv.nvkv_status_string(99)
+
+
+def cache(pool=0x1000, num_pages=4, hkv=2, d=128):
+    return nv._CacheC(pool, num_pages, hkv, d)
+
+
+def seqs(batch=1, maxp=4, max_len=64, pt=0x2000, lens=0x3000):
+    return nv._SeqsC(pt, maxp, lens, batch, max_len, None)
+
+
+def test_append_rejects_bad_arguments_without_launch(lib):
+    c, s = cache(), seqs()
+    f = lib.nvkv_append
+    B = ctypes.byref
+    assert f(None, B(s), 0x10, 0x20, 0x30, 1, 1, None) == nv.ERR_INVALID_ARG
+    assert f(B(c), None, 0x10, 0x20, 0x30, 1, 1, None) == nv.ERR_INVALID_ARG
+    assert f(B(cache(d=64)), B(s), 0x10, 0x20, 0x30, 1, 1, None) == nv.ERR_UNSUPPORTED
+    assert f(B(cache(pool=0x1001)), B(s), 0x10, 0x20, 0x30, 1, 1, None) == nv.ERR_INVALID_ARG
+    assert f(B(c), B(seqs(max_len=65)), 0x10, 0x20, 0x30, 1, 1, None) == nv.ERR_INVALID_ARG
+    assert f(B(c), B(s), None, 0x20, 0x30, 1, 1, None) == nv.ERR_INVALID_ARG
+    assert f(B(c), B(s), 0x18, 0x20, 0x30, 1, 1, None) == nv.ERR_INVALID_ARG  # misaligned
+    assert f(B(c), B(s), 0x10, 0x20, 0x30, -1, 1, None) == nv.ERR_INVALID_ARG
+    assert f(B(c), B(s), None, None, None, 0, 0, None) == nv.OK  # nothing to do
+
+
+def test_decode_rejects_bad_arguments_without_launch(lib):
+    c, s = cache(hkv=4, d=256), seqs()
+    f = lib.nvkv_decode_attn
+    B = ctypes.byref
+    need = lib.nvkv_decode_workspace_bytes(1, 1, 24, 4, 256, 8)
+    assert need > 0
+    assert f(B(c), B(s), 0x100, 1, 25, 0.1, 8, 0x1000, need, None) == nv.ERR_INVALID_ARG  # Hq % Hkv
+    assert f(B(c), B(s), 0x100, 17, 24, 0.1, 8, 0x1000, need, None) == nv.ERR_UNSUPPORTED  # T
+    assert f(B(c), B(s), 0x100, 6, 96, 0.1, 8, 0x1000, need, None) == nv.ERR_UNSUPPORTED  # rows
+    assert f(B(c), B(s), 0x100, 0, 24, 0.1, 8, 0x1000, need, None) == nv.ERR_INVALID_ARG
+    assert f(B(c), B(s), None, 1, 24, 0.1, 8, 0x1000, need, None) == nv.ERR_INVALID_ARG
+    assert f(B(c), B(s), 0x100, 1, 24, float("nan"), 8, 0x1000, need, None) == nv.ERR_INVALID_ARG
+    assert f(B(c), B(s), 0x100, 1, 24, 0.1, 8, None, need, None) == nv.ERR_WORKSPACE
+    assert f(B(c), B(s), 0x100, 1, 24, 0.1, 8, 0x1000, need - 1, None) == nv.ERR_WORKSPACE
+    assert f(B(c), B(s), 0x100, 1, 24, 0.1, 8, 0x1008, need, None) == nv.ERR_WORKSPACE
+
+
+def test_combine_and_prefill_reject_bad_arguments(lib):
+    B = ctypes.byref
+    s = seqs()
+    assert lib.nvkv_combine(B(s), 0x1000, 1, 24, 4, 256, 8, None, None) == nv.ERR_INVALID_ARG
+    assert lib.nvkv_combine(B(s), None, 1, 24, 4, 256, 8, 0x100, None) == nv.ERR_WORKSPACE
+    assert lib.nvkv_combine(B(s), 0x1000, 1, 24, 5, 256, 8, 0x100, None) == nv.ERR_INVALID_ARG
+    c = cache(hkv=4, d=256)
+    f = lib.nvkv_prefill_attn
+    assert f(B(c), B(s), 0x100, 0x200, 10, 10, 25, 0.1, 0x300, None) == nv.ERR_INVALID_ARG
+    assert f(B(c), B(s), None, 0x200, 10, 10, 24, 0.1, 0x300, None) == nv.ERR_INVALID_ARG
+    assert f(B(c), B(s), None, None, 0, 0, 24, 0.1, None, None) == nv.OK
+
+
+def test_workspace_size_formula(lib):
+    for batch, T, hq, hkv, d, S in [(3, 1, 24, 4, 256, 296), (64, 1, 24, 4, 256, 100),
+                                     (1, 1, 8, 2, 128, 5), (2, 4, 24, 4, 256, 1)]:
+        R = T * hq // hkv
+        slots = S + batch * hkv - 1
+        a256 = lambda x: (x + 255) // 256 * 256
+        assert lib.nvkv_decode_workspace_bytes(batch, T, hq, hkv, d, S) == \
+            a256(slots * R * d * 4) + a256(slots * R * 4)
+    assert lib.nvkv_decode_workspace_bytes(0, 1, 24, 4, 256, 8) == 0
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_split_plan_partitions_units(lib, seed):
+    """Every 128-token unit of every (b, h) pair lies in exactly one split
+    range; ranges are contiguous and balanced to within one unit; the
+    workspace slots c + b*Hkv + h written by a range are unique."""
+    rng = np.random.default_rng(seed)
+    B = int(rng.integers(1, 40))
+    hkv = int(rng.integers(1, 6))
+    lens = rng.integers(0, 5000, size=B).astype(np.int32)
+    lens[rng.random(B) < 0.2] = 0
+    S = int(rng.choice([1, 3, 7, 148, 296, 1000]))
+    first, last = nv.nvkv_split_plan(lens, hkv, S)
+    units = [(int(l) + 127) // 128 for l in lens]
+    U = sum(u * hkv for u in units)
+    begin = [c * U // S for c in range(S + 1)]
+    owner = np.full(U, -1)
+    for c in range(S):
+        owner[begin[c]:begin[c + 1]] = c
+        assert begin[c + 1] - begin[c] in (U // S, -(-U // S)) or U == 0
+    assert (owner >= 0).all() or U == 0
+    start = 0
+    slots = set()
+    for b in range(B):
+        for h in range(hkv):
+            bh = b * hkv + h
+            if units[b] == 0:
+                assert first[bh] > last[bh]
+                continue
+            touched = sorted(set(owner[start:start + units[b]]))
+            assert first[bh] == touched[0] and last[bh] == touched[-1]
+            for c in touched:
+                assert (c, bh) not in slots
+                slots.add((c, bh))
+            start += units[b]
+    used = {c + bh for c, bh in slots}
+    assert len(used) == len(slots)
+    assert max(used, default=0) <= S + B * hkv - 2

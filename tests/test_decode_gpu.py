@@ -1,0 +1,141 @@
+"""GPU parity of the split-K decode / MTP-verify attention (nvkv_decode_attn
++ nvkv_combine) against the float64 oracle, on the seeded synthetic
+workloads: all rows for small cases, sampled rows at full size.  The
+tolerance is |err| <= 8e-3 + 8e-3 |ref| (parity_util)."""
+import zlib
+
+import numpy as np
+import pytest
+import torch
+
+import nvfp4_quantized_kv_b200 as nv
+from nvfp4_quantized_kv_b200 import workload as W
+from nvfp4_quantized_kv_b200.harness import DeviceWorkload
+
+from parity_util import all_rows, assert_close, gpu_rows, oracle_outputs, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+def run_step(wl, num_splits=0):
+    dw = DeviceWorkload(wl, num_splits=num_splits)
+    dw.fill_context()
+    dw.load_step_inputs()
+    dw.step()
+    torch.cuda.synchronize()
+    assert dw.err_bits() == 0
+    return dw
+
+
+SMALL = [
+    # name, batch, hq, hkv, d, T, ctx
+    ("one_token", 1, 8, 2, 128, 1, [0]),
+    ("tail_ragged", 2, 8, 2, 128, 1, [17, 300]),
+    ("gqa6_d256", 3, 24, 4, 256, 1, [1000, 129, 5]),
+    ("mtp4_short", 2, 24, 4, 256, 4, [127, 520]),
+    ("mtp6", 1, 12, 2, 256, 6, [777]),
+    ("mha", 2, 4, 4, 128, 2, [250, 33]),
+    ("t16_g8", 1, 8, 1, 128, 16, [300]),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
+@pytest.mark.parametrize("num_splits", [0, 3])
+def test_decode_small_all_rows(case, num_splits):
+    name, b, hq, hkv, d, T, ctx = case
+    wl = W.small(name, b, hq, hkv, d, T, ctx, seed=zlib.crc32(name.encode()) % 1000)
+    dw = run_step(wl, num_splits)
+    rows = all_rows(wl)
+    assert_close(gpu_rows(dw.out, wl, rows), oracle_outputs(wl, rows), name)
+
+
+def test_tiny_decode_config():
+    wl = W.tiny_decode()
+    dw = run_step(wl)
+    rows = all_rows(wl)
+    assert_close(gpu_rows(dw.out, wl, rows), oracle_outputs(wl, rows), wl.name)
+
+
+def test_batch2_verify_config():
+    wl = W.batch2_verify()
+    dw = run_step(wl)
+    rows = sample_rows(wl, 40, seed=1)
+    assert_close(gpu_rows(dw.out, wl, rows), oracle_outputs(wl, rows), wl.name)
+
+
+def test_ragged_batch_config():
+    wl = W.ragged_batch()
+    dw = run_step(wl)
+    rows = sample_rows(wl, 48, seed=2)
+    assert_close(gpu_rows(dw.out, wl, rows), oracle_outputs(wl, rows), wl.name)
+
+
+@pytest.mark.parametrize("T", [1, 6])
+def test_long_context_config_sampled(T):
+    wl = W.long_context(T=T)
+    dw = run_step(wl)
+    rows = [(0, T - 1, 0), (1, 0, 13), (2, T - 1, 23), (2, 0, 6)]
+    assert_close(gpu_rows(dw.out, wl, rows), oracle_outputs(wl, rows), wl.name)
+
+
+def test_split_count_does_not_change_the_result():
+    """Combine metamorphic check: 1 split per pair up to more splits than
+    units give the same outputs up to bf16 rounding of the final result."""
+    wl = W.small("splits", 3, 24, 4, 256, 3, [2000, 50, 900], seed=4)
+    dw = DeviceWorkload(wl, num_splits=1)
+    dw.fill_context()
+    dw.load_step_inputs()
+    dw.append()
+    outs = []
+    for S in (1, 2, 7, 64, 296, 5000):
+        dw.num_splits = S
+        dw.workspace = torch.empty(
+            nv.nvkv_decode_workspace_bytes(wl.batch, wl.T, wl.num_q_heads, wl.num_kv_heads,
+                                           wl.head_dim, S), dtype=torch.uint8, device="cuda")
+        dw.attend()
+        torch.cuda.synchronize()
+        outs.append(dw.out.float().clone())
+    for o in outs[1:]:
+        diff = (o - outs[0]).abs()
+        assert (diff <= 2 ** -7 * outs[0].abs() + 1e-6).all(), float(diff.max())
+
+
+def test_queries_without_keys_give_zeros():
+    """kv_len < T: the first queries of the block see no key."""
+    dev = torch.device("cuda")
+    hkv, hq, d, T = 2, 4, 128, 4
+    cache = nv.Cache.allocate(2, hkv, d, dev, fill=0)
+    pt = torch.tensor([[0, 1]], dtype=torch.int32, device=dev)
+    lens = torch.tensor([2], dtype=torch.int32, device=dev)
+    seqs = nv.Seqs(pt, lens, 2)
+    rng = np.random.default_rng(0)
+    q = torch.from_numpy(rng.standard_normal((T, hq, d)).astype(np.float32)).to(dev).bfloat16()
+    S = 4
+    ws = torch.empty(nv.nvkv_decode_workspace_bytes(1, T, hq, hkv, d, S), dtype=torch.uint8,
+                     device=dev)
+    out = torch.full((T, hq, d), 7.0, dtype=torch.bfloat16, device=dev)
+    nv.nvkv_decode_attn(cache, seqs, q, T, hq, 0.1, S, ws)
+    nv.nvkv_combine(seqs, ws, T, hq, hkv, d, S, out)
+    torch.cuda.synchronize()
+    assert (out[:2] == 0).all()          # positions -2, -1: no key
+    assert torch.isfinite(out[2:]).all()  # positions 0 and 1 see the (zero) cache
+    assert (out[2:] == 0).all()           # an all-zero pool dequantises to 0
+
+
+def test_decode_reports_bad_page():
+    dev = torch.device("cuda")
+    hkv, hq, d = 2, 4, 128
+    cache = nv.Cache.allocate(2, hkv, d, dev, fill=0)
+    pt = torch.tensor([[0, 9]], dtype=torch.int32, device=dev)
+    lens = torch.tensor([20], dtype=torch.int32, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    seqs = nv.Seqs(pt, lens, 20, err)
+    q = torch.zeros((1, hq, d), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(nv.nvkv_decode_workspace_bytes(1, 1, hq, hkv, d, 2), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty((1, hq, d), dtype=torch.bfloat16, device=dev)
+    nv.nvkv_decode_attn(cache, seqs, q, 1, hq, 0.1, 2, ws)
+    nv.nvkv_combine(seqs, ws, 1, hq, hkv, d, 2, out)
+    torch.cuda.synchronize()
+    assert int(err.item()) & nv.DEVERR_PAGE_ID
+    assert torch.isfinite(out.float()).all()
