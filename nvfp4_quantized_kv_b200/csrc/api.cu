@@ -2,6 +2,8 @@
 // host-side argument checks, workspace carving and kernel dispatch.  Nothing
 // here allocates, synchronises or reads device memory.
 #include <cmath>
+#include <cstdlib>
+#include <cstring>
 
 #include "nvkv_common.cuh"
 
@@ -10,6 +12,9 @@ cudaError_t launch_append(const nvkv_cache &, const nvkv_seqs &, const void *, c
                           const int32_t *, int, int, cudaStream_t);
 cudaError_t launch_decode_simt(const nvkv_cache &, const nvkv_seqs &, const void *, int, int,
                                float, int, float *, float *, cudaStream_t);
+bool decode_tc_supported(const nvkv_cache &, int, int);
+cudaError_t launch_decode_tc(const nvkv_cache &, const nvkv_seqs &, const void *, int, int, float,
+                             int, float *, float *, cudaStream_t);
 cudaError_t launch_combine(const nvkv_seqs &, const void *, const void *, int, int, int, int, int,
                            void *, cudaStream_t);
 cudaError_t launch_prefill_simt(const nvkv_cache &, const nvkv_seqs &, const void *,
@@ -69,6 +74,13 @@ WorkspaceLayout layout(int batch, int T, int Hq, int Hkv, int D, int S) {
 
 nvkv_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NVKV_OK : NVKV_ERR_CUDA; }
 
+// NVKV_DECODE_KERNEL=simt forces the CUDA-core decode kernel (used by the
+// tests to cross-check the two kernels on the same shapes).
+bool force_simt() {
+  const char *v = std::getenv("NVKV_DECODE_KERNEL");
+  return v && std::strcmp(v, "simt") == 0;
+}
+
 }  // namespace
 
 extern "C" {
@@ -85,7 +97,7 @@ int32_t nvkv_default_num_splits(void) {
     cudaGetLastError();  // the failed query leaves a (non-sticky) error; clear it
     sms = 148;           // B200
   }
-  return 2 * sms;
+  return sms;
 }
 
 size_t nvkv_decode_workspace_bytes(int32_t batch, int32_t T, int32_t num_q_heads,
@@ -152,8 +164,12 @@ nvkv_status nvkv_decode_attn(const nvkv_cache *cache, const nvkv_seqs *seqs, con
   if (!workspace || !aligned16(workspace) || workspace_bytes < w.total) return NVKV_ERR_WORKSPACE;
   float *ws_o = static_cast<float *>(workspace);
   float *ws_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) + w.lse_off);
-  return cuda_status(launch_decode_simt(*cache, *seqs, q, T, num_q_heads, sm_scale, S, ws_o,
-                                        ws_lse, reinterpret_cast<cudaStream_t>(stream)));
+  cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
+  if (!force_simt() && decode_tc_supported(*cache, T, num_q_heads))
+    return cuda_status(
+        launch_decode_tc(*cache, *seqs, q, T, num_q_heads, sm_scale, S, ws_o, ws_lse, st_));
+  return cuda_status(
+      launch_decode_simt(*cache, *seqs, q, T, num_q_heads, sm_scale, S, ws_o, ws_lse, st_));
 }
 
 nvkv_status nvkv_combine(const nvkv_seqs *seqs, const void *workspace, int32_t T,

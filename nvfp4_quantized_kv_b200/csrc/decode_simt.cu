@@ -21,27 +21,6 @@ namespace nvkv {
 
 constexpr int kSimtWarps = 8;
 
-struct SegmentWalker {
-  // Finds the (b, h) pair and unit index holding global unit u.
-  __device__ static void locate(const int32_t *kv_lens, int B, int Hkv, int64_t u, int &b, int &h,
-                                int64_t &pair_start, int &units) {
-    int64_t acc = 0;
-    for (b = 0; b < B; ++b) {
-      int ub = units_of_len(kv_lens[b]);
-      int64_t span = (int64_t)ub * Hkv;
-      if (u < acc + span) {
-        h = (int)((u - acc) / ub);
-        pair_start = acc + (int64_t)h * ub;
-        units = ub;
-        return;
-      }
-      acc += span;
-    }
-    h = 0;
-    pair_start = acc;
-    units = 0;
-  }
-};
 
 
 // Online softmax of one query row (qr: fp32, pre-scaled to base-2 scores)
@@ -150,7 +129,7 @@ decode_simt_kernel(const uint8_t *__restrict__ pool, int num_pages, int Hkv, int
   while (u < u1) {
     int b, h, units;
     int64_t pair_start;
-    SegmentWalker::locate(kv_lens, B, Hkv, u, b, h, pair_start, units);
+    locate_pair(kv_lens, B, Hkv, u, b, h, pair_start, units);
     const int64_t seg_end = min(u1, pair_start + units);
     const int kv_len = kv_lens[b];
     const int tok_begin = (int)(u - pair_start) * kUnitTokens;

@@ -42,6 +42,27 @@ __host__ __device__ inline int units_of_len(int kv_len) {
   return kv_len > 0 ? (kv_len + kUnitTokens - 1) / kUnitTokens : 0;
 }
 
+// Finds the (b, h) pair holding global unit u of the split plan: its first
+// unit pair_start and its unit count (0 when u is past the last unit).
+__device__ inline void locate_pair(const int32_t *kv_lens, int B, int Hkv, int64_t u, int &b,
+                                   int &h, int64_t &pair_start, int &units) {
+  int64_t acc = 0;
+  for (b = 0; b < B; ++b) {
+    const int ub = units_of_len(kv_lens[b]);
+    const int64_t span = (int64_t)ub * Hkv;
+    if (u < acc + span) {
+      h = (int)((u - acc) / ub);
+      pair_start = acc + (int64_t)h * ub;
+      units = ub;
+      return;
+    }
+    acc += span;
+  }
+  h = 0;
+  pair_start = acc;
+  units = 0;
+}
+
 // ---------------------------------------------------------------------------
 // Error reporting: never trap, OR a bit into the caller's word.
 // ---------------------------------------------------------------------------

@@ -36,6 +36,9 @@ SMALL = [
     ("mtp6", 1, 12, 2, 256, 6, [777]),
     ("mha", 2, 4, 4, 128, 2, [250, 33]),
     ("t16_g8", 1, 8, 1, 128, 16, [300]),
+    ("rows80_d256", 1, 8, 1, 256, 10, [1000]),
+    ("rows96_d256", 2, 24, 4, 256, 16, [400, 130]),
+    ("many_short", 9, 24, 4, 256, 1, [1, 15, 16, 17, 127, 128, 129, 255, 256]),
 ]
 
 
@@ -139,3 +142,19 @@ def test_decode_reports_bad_page():
     torch.cuda.synchronize()
     assert int(err.item()) & nv.DEVERR_PAGE_ID
     assert torch.isfinite(out.float()).all()
+
+
+@pytest.mark.parametrize("case", [c for c in SMALL if c[4] == 256], ids=[c[0] for c in SMALL if c[4] == 256])
+def test_tensor_core_and_cuda_core_kernels_agree(case, monkeypatch):
+    """The same workload through both decode kernels (the tensor-core one is
+    the default for head_dim 256; NVKV_DECODE_KERNEL=simt forces the other):
+    both within tolerance of the oracle."""
+    name, b, hq, hkv, d, T, ctx = case
+    wl = W.small(name, b, hq, hkv, d, T, ctx, seed=zlib.crc32(name.encode()) % 1000 + 1)
+    rows = all_rows(wl)
+    ref = oracle_outputs(wl, rows)
+    for kernel in ("default", "simt"):
+        if kernel == "simt":
+            monkeypatch.setenv("NVKV_DECODE_KERNEL", "simt")
+        dw = run_step(wl)
+        assert_close(gpu_rows(dw.out, wl, rows), ref, f"{name}/{kernel}")
