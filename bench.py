@@ -157,6 +157,9 @@ def main():
                     help="reference arm: cap the sampled context (default: whole sequence 0)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--ctx", type=str, default=None,
+                    help="comma-separated cached lengths replacing 330000,420000,470000 "
+                         "(smaller cases for profiling)")
     args = ap.parse_args()
     if args.warmup < 3:
         raise SystemExit("--warmup must be >= 3")
@@ -178,7 +181,8 @@ def main():
     if world > 1:
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=300), device_id=dev)
 
-    wl = W.long_context(T=args.T)
+    ctx = tuple(int(x) for x in args.ctx.split(",")) if args.ctx else (330000, 420000, 470000)
+    wl = W.long_context(T=args.T, ctx=ctx)
     dw = DeviceWorkload(wl, dev, fill=None, num_splits=args.num_splits)
     dw.fill_context()
     dw.load_step_inputs()
@@ -292,7 +296,8 @@ def main():
             "config": {"workload": wl.name, "batch": wl.batch, "context": list(wl.ctx),
                        "T": wl.T, "q_heads": wl.num_q_heads, "kv_heads": wl.num_kv_heads,
                        "head_dim": wl.head_dim, "page_tokens": 16, "num_splits": S,
-                       "kv_bytes_per_step": kv_bytes, "l2": "inputs larger than L2 (1.4 GB pool)",
+                       "kv_bytes_per_step": kv_bytes,
+                       "l2": f"inputs larger than L2 ({kv_bytes / 1e9:.2f} GB of KV per step)",
                        "parallelism": f"replicas{world}" if world > 1 else "single-gpu"},
             "hbm_frac": value / world / peak,
             "decode_tokens_per_s": tokens_per_s,

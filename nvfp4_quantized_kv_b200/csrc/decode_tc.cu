@@ -71,7 +71,8 @@ struct Cfg {
   static constexpr int kOffAlpha = kOffM + 80 * 4;
   static constexpr int kOffL = kOffAlpha + 80 * 4;
   static constexpr int kOffFlags = kOffL + 80 * 4;     // int[4]: rescale[2], abort, pad
-  static constexpr int kOffBars = kOffFlags + 16;      // 8-byte aligned
+  static constexpr int kOffPages = kOffFlags + 16;     // int[NST][8]: staged page ids
+  static constexpr int kOffBars = kOffPages + NST * kUnitPages * 4;  // 8-byte aligned
   static constexpr int kNumBars = 2 * NST + 6;
   static constexpr int kOffTmem = kOffBars + kNumBars * 8;
   static constexpr int kSmemBytes = kOffTmem + 16 + 1024;  // + alignment slack
@@ -81,6 +82,7 @@ struct Shared {
   uint8_t *stages, *qtile, *ptile;
   float *red, *m_s, *alpha_s, *l_s;
   volatile int *flags;
+  int32_t *pages;  // [NST][8], -1 = not loaded
   uint64_t *full, *empty, *kready, *sready, *pready, *vready, *pvdone, *final_bar;
   uint32_t *tmem_slot;
 };
@@ -146,6 +148,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
   sh.alpha_s = reinterpret_cast<float *>(smem + C::kOffAlpha);
   sh.l_s = reinterpret_cast<float *>(smem + C::kOffL);
   sh.flags = reinterpret_cast<volatile int *>(smem + C::kOffFlags);
+  sh.pages = reinterpret_cast<int32_t *>(smem + C::kOffPages);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBars);
   sh.full = bars;
   sh.empty = bars + C::NST;
@@ -211,7 +214,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
             pages[p] = page_of(pt, tok0 + p * kPageTokens, sg.kv_len, num_pages);
             if (tok0 + p * kPageTokens < sg.kv_len && pages[p] < 0) report(err, NVKV_DEVERR_PAGE_ID);
             if (pages[p] >= 0) bytes += kHeadBytes;
+            sh.pages[stage * kUnitPages + p] = pages[p];
           }
+          // The arrive releases the page ids to the workers that wait on it.
           mbar_arrive_expect_tx(&sh.full[stage], bytes);
 #pragma unroll
           for (int p = 0; p < kUnitPages; ++p)
@@ -311,6 +316,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
       fence_proxy_async_smem();
 #pragma unroll
       for (int i = 0; i < NH; ++i) l_part[i] = 0.f;
+      // Keys visible to this thread's score columns n = hf*NH + i: row n is
+      // query t = n / G at position kv_len - T + t; padding rows see none.
+      int n_vis[NH];
+#pragma unroll
+      for (int i = 0; i < NH; ++i) {
+        const int n = hf * NH + i;
+        n_vis[i] = n < R ? sg.kv_len - T + n / G + 1 : 0;
+      }
 
       for (; u < sg.seg_end; ++u, ++uc) {
         const bool first = (u == seg_start);
@@ -318,20 +331,25 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
         const uint8_t *stg = sh.stages + stage * kStageBytes;
         const int tok0 = (int)(u - sg.pair_start) * kUnitTokens;
         wait_bar(&sh.full[stage], (uc / C::NST) & 1, sh.flags, err);
+        const int4 pa = *reinterpret_cast<const int4 *>(sh.pages + stage * kUnitPages);
+        const int4 pb = *reinterpret_cast<const int4 *>(sh.pages + stage * kUnitPages + 4);
+        const int pg_id[kUnitPages] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
+        const bool full_unit = tok0 + kUnitTokens <= sg.kv_len &&
+                               min(min(min(pa.x, pa.y), min(pa.z, pa.w)),
+                                   min(min(pb.x, pb.y), min(pb.z, pb.w))) >= 0;
 
         // ---- K tile: thread = token jl, d in [128*hf, 128*hf + 128) ----
         {
           const int jl = 32 * lq + lane;
           const int p = jl >> 4, slot = jl & 15;
-          const bool ok = page_of(pt, tok0 + p * kPageTokens, sg.kv_len, num_pages) >= 0 &&
-                          tok0 + jl < sg.kv_len;
+          const bool ok = full_unit ||
+                          (sh.pages[stage * kUnitPages + p] >= 0 && tok0 + jl < sg.kv_len);
           const uint8_t *pg = stg + p * kPagePitch;
-          uint32_t sc[4] = {0, 0, 0, 0};
-          if (ok) {
-            const uint4 s4 = *reinterpret_cast<const uint4 *>(
-                pg + (16 + (slot >> 3)) * 128 + (((slot & 7) ^ (slot >> 3)) << 4));
-            sc[0] = s4.x; sc[1] = s4.y; sc[2] = s4.z; sc[3] = s4.w;
-          }
+          // Scale bytes of groups 8*hf .. 8*hf+7 of this token.
+          uint2 sc = make_uint2(0u, 0u);
+          if (ok)
+            sc = *reinterpret_cast<const uint2 *>(pg + (16 + (slot >> 3)) * 128 +
+                                                  (((slot & 7) ^ (slot >> 3)) << 4) + hf * 8);
 #pragma unroll
           for (int ci = 0; ci < 4; ++ci) {
             const int cch = 4 * hf + ci;  // 16-byte chunk = 32 d = groups 2cch, 2cch+1
@@ -339,16 +357,18 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
             if (ok) {
               const uint4 w4 = *reinterpret_cast<const uint4 *>(pg + slot * 128 +
                                                                 ((cch ^ (slot & 7)) << 4));
-              const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
-              const uint32_t sword = sc[cch >> 1];
-              const uint32_t sb0 = (sword >> (16 * (cch & 1))) & 0xffu;
-              const uint32_t sb1 = (sword >> (16 * (cch & 1) + 8)) & 0xffu;
+              const uint32_t sword = ci < 2 ? sc.x : sc.y;
+              const uint32_t sb0 = (sword >> (16 * (ci & 1))) & 0xffu;
+              const uint32_t sb1 = (sword >> (16 * (ci & 1) + 8)) & 0xffu;
               const uint32_t s0 = e4m3x2_to_f16x2(sb0 | (sb0 << 8));
               const uint32_t s1 = e4m3x2_to_f16x2(sb1 | (sb1 << 8));
+              const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
 #pragma unroll
-              for (int i = 0; i < 16; ++i) {
-                const uint32_t byte = (w[i >> 2] >> (8 * (i & 3))) & 0xffu;
-                words[i] = hmul2_u32(e2m1x2_to_f16x2(byte), i < 8 ? s0 : s1);
+              for (int wi = 0; wi < 4; ++wi) {
+                uint32_t t4[4];
+                e2m1x8_to_f16x2x4(w[wi], t4);
+#pragma unroll
+                for (int k = 0; k < 4; ++k) words[4 * wi + k] = hmul2_u32(t4[k], wi < 2 ? s0 : s1);
               }
             } else {
 #pragma unroll
@@ -362,25 +382,79 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
           if (lane == 0) mbar_arrive(sh.kready);
         }
 
+        // PV of the previous unit must be done before O^T, P^T and the V^T
+        // tile are touched.
+        if (uc > 0) {
+          wait_bar(sh.pvdone, (uc - 1) & 1, sh.flags, err);
+          tc_fence_after();
+        }
+
+        // ---- V^T tile: thread = head_dim row d, 128 tokens (overlaps QK) ----
+        {
+          const int d = 128 * hf + 32 * lq + lane;
+          const int g = d >> 4;
+          const int vrow = 18 + (d >> 4);
+          const int vchunk = ((d & 15) >> 1) ^ (vrow & 7);
+          const int srow = 34 + (g >> 3);
+          const int schunk = (g & 7) ^ (srow & 7);
+#pragma unroll
+          for (int p = 0; p < kUnitPages; ++p) {
+            const int ptok = tok0 + p * kPageTokens;
+            uint32_t o8[8];
+            if (pg_id[p] >= 0) {
+              const uint8_t *pg = stg + p * kPagePitch;
+              const uint2 cw = *reinterpret_cast<const uint2 *>(pg + vrow * 128 + vchunk * 16 +
+                                                                (d & 1) * 8);
+              const uint4 s4 = *reinterpret_cast<const uint4 *>(pg + srow * 128 + schunk * 16);
+              uint32_t c0[4], c1[4], sp[8];
+              e2m1x8_to_f16x2x4(cw.x, c0);
+              e2m1x8_to_f16x2x4(cw.y, c1);
+              {
+                uint32_t t2[2];
+                e4m3x4_to_f16x2x2(s4.x, t2); sp[0] = t2[0]; sp[1] = t2[1];
+                e4m3x4_to_f16x2x2(s4.y, t2); sp[2] = t2[0]; sp[3] = t2[1];
+                e4m3x4_to_f16x2x2(s4.z, t2); sp[4] = t2[0]; sp[5] = t2[1];
+                e4m3x4_to_f16x2x2(s4.w, t2); sp[6] = t2[0]; sp[7] = t2[1];
+              }
+#pragma unroll
+              for (int i = 0; i < 8; ++i) o8[i] = hmul2_u32(i < 4 ? c0[i] : c1[i - 4], sp[i]);
+              if (!full_unit && ptok + kPageTokens > sg.kv_len) {
+#pragma unroll
+                for (int i = 0; i < 8; ++i) {
+                  const int t0 = ptok + 2 * i;
+                  if (t0 >= sg.kv_len) o8[i] = 0u;
+                  else if (t0 + 1 >= sg.kv_len) o8[i] &= 0xffffu;
+                }
+              }
+            } else {
+#pragma unroll
+              for (int i = 0; i < 8; ++i) o8[i] = 0u;
+            }
+            tmem_st8(tl + kColV + hf * 64 + 8 * p, o8);
+          }
+          tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(sh.vready);
+            mbar_arrive(&sh.empty[stage]);  // every read of the stage is done
+          }
+        }
+
         // ---- softmax on S^T: thread = token jl, columns hf*NH .. +NH ----
         wait_bar(sh.sready, uc & 1, sh.flags, err);
         tc_fence_after();
         float sv[NH];
         {
-          const int jl = 32 * lq + lane;
-          const int pos = tok0 + jl;
+          const int pos = tok0 + 32 * lq + lane;
 #pragma unroll
           for (int i8 = 0; i8 < NH / 8; ++i8) {
             uint32_t r[8];
             tmem_ld8(tl + kColS + hf * NH + i8 * 8, r);
             tmem_wait_ld();
 #pragma unroll
-            for (int j = 0; j < 8; ++j) {
-              const int n = hf * NH + i8 * 8 + j;
-              const int n_vis = sg.kv_len - T + (n / G) + 1;  // keys 0 .. n_vis-1 visible
-              const bool valid = n < R && pos < n_vis;
-              sv[i8 * 8 + j] = valid ? __uint_as_float(r[j]) : -INFINITY;
-            }
+            for (int j = 0; j < 8; ++j)
+              sv[i8 * 8 + j] = pos < n_vis[i8 * 8 + j] ? __uint_as_float(r[j]) : -INFINITY;
           }
 #pragma unroll
           for (int i = 0; i < NH; ++i) {
@@ -417,12 +491,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
           pv[i] = sv[i] > -INFINITY ? exp2f(sv[i] - mu) : 0.f;
           l_part[i] += pv[i];
         }
-        // PV of the previous unit must be done before O^T, P^T and the V^T
-        // tile are touched.
-        if (uc > 0) {
-          wait_bar(sh.pvdone, (uc - 1) & 1, sh.flags, err);
-          tc_fence_after();
-        }
         if (rescale && !first) {
           // O^T rows d = 128*hf + 32*lq + lane: column n *= alpha_n.
 #pragma unroll
@@ -457,52 +525,6 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(sh.pready);
-        }
-
-        // ---- V^T tile: thread = head_dim row d, 128 tokens ----
-        {
-          const int d = 128 * hf + 32 * lq + lane;
-          const int g = d >> 4;
-          const int vrow = 18 + (d >> 4);
-          const int vchunk = ((d & 15) >> 1) ^ (vrow & 7);
-          const int srow = 34 + (g >> 3);
-          const int schunk = (g & 7) ^ (srow & 7);
-          uint32_t words[64];
-#pragma unroll
-          for (int p = 0; p < kUnitPages; ++p) {
-            const int ptok = tok0 + p * kPageTokens;
-            const bool ok = page_of(pt, ptok, sg.kv_len, num_pages) >= 0;
-            if (ok) {
-              const uint8_t *pg = stg + p * kPagePitch;
-              const uint2 cw = *reinterpret_cast<const uint2 *>(pg + vrow * 128 + vchunk * 16 +
-                                                                (d & 1) * 8);
-              const uint4 s4 = *reinterpret_cast<const uint4 *>(pg + srow * 128 + schunk * 16);
-              const uint32_t cws[2] = {cw.x, cw.y};
-              const uint32_t sws[4] = {s4.x, s4.y, s4.z, s4.w};
-#pragma unroll
-              for (int i = 0; i < 8; ++i) {
-                const uint32_t cb = (cws[i >> 2] >> (8 * (i & 3))) & 0xffu;
-                const uint32_t s2 = e4m3x2_to_f16x2(sws[i >> 1] >> (16 * (i & 1)));
-                uint32_t w = hmul2_u32(e2m1x2_to_f16x2(cb), s2);
-                const int t0 = ptok + 2 * i;
-                if (t0 >= sg.kv_len) w = 0u;
-                else if (t0 + 1 >= sg.kv_len) w &= 0xffffu;
-                words[p * 8 + i] = w;
-              }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 8; ++i) words[p * 8 + i] = 0u;
-            }
-          }
-#pragma unroll
-          for (int j = 0; j < 4; ++j) tmem_st16(tl + kColV + hf * 64 + j * 16, words + 16 * j);
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(sh.vready);
-            mbar_arrive(&sh.empty[stage]);
-          }
         }
       }
 

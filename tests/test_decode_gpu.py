@@ -83,7 +83,11 @@ def test_long_context_config_sampled(T):
 
 def test_split_count_does_not_change_the_result():
     """Combine metamorphic check: 1 split per pair up to more splits than
-    units give the same outputs up to bf16 rounding of the final result."""
+    units.  Moving split boundaries changes the fp32 summation order and
+    which running max the f16 softmax weights are rounded against (relative
+    error up to 2^-11 per weight), so the outputs agree to the attention
+    tolerance rather than bit for bit; each is also checked against the
+    oracle by the other tests."""
     wl = W.small("splits", 3, 24, 4, 256, 3, [2000, 50, 900], seed=4)
     dw = DeviceWorkload(wl, num_splits=1)
     dw.fill_context()
@@ -100,7 +104,7 @@ def test_split_count_does_not_change_the_result():
         outs.append(dw.out.float().clone())
     for o in outs[1:]:
         diff = (o - outs[0]).abs()
-        assert (diff <= 2 ** -7 * outs[0].abs() + 1e-6).all(), float(diff.max())
+        assert (diff <= 8e-3 + 8e-3 * outs[0].abs()).all(), float(diff.max())
 
 
 def test_queries_without_keys_give_zeros():
