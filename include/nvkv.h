@@ -152,6 +152,32 @@ nvkv_status nvkv_combine(const nvkv_seqs *seqs, const void *workspace, int32_t T
                          int32_t num_q_heads, int32_t num_kv_heads, int32_t head_dim,
                          int32_t num_splits, void *out, nvkv_stream_t stream);
 
+/* Decode / MTP-verify attention without a caller workspace: the same
+ * computation as nvkv_decode_attn followed by nvkv_combine (same arguments,
+ * same q / out layouts), with the split-K partial results kept in a
+ * library-owned device array of nvkv_decode_static_scratch_bytes() bytes
+ * (8 MiB) instead of caller memory.  The pages describe no such call; it is
+ * here for callers that cannot allocate device memory where they run
+ * attention (inside a CUDA Graph capture, under an allocator they do not
+ * own, or on a path that must not take allocator locks).  It allocates and
+ * frees nothing.
+ *  - Every GPU that loads the library holds the 8 MiB array until the process
+ *    exits.
+ *  - Shapes whose nvkv_decode_workspace_bytes() exceeds the array return
+ *    NVKV_ERR_WORKSPACE without launching.
+ *  - The first call on each device (with that device current) looks up the
+ *    array's device address (cudaGetSymbolAddress) and caches it; make that
+ *    first call before any stream capture.  NVKV_ERR_CUDA if the lookup fails.
+ *  - All calls on a device share the one array, and it keeps the last call's
+ *    contents (nothing needs to start at zero).  Calls whose kernels overlap
+ *    on the GPU (different streams without ordering) race on it: order them
+ *    on one stream or with events. */
+size_t nvkv_decode_static_scratch_bytes(void);
+nvkv_status nvkv_decode_attn_static(const nvkv_cache *cache, const nvkv_seqs *seqs,
+                                    const void *q, int32_t T, int32_t num_q_heads,
+                                    float sm_scale, int32_t num_splits, void *out,
+                                    nvkv_stream_t stream);
+
 /* Chunked-prefill attention ("knoopx/ninfer" README, "Capabilities and
  * limits": chunked prefill): causal attention of a chunk of new queries
  * against the whole cache of their sequence, whose K/V rows (including the

@@ -21,7 +21,8 @@ __all__ = [
     "NvkvError", "Cache", "Seqs", "library", "library_path",
     "nvkv_page_bytes", "nvkv_default_num_splits", "nvkv_decode_workspace_bytes",
     "nvkv_split_plan", "nvkv_append", "nvkv_decode_attn", "nvkv_combine",
-    "nvkv_prefill_attn", "nvkv_status_string",
+    "nvkv_prefill_attn", "nvkv_status_string", "nvkv_decode_attn_static",
+    "nvkv_decode_static_scratch_bytes",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -71,6 +72,8 @@ def library():
             "nvkv_decode_attn": (ctypes.c_int, [cp, sp, vp, i32, i32, f32, i32, vp, sz, vp]),
             "nvkv_combine": (ctypes.c_int, [sp, vp, i32, i32, i32, i32, i32, vp, vp]),
             "nvkv_prefill_attn": (ctypes.c_int, [cp, sp, vp, vp, i32, i32, i32, f32, vp, vp]),
+            "nvkv_decode_static_scratch_bytes": (sz, []),
+            "nvkv_decode_attn_static": (ctypes.c_int, [cp, sp, vp, i32, i32, f32, i32, vp, vp]),
             "nvkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         }
         for name, (res, args) in sig.items():
@@ -208,3 +211,18 @@ def nvkv_prefill_attn(cache: Cache, seqs: Seqs, q: torch.Tensor, cu_q: torch.Ten
         ctypes.byref(cache._c), ctypes.byref(seqs._c), _dev(q, torch.bfloat16, "q"),
         _dev(cu_q, torch.int32, "cu_q"), int(total_q), int(max_q), int(num_q_heads),
         float(sm_scale), _dev(out, torch.bfloat16, "out"), _stream(stream)), "nvkv_prefill_attn")
+
+
+def nvkv_decode_static_scratch_bytes() -> int:
+    return int(library().nvkv_decode_static_scratch_bytes())
+
+
+def nvkv_decode_attn_static(cache: Cache, seqs: Seqs, q: torch.Tensor, T: int, num_q_heads: int,
+                            sm_scale: float, num_splits: int, out: torch.Tensor,
+                            stream=None) -> None:
+    """Decode attention + combine with the library's own device scratch (no
+    workspace argument, nothing allocated); see include/nvkv.h."""
+    _check(library().nvkv_decode_attn_static(
+        ctypes.byref(cache._c), ctypes.byref(seqs._c), _dev(q, torch.bfloat16, "q"), int(T),
+        int(num_q_heads), float(sm_scale), int(num_splits), _dev(out, torch.bfloat16, "out"),
+        _stream(stream)), "nvkv_decode_attn_static")
