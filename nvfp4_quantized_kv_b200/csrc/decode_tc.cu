@@ -13,20 +13,25 @@
 // Design (one CTA per split-plan range, persistent over its units):
 //  * A unit is 128 tokens = 8 pages of one (sequence, kv-head).  The TMA
 //    producer warp copies each page's 4608-byte kv-head block (36 rows of
-//    128 B) into a 4-stage shared-memory ring with one 2-D tiled load per page
-//    (128-byte swizzle, so the dequantising reads below are bank-conflict
-//    free).  No multicast.
+//    128 B) into a 4-stage shared-memory ring with one 2-D tiled load per
+//    page (128-byte swizzle: the dequantising reads are bank-conflict free).
+//    No multicast.
 //  * Swap-AB: the dequantised K tile (128 tokens x 256 d, f16) and V^T tile
 //    (2 x 128 d x 128 tokens) are the A operands, written straight from
 //    registers into Tensor Memory; the G*T query rows (Q, then P) are the
 //    small N side of the MMA, in shared memory.  S^T and O^T accumulate in
-//    Tensor Memory in fp32.  Dequantisation is exact in f16
+//    Tensor Memory in fp32, and so does the softmax denominator: one more
+//    MMA of an all-ones A tile against P^T sums P over the tokens, with the
+//    same f16 P the value sums use.  Dequantisation is exact in f16
 //    (E2M1 x E4M3 has at most 6 significant bits).
-//  * 8 worker warps dequantise (K: one token per thread; V: one head_dim row
-//    per thread), run the online softmax on S^T (one token per thread,
-//    column maxima across the 128 lanes through shared memory) and write
-//    P^T; one thread issues the MMAs.  The running max is only raised when
-//    a tile max exceeds it by more than 2^8, so O^T is rarely rescaled.
+//  * 16 dequantising warps (4 per SM sub-partition): each converts a quarter
+//    of the K tile (one token per thread, 32 d per QK phase) and of the V^T
+//    tile (one d row per thread, 64 tokens).  4 dedicated softmax warps run
+//    the softmax on S^T (one token per thread): the running max of a row is only
+//    raised when a score exceeds it by more than 2^8, which one warp vote per
+//    row detects; the full cross-lane max (and the rescale of O^T and of the
+//    denominator) runs only then -- on the first unit of a segment and rarely
+//    after.  One thread issues the MMAs.
 //  * Every wait is bounded; a timeout sets NVKV_DEVERR_TIMEOUT, turns all
 //    later waits into no-ops and lets the kernel drain and free its Tensor
 //    Memory.
@@ -44,46 +49,66 @@ constexpr int kHeadBytes = 18 * kD;   // 4608
 constexpr int kPagePitch = 5120;      // staged page pitch (1024-aligned)
 constexpr int kUnitPages = 8;
 constexpr int kStageBytes = kUnitPages * kPagePitch;
-constexpr int kWorkerWarps = 8;
-constexpr int kProducerWarp = 8;
-constexpr int kMmaWarp = 9;
-constexpr int kThreads = 320;
+constexpr int kStages = 4;
+constexpr int kWorkerWarps = 16;      // dequantising warps 0..15
+constexpr int kSoftmaxWarps = 4;      // softmax warps 16..19
+constexpr int kSoftmaxWarp0 = 16;
+constexpr int kProducerWarp = 20;
+constexpr int kMmaWarp = 21;
+constexpr int kThreads = 22 * 32;
+constexpr int kSegThreads = (kWorkerWarps + kSoftmaxWarps) * 32;  // segment-end barrier
 constexpr uint32_t kTmemCols = 512;
 constexpr long long kWaitBudget = 2000000000LL;  // clock cycles (~1 s)
 constexpr float kLazyRescale = 8.0f;             // log2 units
 
-constexpr uint32_t kColK = 0;    // 128 columns: K tile (token lanes, d pairs)
-constexpr uint32_t kColV = 128;  // 2 x 64 columns: V^T halves (d lanes, token pairs)
-constexpr uint32_t kColS = 256;  // N columns: S^T; then O^T halves of N columns each
+// Tensor Memory columns.  The K tile is dequantised in two head_dim halves
+// (64 columns each, one QK phase per half); the V^T tile, S^T and the P^T tile
+// are double-buffered by unit parity, so the QK of unit u+1 and the
+// dequantisation of unit u+1 overlap the softmax and PV of unit u.  When
+// N <= 32 the two K halves also get their own columns, so the first half of
+// unit u+1 only waits for the first QK phase of unit u.
+constexpr uint32_t kColK = 0;      // K half of phase A (and B when N > 32)
 
 template <int N>
 struct Cfg {
-  static constexpr int NH = N / 2;               // S^T columns per worker warp
-  static constexpr int NST = N <= 64 ? 4 : 3;    // pipeline stages
-  static constexpr uint32_t kColO = kColS + N;
-  static constexpr int kQBytes = N * kD * 2;     // Q tile, K-major, no swizzle
-  static constexpr int kPBytes = N * 128 * 2;    // P^T tile, MN-major, no swizzle
-  static constexpr int kRedFloats = kWorkerWarps * 40;
-  static constexpr int kOffQ = NST * kStageBytes;
-  static constexpr int kOffP = kOffQ + kQBytes;
-  static constexpr int kOffRed = kOffP + kPBytes;
-  static constexpr int kOffM = kOffRed + kRedFloats * 4;
-  static constexpr int kOffAlpha = kOffM + 80 * 4;
-  static constexpr int kOffL = kOffAlpha + 80 * 4;
-  static constexpr int kOffFlags = kOffL + 80 * 4;     // int[4]: rescale[2], abort, pad
-  static constexpr int kOffPages = kOffFlags + 16;     // int[NST][8]: staged page ids
-  static constexpr int kOffBars = kOffPages + NST * kUnitPages * 4;  // 8-byte aligned
-  static constexpr int kNumBars = 2 * NST + 6;
+  static constexpr bool kSplitK = N <= 32;
+  static constexpr uint32_t kColKB = kSplitK ? 64 : 0;       // K half of phase B
+  static constexpr uint32_t kColV = kSplitK ? 128 : 64;      // 2 slots x 128: V^T
+  static constexpr uint32_t kColS = kColV + 256;             // 2 slots x N: S^T
+  static constexpr uint32_t kColO = kColS + 2 * N;           // O^T half hf at kColO + hf*N
+  static_assert(N % 16 == 0 && N >= 16 && N <= 48 && kColO + 2 * N <= kTmemCols, "N");
+  static constexpr int kMaskWords = (N + 31) / 32;
+  static constexpr int kQBytes = N * kD * 2;        // Q tile, K-major, no swizzle
+  static constexpr int kPBytes = N * 128 * 2;       // one P^T tile, MN-major, no swizzle
+  static constexpr int kOffQ = kStages * kStageBytes;
+  static constexpr int kOffP = kOffQ + kQBytes;                 // 2 P^T tiles
+  static constexpr int kOffRed = kOffP + 2 * kPBytes;           // float [4][N]
+  static constexpr int kOffMask = kOffRed + kSoftmaxWarps * N * 4;  // u32 [2][4][4]
+  static constexpr int kOffM = kOffMask + 2 * kSoftmaxWarps * 4 * 4;
+  static constexpr int kOffAlpha = kOffM + N * 4;
+  static constexpr int kOffNvis = kOffAlpha + N * 4;
+  static constexpr int kOffFlags = kOffNvis + N * 4;            // int[4]: abort at [2]
+  static constexpr int kOffPages = kOffFlags + 16;              // int[stages][8]
+  static constexpr int kOffBars = kOffPages + kStages * kUnitPages * 4;
+  static constexpr int kNumBars = 2 * kStages + 12;
   static constexpr int kOffTmem = kOffBars + kNumBars * 8;
-  static constexpr int kSmemBytes = kOffTmem + 16 + 1024;  // + alignment slack
+  static constexpr int kSmemBytes = kOffTmem + 16 + 1024;      // + alignment slack
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+  static_assert(kOffQ % 1024 == 0 && kOffP % 16 == 0 && kPBytes % 16 == 0 &&
+                kOffPages % 16 == 0 && kOffBars % 8 == 0, "alignment");
 };
 
 struct Shared {
   uint8_t *stages, *qtile, *ptile;
-  float *red, *m_s, *alpha_s, *l_s;
+  float *red, *m_s, *alpha_s;
+  int32_t *nvis_s, *pages;
+  uint32_t *masks;
   volatile int *flags;
-  int32_t *pages;  // [NST][8], -1 = not loaded
-  uint64_t *full, *empty, *kready, *sready, *pready, *vready, *pvdone, *final_bar;
+  // sready, pready, vready and pvdone exist once per S^T / P^T / V^T slot:
+  // slot s completes once per unit with (unit & 1) == s, so no wait is ever
+  // more than one phase behind (a parity wait cannot tell phases two apart).
+  uint64_t *full, *empty, *kready_a, *kdone_a, *kready_b, *sready, *pready, *vready, *pvdone,
+      *final_bar;
   uint32_t *tmem_slot;
 };
 
@@ -128,6 +153,10 @@ __device__ __forceinline__ int page_of(const int32_t *pt_row, int tok, int kv_le
   return (p >= 0 && p < num_pages) ? p : -1;
 }
 
+__device__ __forceinline__ uint32_t dup_scale(uint32_t byte) {
+  return e4m3x2_to_f16x2(byte | (byte << 8));
+}
+
 template <int N>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hkv,
@@ -144,20 +173,23 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
   sh.qtile = smem + C::kOffQ;
   sh.ptile = smem + C::kOffP;
   sh.red = reinterpret_cast<float *>(smem + C::kOffRed);
+  sh.masks = reinterpret_cast<uint32_t *>(smem + C::kOffMask);
   sh.m_s = reinterpret_cast<float *>(smem + C::kOffM);
   sh.alpha_s = reinterpret_cast<float *>(smem + C::kOffAlpha);
-  sh.l_s = reinterpret_cast<float *>(smem + C::kOffL);
+  sh.nvis_s = reinterpret_cast<int32_t *>(smem + C::kOffNvis);
   sh.flags = reinterpret_cast<volatile int *>(smem + C::kOffFlags);
   sh.pages = reinterpret_cast<int32_t *>(smem + C::kOffPages);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + C::kOffBars);
   sh.full = bars;
-  sh.empty = bars + C::NST;
-  sh.kready = bars + 2 * C::NST;
-  sh.sready = sh.kready + 1;
-  sh.pready = sh.kready + 2;
-  sh.vready = sh.kready + 3;
-  sh.pvdone = sh.kready + 4;
-  sh.final_bar = sh.kready + 5;
+  sh.empty = bars + kStages;
+  sh.kready_a = bars + 2 * kStages;
+  sh.kdone_a = sh.kready_a + 1;
+  sh.kready_b = sh.kready_a + 2;
+  sh.sready = sh.kready_a + 3;  // [2]
+  sh.pready = sh.kready_a + 5;  // [2]
+  sh.vready = sh.kready_a + 7;  // [2]
+  sh.pvdone = sh.kready_a + 9;  // [2]
+  sh.final_bar = sh.kready_a + 11;
   sh.tmem_slot = reinterpret_cast<uint32_t *>(smem + C::kOffTmem);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -165,20 +197,25 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
   const int R = T * G;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < C::NST; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(&sh.full[i], 1);
       mbar_init(&sh.empty[i], kWorkerWarps);
     }
-    mbar_init(sh.kready, kWorkerWarps);
-    mbar_init(sh.sready, 1);
-    mbar_init(sh.pready, kWorkerWarps);
-    mbar_init(sh.vready, kWorkerWarps);
-    mbar_init(sh.pvdone, 1);
+    mbar_init(sh.kready_a, kWorkerWarps);
+    mbar_init(sh.kdone_a, 1);
+    mbar_init(sh.kready_b, kWorkerWarps);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sh.sready[i], 1);
+      mbar_init(&sh.pready[i], kSoftmaxWarps);
+    }
+    mbar_init(&sh.vready[0], kWorkerWarps);
+    mbar_init(&sh.vready[1], kWorkerWarps);
+    mbar_init(&sh.pvdone[0], 1);
+    mbar_init(&sh.pvdone[1], 1);
     mbar_init(sh.final_bar, 1);
     fence_mbar_init();
   }
   if (threadIdx.x < 4) sh.flags[threadIdx.x] = 0;
-  if (threadIdx.x < 80) sh.m_s[threadIdx.x] = -INFINITY;
   if (warp == kMmaWarp) {
     tmem_alloc(sh.tmem_slot, kTmemCols);
     tmem_relinquish();
@@ -196,80 +233,122 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ TMA
-    if (lane == 0) {
-      prefetch_tmap(&tmap);
-      uint32_t uc = 0;
-      for (int64_t u = u0; u < u1;) {
-        const Seg sg = segment_at(u, u1, kv_lens, B, Hkv, max_kv_len, max_pages);
-        const int32_t *pt = page_table + (size_t)sg.b * max_pages;
-        for (; u < sg.seg_end; ++u, ++uc) {
-          const int stage = uc % C::NST;
-          if (uc >= (uint32_t)C::NST)
-            wait_bar(&sh.empty[stage], ((uc / C::NST) + 1) & 1, sh.flags, err);
-          const int tok0 = (int)(u - sg.pair_start) * kUnitTokens;
-          int pages[kUnitPages];
-          uint32_t bytes = 0;
-#pragma unroll
-          for (int p = 0; p < kUnitPages; ++p) {
-            pages[p] = page_of(pt, tok0 + p * kPageTokens, sg.kv_len, num_pages);
-            if (tok0 + p * kPageTokens < sg.kv_len && pages[p] < 0) report(err, NVKV_DEVERR_PAGE_ID);
-            if (pages[p] >= 0) bytes += kHeadBytes;
-            sh.pages[stage * kUnitPages + p] = pages[p];
-          }
-          // The arrive releases the page ids to the workers that wait on it.
-          mbar_arrive_expect_tx(&sh.full[stage], bytes);
-#pragma unroll
-          for (int p = 0; p < kUnitPages; ++p)
-            if (pages[p] >= 0)
-              tma_load_2d(sh.stages + stage * kStageBytes + p * kPagePitch, &tmap, 0,
-                          (pages[p] * Hkv + sg.h) * kRowsPerHead, &sh.full[stage]);
-        }
+    // The whole warp produces: lane p < 8 owns page p of a unit.  The page
+    // ids of unit u+1 are loaded while unit u's copies are issued, so the
+    // page-table latency is off the critical path.
+    prefetch_tmap(&tmap);
+    const int p = lane & 7;
+    int64_t u = u0;
+    Seg sg = segment_at(u, u1, kv_lens, B, Hkv, max_kv_len, max_pages);
+    auto page_for = [&](const Seg &g, int64_t uu) -> int {
+      const int tok = (int)(uu - g.pair_start) * kUnitTokens + p * kPageTokens;
+      const int32_t *pt = page_table + (size_t)g.b * max_pages;
+      const int pg = page_of(pt, tok, g.kv_len, num_pages);
+      if (lane < kUnitPages && tok < g.kv_len && pg < 0) report(err, NVKV_DEVERR_PAGE_ID);
+      return pg;
+    };
+    int cur = u < u1 ? page_for(sg, u) : -1;
+    uint32_t uc = 0;
+    for (; u < u1; ++u, ++uc) {
+      const int stage = uc % kStages;
+      // Next unit's page id (possibly in the next segment).
+      int nxt = -1;
+      Seg nsg = sg;
+      if (u + 1 < u1) {
+        if (u + 1 >= sg.seg_end) nsg = segment_at(u + 1, u1, kv_lens, B, Hkv, max_kv_len, max_pages);
+        nxt = page_for(nsg, u + 1);
       }
-      // Drain: every issued copy must land before the CTA may exit.
-      const uint32_t first = uc > (uint32_t)C::NST ? uc - C::NST : 0;
-      for (uint32_t k = first; k < uc; ++k)
-        mbar_wait(&sh.full[k % C::NST], (k / C::NST) & 1, kWaitBudget);
+      if (uc >= (uint32_t)kStages) {
+        if (lane == 0) wait_bar(&sh.empty[stage], ((uc / kStages) + 1) & 1, sh.flags, err);
+        __syncwarp();
+      }
+      const bool mine = lane < kUnitPages && cur >= 0;
+      if (lane < kUnitPages) sh.pages[stage * kUnitPages + lane] = cur;
+      const uint32_t bytes = __popc(__ballot_sync(0xffffffffu, mine)) * kHeadBytes;
+      __syncwarp();
+      // The arrive releases the page ids to the workers that wait on it.
+      if (lane == 0) mbar_arrive_expect_tx(&sh.full[stage], bytes);
+      __syncwarp();
+      if (mine)
+        tma_load_2d(sh.stages + stage * kStageBytes + lane * kPagePitch, &tmap, 0,
+                    (cur * Hkv + sg.h) * kRowsPerHead, &sh.full[stage]);
+      cur = nxt;
+      sg = nsg;
     }
+    // Drain: every issued copy must land before the CTA may exit.
+    if (lane == 0) {
+      const uint32_t first = uc > (uint32_t)kStages ? uc - kStages : 0;
+      for (uint32_t k = first; k < uc; ++k)
+        mbar_wait(&sh.full[k % kStages], (k / kStages) & 1, kWaitBudget);
+    }
+    __syncwarp();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA
+    // Software-pipelined: the QK of unit u is issued before the PV of unit
+    // u-1, so the softmax of a unit overlaps the next unit's QK.  At a segment
+    // boundary the pending PV is issued first (the workers wait for it before
+    // they load the next pair's queries).
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_f16_f32(128, N, false, false);
       const uint32_t idesc_pv = idesc_f16_f32(128, N, false, true);
       const uint32_t qb = smem_u32(sh.qtile), pb = smem_u32(sh.ptile);
-      uint32_t uc = 0;
       bool issued = false;
+      bool pend = false, pend_first = false;  // a PV waiting to be issued
+      uint32_t pend_uc = 0;
+      auto issue_pv = [&]() {
+        const uint32_t puc = pend_uc;
+        const bool ok_v = wait_bar(&sh.vready[puc & 1], (puc >> 1) & 1, sh.flags, err);
+        const bool ok_p = wait_bar(&sh.pready[puc & 1], (puc >> 1) & 1, sh.flags, err);
+        if (ok_p && ok_v) {
+          tc_fence_after();
+          const uint32_t pslot = pb + (puc & 1) * C::kPBytes;
+          const uint32_t vslot = tmem + C::kColV + (puc & 1) * 128;
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t bd = smem_desc(pslot + ks * 256, 128, 2048);
+            const uint32_t acc = (!pend_first) || ks > 0;
+            mma_f16_ts(tmem + C::kColO, vslot + ks * 8, bd, idesc_pv, acc);
+            mma_f16_ts(tmem + C::kColO + N, vslot + 64 + ks * 8, bd, idesc_pv, acc);
+          }
+          issued = true;
+        }
+        mma_commit(&sh.pvdone[puc & 1]);
+        pend = false;
+      };
+      uint32_t uc = 0;
       for (int64_t u = u0; u < u1;) {
         const Seg sg = segment_at(u, u1, kv_lens, B, Hkv, max_kv_len, max_pages);
         const int64_t seg_start = u;
+        if (pend) issue_pv();  // drain at the segment boundary
         for (; u < sg.seg_end; ++u, ++uc) {
-          const bool first = (u == seg_start);
-          if (wait_bar(sh.kready, uc & 1, sh.flags, err)) {
+          const uint32_t sslot = tmem + C::kColS + (uc & 1) * N;
+          // QK, phase A: head_dim 0..127 (K slices 0..7), phase B: 128..255.
+          if (wait_bar(sh.kready_a, uc & 1, sh.flags, err)) {
             tc_fence_after();
 #pragma unroll
-            for (int ks = 0; ks < kD / 16; ++ks) {
+            for (int ks = 0; ks < 8; ++ks) {
               const uint64_t bd = smem_desc(qb + ks * 2 * (N * 16), N * 16, 128);
-              mma_f16_ts(tmem + kColS, tmem + kColK + ks * 8, bd, idesc_qk, ks > 0);
+              mma_f16_ts(sslot, tmem + kColK + ks * 8, bd, idesc_qk, ks > 0);
             }
             issued = true;
           }
-          mma_commit(sh.sready);
-          const bool ok_p = wait_bar(sh.pready, uc & 1, sh.flags, err);
-          const bool ok_v = wait_bar(sh.vready, uc & 1, sh.flags, err);
-          if (ok_p && ok_v) {
+          mma_commit(sh.kdone_a);
+          if (wait_bar(sh.kready_b, uc & 1, sh.flags, err)) {
             tc_fence_after();
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf)
-#pragma unroll
-              for (int ks = 0; ks < 8; ++ks) {
-                const uint64_t bd = smem_desc(pb + ks * 256, 128, 2048);
-                mma_f16_ts(tmem + C::kColO + hf * N, tmem + kColV + hf * 64 + ks * 8, bd,
-                           idesc_pv, (!first) || ks > 0);
-              }
-            issued = true;
+            for (int ks = 8; ks < 16; ++ks) {
+              const uint64_t bd = smem_desc(qb + ks * 2 * (N * 16), N * 16, 128);
+              mma_f16_ts(sslot, tmem + C::kColKB + (ks - 8) * 8, bd, idesc_qk, 1u);
+            }
           }
-          mma_commit(sh.pvdone);
+          mma_commit(&sh.sready[uc & 1]);
+          if (pend) issue_pv();
+          pend = true;
+          pend_uc = uc;
+          pend_first = (u == seg_start);
         }
       }
+      if (pend) issue_pv();
       if (issued) {
         mma_commit(sh.final_bar);
         mbar_wait(sh.final_bar, 0, kWaitBudget);
@@ -277,23 +356,28 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
     }
   } else {
     // -------------------------------------------------------------- workers
-    const int lq = warp & 3, hf = warp >> 2;
-    const uint32_t lane_base = (uint32_t)(32 * lq) << 16;
-    const uint32_t tl = tmem + lane_base;  // this warp's lane quarter
-    const int tid = threadIdx.x;           // 0..255
-    constexpr int NH = C::NH;
-    float l_part[NH];
+    const bool smx = warp >= kSoftmaxWarp0;                    // softmax warps 16..19
+    const int lq = warp & 3, sub = smx ? 0 : warp >> 2;
+    const uint32_t tl = tmem + ((uint32_t)(32 * lq) << 16);  // this warp's lane quarter
+    const int tid = smx ? threadIdx.x - kSoftmaxWarp0 * 32 : threadIdx.x;  // 0..127 / 0..511
+    // Per-token partial softmax denominators (softmax threads): the sums of
+    // the same f16 weights the PV MMAs use.
+    float l_part[N];
+#pragma unroll
+    for (int i = 0; i < N; ++i) l_part[i] = 0.f;
+
     uint32_t uc = 0;
     for (int64_t u = u0; u < u1;) {
       const Seg sg = segment_at(u, u1, kv_lens, B, Hkv, max_kv_len, max_pages);
       if (sg.bad && tid == 0) report(err, NVKV_DEVERR_LENGTH);
-      const int32_t *pt = page_table + (size_t)sg.b * max_pages;
       const int64_t seg_start = u;
       const size_t slot = (size_t)c + (size_t)sg.b * Hkv + sg.h;
 
       // Q tile of this pair: rows n < R are (t, g) = (n / G, n % G), pre-scaled
       // to base-2 scores, f16, K-major core-matrix layout; rows >= R are zero.
-      for (int ci = tid; ci < N * (kD / 8); ci += kWorkerWarps * 32) {
+      // (The previous segment's QK MMAs completed: every worker waited for
+      // its last PV, which follows them.)
+      for (int ci = smx ? N * (kD / 8) : tid; ci < N * (kD / 8); ci += kWorkerWarps * 32) {
         const int n = ci / (kD / 8), k8 = ci % (kD / 8);
         uint4 v = make_uint4(0, 0, 0, 0);
         if (n < R) {
@@ -314,260 +398,365 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
         *reinterpret_cast<uint4 *>(sh.qtile + k8 * (N * 16) + (n >> 3) * 128 + (n & 7) * 16) = v;
       }
       fence_proxy_async_smem();
+      if (smx) {
+        if (tid < N) {
+          // Keys visible to score row n (query t = n / G at kv_len - T + t).
+          sh.nvis_s[tid] = tid < R ? sg.kv_len - T + tid / G + 1 : 0;
+          sh.m_s[tid] = -INFINITY;
+        }
 #pragma unroll
-      for (int i = 0; i < NH; ++i) l_part[i] = 0.f;
-      // Keys visible to this thread's score columns n = hf*NH + i: row n is
-      // query t = n / G at position kv_len - T + t; padding rows see none.
-      int n_vis[NH];
-#pragma unroll
-      for (int i = 0; i < NH; ++i) {
-        const int n = hf * NH + i;
-        n_vis[i] = n < R ? sg.kv_len - T + n / G + 1 : 0;
+        for (int i = 0; i < N; ++i) l_part[i] = 0.f;
+        named_barrier(1, kSoftmaxWarps * 32);
       }
 
       for (; u < sg.seg_end; ++u, ++uc) {
         const bool first = (u == seg_start);
-        const int stage = uc % C::NST;
+        const int stage = uc % kStages;
         const uint8_t *stg = sh.stages + stage * kStageBytes;
         const int tok0 = (int)(u - sg.pair_start) * kUnitTokens;
-        wait_bar(&sh.full[stage], (uc / C::NST) & 1, sh.flags, err);
-        const int4 pa = *reinterpret_cast<const int4 *>(sh.pages + stage * kUnitPages);
-        const int4 pb = *reinterpret_cast<const int4 *>(sh.pages + stage * kUnitPages + 4);
-        const int pg_id[kUnitPages] = {pa.x, pa.y, pa.z, pa.w, pb.x, pb.y, pb.z, pb.w};
-        const bool full_unit = tok0 + kUnitTokens <= sg.kv_len &&
-                               min(min(min(pa.x, pa.y), min(pa.z, pa.w)),
-                                   min(min(pb.x, pb.y), min(pb.z, pb.w))) >= 0;
+        if (!smx) {
+          wait_bar(&sh.full[stage], (uc / kStages) & 1, sh.flags, err);
+          const int4 pa = *reinterpret_cast<const int4 *>(sh.pages + stage * kUnitPages);
+          const int4 pb4 = *reinterpret_cast<const int4 *>(sh.pages + stage * kUnitPages + 4);
+          const bool full_unit = tok0 + kUnitTokens <= sg.kv_len &&
+                                 min(min(min(pa.x, pa.y), min(pa.z, pa.w)),
+                                     min(min(pb4.x, pb4.y), min(pb4.z, pb4.w))) >= 0;
 
-        // ---- K tile: thread = token jl, d in [128*hf, 128*hf + 128) ----
-        {
+          // K tile half (phase 0: d 0..127, phase 1: d 128..255): thread = token
+          // jl, one 16-byte chunk (32 d, two scale groups) per warp.
           const int jl = 32 * lq + lane;
-          const int p = jl >> 4, slot = jl & 15;
-          const bool ok = full_unit ||
-                          (sh.pages[stage * kUnitPages + p] >= 0 && tok0 + jl < sg.kv_len);
-          const uint8_t *pg = stg + p * kPagePitch;
-          // Scale bytes of groups 8*hf .. 8*hf+7 of this token.
-          uint2 sc = make_uint2(0u, 0u);
-          if (ok)
-            sc = *reinterpret_cast<const uint2 *>(pg + (16 + (slot >> 3)) * 128 +
-                                                  (((slot & 7) ^ (slot >> 3)) << 4) + hf * 8);
-#pragma unroll
-          for (int ci = 0; ci < 4; ++ci) {
-            const int cch = 4 * hf + ci;  // 16-byte chunk = 32 d = groups 2cch, 2cch+1
+          const int kp = jl >> 4, kslot = jl & 15;
+          const bool kok = full_unit ||
+                           (sh.pages[stage * kUnitPages + kp] >= 0 && tok0 + jl < sg.kv_len);
+          const uint8_t *kpg = stg + kp * kPagePitch;
+          // Scale bytes of the chunk's two groups: 2*sub, 2*sub+1 (phase 0) and
+          // 8 + 2*sub, 8 + 2*sub + 1 (phase 1); 2-byte loads at 2-byte offsets.
+          uint32_t ksc = 0, ksc1 = 0;
+          if (kok) {
+            const uint8_t *sp = kpg + (16 + (kslot >> 3)) * 128 + (((kslot & 7) ^ (kslot >> 3)) << 4);
+            ksc = *reinterpret_cast<const uint16_t *>(sp + 2 * sub);
+            ksc1 = *reinterpret_cast<const uint16_t *>(sp + 8 + 2 * sub);
+          }
+          auto k_half = [&](int phase) {
+            const int cch = 4 * phase + sub;  // chunk = 32 d = groups 2cch, 2cch+1
+            const uint32_t scw = phase ? ksc1 : ksc;
             uint32_t words[16];
-            if (ok) {
-              const uint4 w4 = *reinterpret_cast<const uint4 *>(pg + slot * 128 +
-                                                                ((cch ^ (slot & 7)) << 4));
-              const uint32_t sword = ci < 2 ? sc.x : sc.y;
-              const uint32_t sb0 = (sword >> (16 * (ci & 1))) & 0xffu;
-              const uint32_t sb1 = (sword >> (16 * (ci & 1) + 8)) & 0xffu;
-              const uint32_t s0 = e4m3x2_to_f16x2(sb0 | (sb0 << 8));
-              const uint32_t s1 = e4m3x2_to_f16x2(sb1 | (sb1 << 8));
+            if (kok) {
+              const uint4 w4 = *reinterpret_cast<const uint4 *>(kpg + kslot * 128 +
+                                                                ((cch ^ (kslot & 7)) << 4));
+              const uint32_t s0 = dup_scale(scw & 0xffu);
+              const uint32_t s1 = dup_scale((scw >> 8) & 0xffu);
               const uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
+  #pragma unroll
               for (int wi = 0; wi < 4; ++wi) {
                 uint32_t t4[4];
                 e2m1x8_to_f16x2x4(w[wi], t4);
-#pragma unroll
+  #pragma unroll
                 for (int k = 0; k < 4; ++k) words[4 * wi + k] = hmul2_u32(t4[k], wi < 2 ? s0 : s1);
               }
             } else {
-#pragma unroll
+  #pragma unroll
               for (int i = 0; i < 16; ++i) words[i] = 0u;
             }
-            tmem_st16(tl + kColK + hf * 64 + ci * 16, words);
+            tmem_st16(tl + (phase ? C::kColKB : kColK) + 16 * sub, words);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+          };
+
+          // A K half may only be rewritten once the QK phase reading it has
+          // completed: phase A of unit uc-1 (split halves) or phase B of uc-1.
+          if (uc > 0) {
+            if (C::kSplitK)
+              wait_bar(sh.kdone_a, (uc - 1) & 1, sh.flags, err);
+            else
+              wait_bar(&sh.sready[(uc - 1) & 1], ((uc - 1) >> 1) & 1, sh.flags, err);
+            tc_fence_after();
           }
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(sh.kready);
-        }
+          k_half(0);
+          if (lane == 0) mbar_arrive(sh.kready_a);
 
-        // PV of the previous unit must be done before O^T, P^T and the V^T
-        // tile are touched.
-        if (uc > 0) {
-          wait_bar(sh.pvdone, (uc - 1) & 1, sh.flags, err);
-          tc_fence_after();
-        }
-
-        // ---- V^T tile: thread = head_dim row d, 128 tokens (overlaps QK) ----
-        {
-          const int d = 128 * hf + 32 * lq + lane;
-          const int g = d >> 4;
-          const int vrow = 18 + (d >> 4);
-          const int vchunk = ((d & 15) >> 1) ^ (vrow & 7);
-          const int srow = 34 + (g >> 3);
-          const int schunk = (g & 7) ^ (srow & 7);
-#pragma unroll
-          for (int p = 0; p < kUnitPages; ++p) {
-            const int ptok = tok0 + p * kPageTokens;
-            uint32_t o8[8];
-            if (pg_id[p] >= 0) {
-              const uint8_t *pg = stg + p * kPagePitch;
-              const uint2 cw = *reinterpret_cast<const uint2 *>(pg + vrow * 128 + vchunk * 16 +
-                                                                (d & 1) * 8);
-              const uint4 s4 = *reinterpret_cast<const uint4 *>(pg + srow * 128 + schunk * 16);
-              uint32_t c0[4], c1[4], sp[8];
-              e2m1x8_to_f16x2x4(cw.x, c0);
-              e2m1x8_to_f16x2x4(cw.y, c1);
-              {
-                uint32_t t2[2];
-                e4m3x4_to_f16x2x2(s4.x, t2); sp[0] = t2[0]; sp[1] = t2[1];
-                e4m3x4_to_f16x2x2(s4.y, t2); sp[2] = t2[0]; sp[3] = t2[1];
-                e4m3x4_to_f16x2x2(s4.z, t2); sp[4] = t2[0]; sp[5] = t2[1];
-                e4m3x4_to_f16x2x2(s4.w, t2); sp[6] = t2[0]; sp[7] = t2[1];
-              }
-#pragma unroll
-              for (int i = 0; i < 8; ++i) o8[i] = hmul2_u32(i < 4 ? c0[i] : c1[i - 4], sp[i]);
-              if (!full_unit && ptok + kPageTokens > sg.kv_len) {
-#pragma unroll
-                for (int i = 0; i < 8; ++i) {
-                  const int t0 = ptok + 2 * i;
-                  if (t0 >= sg.kv_len) o8[i] = 0u;
-                  else if (t0 + 1 >= sg.kv_len) o8[i] &= 0xffffu;
+          // ---- V^T tile into slot uc&1: thread = head_dim row d, 4 pages ----
+          // The slot was last read by the PV of unit uc-2.
+          if (uc > 1) {
+            wait_bar(&sh.pvdone[uc & 1], ((uc >> 1) + 1) & 1, sh.flags, err);  // PV of uc-2
+            tc_fence_after();
+          }
+          {
+            const int hv = sub & 1;
+            const int d = 128 * hv + 32 * lq + lane;
+            const int g = d >> 4;
+            const int vrow = 18 + (d >> 4);
+            const int vchunk = ((d & 15) >> 1) ^ (vrow & 7);
+            const int srow = 34 + (g >> 3);
+            const int schunk = (g & 7) ^ (srow & 7);
+            const uint32_t vcol = C::kColV + (uc & 1) * 128 + 64 * hv;
+  #pragma unroll
+            for (int pp = 0; pp < 4; ++pp) {
+              const int p = 4 * (sub >> 1) + pp;
+              const int ptok = tok0 + p * kPageTokens;
+              uint32_t o8[8];
+              if (full_unit || sh.pages[stage * kUnitPages + p] >= 0) {
+                const uint8_t *pg = stg + p * kPagePitch;
+                const uint2 cw = *reinterpret_cast<const uint2 *>(pg + vrow * 128 + vchunk * 16 +
+                                                                  (d & 1) * 8);
+                const uint4 s4 = *reinterpret_cast<const uint4 *>(pg + srow * 128 + schunk * 16);
+                uint32_t c0[4], c1[4], sp[8];
+                e2m1x8_to_f16x2x4(cw.x, c0);
+                e2m1x8_to_f16x2x4(cw.y, c1);
+                {
+                  uint32_t t2[2];
+                  e4m3x4_to_f16x2x2(s4.x, t2); sp[0] = t2[0]; sp[1] = t2[1];
+                  e4m3x4_to_f16x2x2(s4.y, t2); sp[2] = t2[0]; sp[3] = t2[1];
+                  e4m3x4_to_f16x2x2(s4.z, t2); sp[4] = t2[0]; sp[5] = t2[1];
+                  e4m3x4_to_f16x2x2(s4.w, t2); sp[6] = t2[0]; sp[7] = t2[1];
                 }
+  #pragma unroll
+                for (int i = 0; i < 8; ++i) o8[i] = hmul2_u32(i < 4 ? c0[i] : c1[i - 4], sp[i]);
+                if (!full_unit && ptok + kPageTokens > sg.kv_len) {
+  #pragma unroll
+                  for (int i = 0; i < 8; ++i) {
+                    const int t0 = ptok + 2 * i;
+                    if (t0 >= sg.kv_len) o8[i] = 0u;
+                    else if (t0 + 1 >= sg.kv_len) o8[i] &= 0xffffu;
+                  }
+                }
+              } else {
+  #pragma unroll
+                for (int i = 0; i < 8; ++i) o8[i] = 0u;
               }
-            } else {
-#pragma unroll
-              for (int i = 0; i < 8; ++i) o8[i] = 0u;
+              tmem_st8(tl + vcol + 8 * p, o8);
             }
-            tmem_st8(tl + kColV + hf * 64 + 8 * p, o8);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.vready[uc & 1]);
           }
-          tmem_wait_st();
-          tc_fence_before();
-          __syncwarp();
+
+          // Second K half, once phase A's MMAs are done with the first.
+          if (C::kSplitK) {
+            if (uc > 0) wait_bar(&sh.sready[(uc - 1) & 1], ((uc - 1) >> 1) & 1, sh.flags, err);
+          } else {
+            wait_bar(sh.kdone_a, uc & 1, sh.flags, err);
+          }
+          tc_fence_after();
+          k_half(1);
           if (lane == 0) {
-            mbar_arrive(sh.vready);
+            mbar_arrive(sh.kready_b);
             mbar_arrive(&sh.empty[stage]);  // every read of the stage is done
           }
         }
-
-        // ---- softmax on S^T: thread = token jl, columns hf*NH .. +NH ----
-        wait_bar(sh.sready, uc & 1, sh.flags, err);
-        tc_fence_after();
-        float sv[NH];
-        {
+        if (smx) {
+          // ---- softmax on S^T slot uc&1: thread = token tok0 + 32*lq + lane ----
+          wait_bar(&sh.sready[uc & 1], (uc >> 1) & 1, sh.flags, err);
+          tc_fence_after();
           const int pos = tok0 + 32 * lq + lane;
-#pragma unroll
-          for (int i8 = 0; i8 < NH / 8; ++i8) {
-            uint32_t r[8];
-            tmem_ld8(tl + kColS + hf * NH + i8 * 8, r);
+          const bool vis_all = tok0 + kUnitTokens <= sg.kv_len - T + 1;
+          const uint32_t sslot = tl + C::kColS + (uc & 1) * N;
+          uint32_t *my_mask = sh.masks + ((uc & 1) * kSoftmaxWarps + lq) * 4;
+          // Scores of one 16-row chunk, masked: invisible keys and padding
+          // rows (n >= R) become -inf.  Branch-free over the 16 rows.
+          auto load_chunk = [&](int c16, float (&x)[16]) {
+            uint32_t r[16];
+            tmem_ld16(sslot + 16 * c16, r);
             tmem_wait_ld();
+            int nv[16];
+            if (vis_all) {
 #pragma unroll
-            for (int j = 0; j < 8; ++j)
-              sv[i8 * 8 + j] = pos < n_vis[i8 * 8 + j] ? __uint_as_float(r[j]) : -INFINITY;
-          }
+              for (int j = 0; j < 16; ++j) nv[j] = 16 * c16 + j < R ? 0x7fffffff : 0;
+            } else {
 #pragma unroll
-          for (int i = 0; i < NH; ++i) {
-            const float mx = warp_max(sv[i]);
-            if (lane == 0) sh.red[warp * 40 + i] = mx;
-          }
-        }
-        named_barrier(1, kWorkerWarps * 32);
-        if (tid < N) {
-          const int n = tid, hn = n / NH, i = n % NH;
-          float tmax = -INFINITY;
-#pragma unroll
-          for (int w = 0; w < 4; ++w) tmax = fmaxf(tmax, sh.red[(w + 4 * hn) * 40 + i]);
-          const float m_old = sh.m_s[n];
-          float alpha = 1.f;
-          if (tmax > -INFINITY && (m_old == -INFINITY || tmax > m_old + kLazyRescale)) {
-            alpha = exp2f(m_old - tmax);  // 0 when m_old = -inf
-            sh.m_s[n] = tmax;
-            sh.alpha_s[n] = alpha;
-            sh.flags[uc & 1] = 1;
-          } else {
-            sh.alpha_s[n] = 1.f;
-          }
-        }
-        if (tid == 0) sh.flags[(uc + 1) & 1] = 0;
-        named_barrier(1, kWorkerWarps * 32);
-        const bool rescale = sh.flags[uc & 1] != 0;
-        float pv[NH];
-#pragma unroll
-        for (int i = 0; i < NH; ++i) {
-          const int n = hf * NH + i;
-          const float mu = sh.m_s[n];
-          if (rescale) l_part[i] *= sh.alpha_s[n];
-          pv[i] = sv[i] > -INFINITY ? exp2f(sv[i] - mu) : 0.f;
-          l_part[i] += pv[i];
-        }
-        if (rescale && !first) {
-          // O^T rows d = 128*hf + 32*lq + lane: column n *= alpha_n.
-#pragma unroll
-          for (int j8 = 0; j8 < N / 8; ++j8) {
-            uint32_t r[8];
-            const uint32_t addr = tl + C::kColO + hf * N + j8 * 8;
-            tmem_ld8(addr, r);
-            tmem_wait_ld();
-#pragma unroll
-            for (int j = 0; j < 8; ++j)
-              r[j] = __float_as_uint(__uint_as_float(r[j]) * sh.alpha_s[j8 * 8 + j]);
-            tmem_st8(addr, r);
-          }
-          tmem_wait_st();
-        }
-        {
-          // P^T (MN-major): element (n, k) at (n/8)*2048 + (k/8)*128 + (k%8)*16 + (n%8)*2.
-          const int k = 32 * lq + lane;
-#pragma unroll
-          for (int j = 0; j < NH / 8; ++j) {
-            uint32_t h2[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              __half2 hh = __floats2half2_rn(pv[8 * j + 2 * e], pv[8 * j + 2 * e + 1]);
-              h2[e] = *reinterpret_cast<uint32_t *>(&hh);
+              for (int j4 = 0; j4 < 4; ++j4) {
+                const int4 v = *reinterpret_cast<const int4 *>(sh.nvis_s + 16 * c16 + 4 * j4);
+                nv[4 * j4] = v.x; nv[4 * j4 + 1] = v.y; nv[4 * j4 + 2] = v.z; nv[4 * j4 + 3] = v.w;
+              }
             }
-            const int n8 = (hf * NH) / 8 + j;
-            *reinterpret_cast<uint4 *>(sh.ptile + n8 * 2048 + (k >> 3) * 128 + (k & 7) * 16) =
-                make_uint4(h2[0], h2[1], h2[2], h2[3]);
+#pragma unroll
+            for (int j = 0; j < 16; ++j) x[j] = pos < nv[j] ? __uint_as_float(r[j]) : -INFINITY;
+          };
+          auto load_m = [&](int c16, float (&m)[16]) {
+#pragma unroll
+            for (int j4 = 0; j4 < 4; ++j4) {
+              const float4 v = *reinterpret_cast<const float4 *>(sh.m_s + 16 * c16 + 4 * j4);
+              m[4 * j4] = v.x; m[4 * j4 + 1] = v.y; m[4 * j4 + 2] = v.z; m[4 * j4 + 3] = v.w;
+            }
+          };
+          // One pass: weights against the current running max, kept in
+          // registers while the 4 softmax warps agree whether any score rose
+          // more than 2^8 above its row's running max (then the max is raised,
+          // the accumulators are rescaled and the weights recomputed).
+          uint32_t h2[N / 2];
+          bool up = false;
+#pragma unroll
+          for (int c16 = 0; c16 < N / 16; ++c16) {
+            if (16 * c16 < R) {
+              float x[16], m[16];
+              load_chunk(c16, x);
+              load_m(c16, m);
+#pragma unroll
+              for (int e = 0; e < 8; ++e) {
+                const float d0 = x[2 * e] - m[2 * e], d1 = x[2 * e + 1] - m[2 * e + 1];
+                up |= (d0 > kLazyRescale) | (d1 > kLazyRescale);
+                __half2 hv2 = __floats2half2_rn(exp2f(d0), exp2f(d1));  // exp2(-inf) = 0
+                h2[8 * c16 + e] = *reinterpret_cast<uint32_t *>(&hv2);
+              }
+            } else {
+#pragma unroll
+              for (int e = 0; e < 8; ++e) h2[8 * c16 + e] = 0u;
+            }
+          }
+          const uint32_t wup = __ballot_sync(0xffffffffu, up);
+          if (lane == 0) my_mask[0] = wup;
+          named_barrier(1, kSoftmaxWarps * 32);
+          uint32_t any = 0;
+#pragma unroll
+          for (int w = 0; w < kSoftmaxWarps; ++w) any |= sh.masks[((uc & 1) * kSoftmaxWarps + w) * 4];
+          if (any) {
+            // Slow path (the first unit of a segment and rare max raises):
+            // exact row maxima, new running max, rescale factor of everything
+            // accumulated against the old max, weights recomputed.
+#pragma unroll
+            for (int c16 = 0; c16 < N / 16; ++c16) {
+              if (16 * c16 < R) {
+                float x[16];
+                load_chunk(c16, x);
+#pragma unroll
+                for (int j = 0; j < 16; ++j) {
+                  const float wm = warp_max(x[j]);
+                  if (lane == 0) sh.red[lq * N + 16 * c16 + j] = wm;
+                }
+              }
+            }
+            named_barrier(1, kSoftmaxWarps * 32);
+            if (tid < N) {
+              const int n = tid;
+              float alpha = 1.f;
+              if (n < R) {
+                float tmax = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < kSoftmaxWarps; ++w) tmax = fmaxf(tmax, sh.red[w * N + n]);
+                const float m_old = sh.m_s[n];
+                if (tmax > -INFINITY && (m_old == -INFINITY || tmax > m_old + kLazyRescale)) {
+                  alpha = exp2f(m_old - tmax);  // 0 when the old max was -inf
+                  sh.m_s[n] = tmax;
+                }
+              }
+              sh.alpha_s[n] = alpha;
+            }
+            named_barrier(1, kSoftmaxWarps * 32);
+#pragma unroll
+            for (int n = 0; n < N; ++n) l_part[n] *= sh.alpha_s[n];
+            if (!first) {
+              // O^T rows d = 32*lq + lane and d + 128, accumulated up to the
+              // previous unit, scale by alpha once that unit's PV has finished.
+              wait_bar(&sh.pvdone[(uc - 1) & 1], ((uc - 1) >> 1) & 1, sh.flags, err);
+              tc_fence_after();
+#pragma unroll
+              for (int reg = 0; reg < 2; ++reg) {
+                const uint32_t base = C::kColO + reg * N;
+#pragma unroll
+                for (int j8 = 0; j8 < N / 8; ++j8) {
+                  uint32_t r[8];
+                  tmem_ld8(tl + base + j8 * 8, r);
+                  tmem_wait_ld();
+#pragma unroll
+                  for (int j = 0; j < 8; ++j)
+                    r[j] = __float_as_uint(__uint_as_float(r[j]) * sh.alpha_s[j8 * 8 + j]);
+                  tmem_st8(tl + base + j8 * 8, r);
+                }
+              }
+              tmem_wait_st();
+            }
+#pragma unroll
+            for (int c16 = 0; c16 < N / 16; ++c16) {
+              if (16 * c16 < R) {
+                float x[16], m[16];
+                load_chunk(c16, x);
+                load_m(c16, m);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) {
+                  __half2 hv2 = __floats2half2_rn(exp2f(x[2 * e] - m[2 * e]),
+                                                  exp2f(x[2 * e + 1] - m[2 * e + 1]));
+                  h2[8 * c16 + e] = *reinterpret_cast<uint32_t *>(&hv2);
+                }
+              }
+            }
+          }
+          // P^T into slot uc&1 (MN-major): element (n, k) at
+          // (n/8)*2048 + (k/8)*128 + (k%8)*16 + (n%8)*2; masked rows are 0.
+          // The slot was last read by the PV of unit uc-2.
+          if (uc > 1) {
+            wait_bar(&sh.pvdone[uc & 1], ((uc >> 1) + 1) & 1, sh.flags, err);
+            tc_fence_after();
+          }
+          const int k = 32 * lq + lane;
+          uint8_t *ptile = sh.ptile + (uc & 1) * C::kPBytes;
+#pragma unroll
+          for (int c16 = 0; c16 < N / 16; ++c16) {
+            uint8_t *dst = ptile + (2 * c16) * 2048 + (k >> 3) * 128 + (k & 7) * 16;
+            *reinterpret_cast<uint4 *>(dst) =
+                make_uint4(h2[8 * c16], h2[8 * c16 + 1], h2[8 * c16 + 2], h2[8 * c16 + 3]);
+            *reinterpret_cast<uint4 *>(dst + 2048) =
+                make_uint4(h2[8 * c16 + 4], h2[8 * c16 + 5], h2[8 * c16 + 6], h2[8 * c16 + 7]);
+            // the denominator sums the same f16 weights the PV uses
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float2 back = __half22float2(*reinterpret_cast<const __half2 *>(&h2[8 * c16 + e]));
+              l_part[16 * c16 + 2 * e] += back.x;
+              l_part[16 * c16 + 2 * e + 1] += back.y;
+            }
           }
           fence_proxy_async_smem();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) mbar_arrive(sh.pready);
+          if (lane == 0) mbar_arrive(&sh.pready[uc & 1]);
         }
       }
 
-      // ---- end of segment: l totals, then O^T / l -> workspace ----
+      // ---- end of segment: O^T / l -> workspace, lse ----
       if (uc > 0) {
-        wait_bar(sh.pvdone, (uc - 1) & 1, sh.flags, err);
+        wait_bar(&sh.pvdone[(uc - 1) & 1], ((uc - 1) >> 1) & 1, sh.flags, err);  // last PV
         tc_fence_after();
       }
-#pragma unroll
-      for (int i = 0; i < NH; ++i) {
-        const float ls = warp_sum(l_part[i]);
-        if (lane == 0) sh.red[warp * 40 + i] = ls;
-      }
-      named_barrier(1, kWorkerWarps * 32);
-      if (tid < N) {
-        const int n = tid, hn = n / NH, i = n % NH;
-        float l = 0.f;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) l += sh.red[(w + 4 * hn) * 40 + i];
-        sh.l_s[n] = l;
-        if (n < R) ws_lse[slot * R + n] = l > 0.f ? sh.m_s[n] + log2f(l) : -INFINITY;
-      }
-      named_barrier(1, kWorkerWarps * 32);
       {
-        const int d = 128 * hf + 32 * lq + lane;
+        // Denominators from the softmax threads' partial sums -> sh.alpha_s.
+        if (smx) {
 #pragma unroll
-        for (int j8 = 0; j8 < N / 8; ++j8) {
-          uint32_t r[8];
-          tmem_ld8(tl + C::kColO + hf * N + j8 * 8, r);
+          for (int n = 0; n < N; ++n) {
+            const float ls = warp_sum(l_part[n]);
+            if (lane == 0) sh.red[lq * N + n] = ls;
+          }
+        }
+        named_barrier(2, kSegThreads);
+        if (smx && tid < N) {
+          float l = 0.f;
+#pragma unroll
+          for (int w = 0; w < kSoftmaxWarps; ++w) l += sh.red[w * N + tid];
+          sh.alpha_s[tid] = l;
+        }
+        named_barrier(2, kSegThreads);
+      }
+      if (!smx) {
+        const int hv = sub & 1, cb = (sub >> 1) * (N / 2);  // O half, first column
+        const int d = 128 * hv + 32 * lq + lane;
+#pragma unroll
+        for (int j8 = 0; j8 < N / 16; ++j8) {
+          uint32_t o[8];
+          tmem_ld8(tl + C::kColO + hv * N + cb + j8 * 8, o);
           tmem_wait_ld();
 #pragma unroll
           for (int j = 0; j < 8; ++j) {
-            const int n = j8 * 8 + j;
+            const int n = cb + j8 * 8 + j;
             if (n < R) {
-              const float l = sh.l_s[n];
-              ws_o[(slot * R + n) * kD + d] = l > 0.f ? __uint_as_float(r[j]) / l : 0.f;
+              const float lv = sh.alpha_s[n];
+              ws_o[(slot * R + n) * kD + d] = lv > 0.f ? __uint_as_float(o[j]) / lv : 0.f;
+              if (d == 0) ws_lse[slot * R + n] = lv > 0.f ? sh.m_s[n] + log2f(lv) : -INFINITY;
             }
           }
         }
       }
       tc_fence_before();
-      named_barrier(1, kWorkerWarps * 32);
-      if (tid < N) sh.m_s[tid] = -INFINITY;
+      named_barrier(2, kSegThreads);
     }
   }
 
@@ -615,7 +804,7 @@ cudaError_t launch_n(const CUtensorMap &map, const nvkv_cache &c, const nvkv_seq
 // True when the tensor-core decode kernel takes this shape.
 bool decode_tc_supported(const nvkv_cache &c, int T, int Hq) {
   const int R = T * (Hq / c.num_kv_heads);
-  return c.head_dim == kD && R >= 1 && R <= 80 && encode_fn() != nullptr;
+  return c.head_dim == kD && R >= 1 && R <= 48 && encode_fn() != nullptr;
 }
 
 cudaError_t launch_decode_tc(const nvkv_cache &c, const nvkv_seqs &s, const void *q, int T,
@@ -639,9 +828,7 @@ cudaError_t launch_decode_tc(const nvkv_cache &c, const nvkv_seqs &s, const void
   const float qscale = sm_scale * 1.4426950408889634f;
   if (R <= 16) return launch_n<16>(map, c, s, q, T, Hq, qscale, S, ws_o, ws_lse, stream);
   if (R <= 32) return launch_n<32>(map, c, s, q, T, Hq, qscale, S, ws_o, ws_lse, stream);
-  if (R <= 48) return launch_n<48>(map, c, s, q, T, Hq, qscale, S, ws_o, ws_lse, stream);
-  if (R <= 64) return launch_n<64>(map, c, s, q, T, Hq, qscale, S, ws_o, ws_lse, stream);
-  return launch_n<80>(map, c, s, q, T, Hq, qscale, S, ws_o, ws_lse, stream);
+  return launch_n<48>(map, c, s, q, T, Hq, qscale, S, ws_o, ws_lse, stream);
 }
 
 }  // namespace nvkv
