@@ -284,71 +284,83 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
     __syncwarp();
   } else if (warp == kMmaWarp) {
     // ------------------------------------------------------------------ MMA
-    // Software-pipelined: the QK of unit u is issued before the PV of unit
-    // u-1, so the softmax of a unit overlaps the next unit's QK.  At a segment
-    // boundary the pending PV is issued first (the workers wait for it before
-    // they load the next pair's queries).
+    // Event driven: the issuing thread polls the ready barriers without
+    // blocking and issues whichever step is ready, the oldest PV first (it
+    // frees a V^T and a P^T slot).  Unit qk's QK needs its S^T slot, last read
+    // by the softmax of unit qk-2, so it waits until that unit's PV (issued
+    // after the softmax's arrival) has been issued.  Segment boundaries need
+    // no special case: the workers load a new pair's queries only after its
+    // previous pair's last PV completed.
     if (lane == 0) {
       const uint32_t idesc_qk = idesc_f16_f32(128, N, false, false);
       const uint32_t idesc_pv = idesc_f16_f32(128, N, false, true);
       const uint32_t qb = smem_u32(sh.qtile), pb = smem_u32(sh.ptile);
+      const uint32_t n_units = (uint32_t)(u1 - u0);
+      uint32_t qk = 0, pv = 0;
+      int qk_phase = 0;
+      uint32_t first_bits = 0;  // bit (unit & 31): unit starts its segment
+      int64_t u = u0;
+      Seg sg = segment_at(u, u1, kv_lens, B, Hkv, max_kv_len, max_pages);
+      int64_t seg_start = u;
       bool issued = false;
-      bool pend = false, pend_first = false;  // a PV waiting to be issued
-      uint32_t pend_uc = 0;
-      auto issue_pv = [&]() {
-        const uint32_t puc = pend_uc;
-        const bool ok_v = wait_bar(&sh.vready[puc & 1], (puc >> 1) & 1, sh.flags, err);
-        const bool ok_p = wait_bar(&sh.pready[puc & 1], (puc >> 1) & 1, sh.flags, err);
-        if (ok_p && ok_v) {
+      long long t_last = clock64();
+      while (pv < n_units && !sh.flags[2]) {
+        bool progress = false;
+        if (pv < qk && mbar_test(&sh.vready[pv & 1], (pv >> 1) & 1) &&
+            mbar_test(&sh.pready[pv & 1], (pv >> 1) & 1)) {
           tc_fence_after();
-          const uint32_t pslot = pb + (puc & 1) * C::kPBytes;
-          const uint32_t vslot = tmem + C::kColV + (puc & 1) * 128;
+          const bool first = (first_bits >> (pv & 31)) & 1u;
+          const uint32_t pslot = pb + (pv & 1) * C::kPBytes;
+          const uint32_t vslot = tmem + C::kColV + (pv & 1) * 128;
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
             const uint64_t bd = smem_desc(pslot + ks * 256, 128, 2048);
-            const uint32_t acc = (!pend_first) || ks > 0;
+            const uint32_t acc = (!first) || ks > 0;
             mma_f16_ts(tmem + C::kColO, vslot + ks * 8, bd, idesc_pv, acc);
             mma_f16_ts(tmem + C::kColO + N, vslot + 64 + ks * 8, bd, idesc_pv, acc);
           }
-          issued = true;
-        }
-        mma_commit(&sh.pvdone[puc & 1]);
-        pend = false;
-      };
-      uint32_t uc = 0;
-      for (int64_t u = u0; u < u1;) {
-        const Seg sg = segment_at(u, u1, kv_lens, B, Hkv, max_kv_len, max_pages);
-        const int64_t seg_start = u;
-        if (pend) issue_pv();  // drain at the segment boundary
-        for (; u < sg.seg_end; ++u, ++uc) {
-          const uint32_t sslot = tmem + C::kColS + (uc & 1) * N;
-          // QK, phase A: head_dim 0..127 (K slices 0..7), phase B: 128..255.
-          if (wait_bar(sh.kready_a, uc & 1, sh.flags, err)) {
-            tc_fence_after();
+          mma_commit(&sh.pvdone[pv & 1]);
+          ++pv;
+          progress = issued = true;
+        } else if (qk_phase == 0 && qk < n_units && qk < pv + 2 &&
+                   mbar_test(sh.kready_a, qk & 1)) {
+          tc_fence_after();
+          if (u >= sg.seg_end) {
+            sg = segment_at(u, u1, kv_lens, B, Hkv, max_kv_len, max_pages);
+            seg_start = u;
+          }
+          if (u == seg_start) first_bits |= 1u << (qk & 31);
+          else first_bits &= ~(1u << (qk & 31));
+          const uint32_t sslot = tmem + C::kColS + (qk & 1) * N;
 #pragma unroll
-            for (int ks = 0; ks < 8; ++ks) {
-              const uint64_t bd = smem_desc(qb + ks * 2 * (N * 16), N * 16, 128);
-              mma_f16_ts(sslot, tmem + kColK + ks * 8, bd, idesc_qk, ks > 0);
-            }
-            issued = true;
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t bd = smem_desc(qb + ks * 2 * (N * 16), N * 16, 128);
+            mma_f16_ts(sslot, tmem + kColK + ks * 8, bd, idesc_qk, ks > 0);
           }
           mma_commit(sh.kdone_a);
-          if (wait_bar(sh.kready_b, uc & 1, sh.flags, err)) {
-            tc_fence_after();
+          qk_phase = 1;
+          progress = issued = true;
+        } else if (qk_phase == 1 && mbar_test(sh.kready_b, qk & 1)) {
+          tc_fence_after();
+          const uint32_t sslot = tmem + C::kColS + (qk & 1) * N;
 #pragma unroll
-            for (int ks = 8; ks < 16; ++ks) {
-              const uint64_t bd = smem_desc(qb + ks * 2 * (N * 16), N * 16, 128);
-              mma_f16_ts(sslot, tmem + C::kColKB + (ks - 8) * 8, bd, idesc_qk, 1u);
-            }
+          for (int ks = 8; ks < 16; ++ks) {
+            const uint64_t bd = smem_desc(qb + ks * 2 * (N * 16), N * 16, 128);
+            mma_f16_ts(sslot, tmem + C::kColKB + (ks - 8) * 8, bd, idesc_qk, 1u);
           }
-          mma_commit(&sh.sready[uc & 1]);
-          if (pend) issue_pv();
-          pend = true;
-          pend_uc = uc;
-          pend_first = (u == seg_start);
+          mma_commit(&sh.sready[qk & 1]);
+          qk_phase = 0;
+          ++qk;
+          ++u;
+          progress = true;
+        }
+        if (progress) {
+          t_last = clock64();
+        } else if (clock64() - t_last > kWaitBudget) {
+          sh.flags[2] = 1;
+          report(err, NVKV_DEVERR_TIMEOUT);
         }
       }
-      if (pend) issue_pv();
       if (issued) {
         mma_commit(sh.final_bar);
         mbar_wait(sh.final_bar, 0, kWaitBudget);
