@@ -42,6 +42,15 @@ METRIC = "NVFP4 KV-read GB/s (% of HBM peak) and decode tokens/s at 3x~470k ctx"
 FALLBACK_HBM_GBS = 6650.0
 
 
+def bf16_peak():
+    """Dense 16-bit tensor-core peak (f16 and bf16 MMAs run at the same rate)."""
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            return float(json.load(f)["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
 def hbm_peak():
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
@@ -157,6 +166,7 @@ def main():
                     help="reference arm: cap the sampled context (default: whole sequence 0)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--no-prefill", action="store_true", help="skip the chunked-prefill line")
     ap.add_argument("--ctx", type=str, default=None,
                     help="comma-separated cached lengths replacing 330000,420000,470000 "
                          "(smaller cases for profiling)")
@@ -282,6 +292,37 @@ def main():
     h2d = h_k.numel() * 2 + h_v.numel() * 2 + h_q.numel() * 2
     d2h = h_out.numel() * 2
 
+    # ---- chunked prefill (65536 cached + 2048 new tokens), tensor-core kernel ----
+    prefill = None
+    if not args.no_prefill:
+        del dw
+        torch.cuda.empty_cache()
+        pw = W.chunked_prefill()
+        pdw = DeviceWorkload(pw, dev, fill=None)
+        pdw.fill_context()
+        pdw.load_step_inputs()
+        pdw.append(stream)
+        for _ in range(3):
+            pdw.attend(stream)
+        pe0 = torch.cuda.Event(enable_timing=True)
+        pe1 = torch.cuda.Event(enable_timing=True)
+        torch.cuda.synchronize(dev)
+        pe0.record(stream)
+        reps = 10
+        for _ in range(reps):
+            pdw.attend(stream)
+        pe1.record(stream)
+        torch.cuda.synchronize(dev)
+        p_ms = pe0.elapsed_time(pe1) / reps
+        pairs = sum(int(pw.ctx[0]) + i + 1 for i in range(pw.T))  # causal (query, key) pairs
+        flops = 4.0 * pw.head_dim * pw.num_q_heads * pairs
+        tf_peak, tf_kind = bf16_peak()
+        prefill = {"workload": pw.name, "ms": p_ms, "tflops": flops / (p_ms * 1e-3) / 1e12,
+                   "flop_per_call": flops, "bound": "tensor", "peak_tflops": tf_peak,
+                   "peak_kind": tf_kind, "frac": flops / (p_ms * 1e-3) / 1e12 / tf_peak,
+                   "device_errors": pdw.err_bits()}
+        del pdw
+
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         v, dt, threads, desc = oracle_sample(wl)
@@ -310,6 +351,7 @@ def main():
             "gpu_launches": 3 * K,
             "clocks": clk,
             "device_errors": err,
+            "prefill": prefill,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)

@@ -15,6 +15,9 @@ cudaError_t launch_decode_simt(const nvkv_cache &, const nvkv_seqs &, const void
 bool decode_tc_supported(const nvkv_cache &, int, int);
 cudaError_t launch_decode_tc(const nvkv_cache &, const nvkv_seqs &, const void *, int, int, float,
                              int, float *, float *, cudaStream_t);
+bool prefill_tc_supported(const nvkv_cache &);
+cudaError_t launch_prefill_tc(const nvkv_cache &, const nvkv_seqs &, const void *, const int32_t *,
+                              int, int, int, float, void *, cudaStream_t);
 cudaError_t launch_combine(const nvkv_seqs &, const void *, const void *, int, int, int, int, int,
                            void *, cudaStream_t);
 cudaError_t launch_prefill_simt(const nvkv_cache &, const nvkv_seqs &, const void *,
@@ -74,8 +77,9 @@ WorkspaceLayout layout(int batch, int T, int Hq, int Hkv, int D, int S) {
 
 nvkv_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NVKV_OK : NVKV_ERR_CUDA; }
 
-// NVKV_DECODE_KERNEL=simt forces the CUDA-core decode kernel (used by the
-// tests to cross-check the two kernels on the same shapes).
+// NVKV_DECODE_KERNEL=simt forces the CUDA-core decode and prefill kernels
+// (used by the tests to cross-check the two kernel families on the same
+// shapes).
 bool force_simt() {
   const char *v = std::getenv("NVKV_DECODE_KERNEL");
   return v && std::strcmp(v, "simt") == 0;
@@ -198,8 +202,12 @@ nvkv_status nvkv_prefill_attn(const nvkv_cache *cache, const nvkv_seqs *seqs, co
   if (total_q < 0 || max_q < 0 || !std::isfinite(sm_scale)) return NVKV_ERR_INVALID_ARG;
   if (total_q == 0) return NVKV_OK;
   if (!q || !cu_q || !out || !aligned16(q) || !aligned16(out)) return NVKV_ERR_INVALID_ARG;
-  return cuda_status(launch_prefill_simt(*cache, *seqs, q, cu_q, total_q, num_q_heads, sm_scale,
-                                         out, reinterpret_cast<cudaStream_t>(stream)));
+  cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
+  if (!force_simt() && prefill_tc_supported(*cache))
+    return cuda_status(launch_prefill_tc(*cache, *seqs, q, cu_q, total_q, max_q, num_q_heads,
+                                         sm_scale, out, st_));
+  return cuda_status(
+      launch_prefill_simt(*cache, *seqs, q, cu_q, total_q, num_q_heads, sm_scale, out, st_));
 }
 
 const char *nvkv_status_string(nvkv_status status) {

@@ -819,23 +819,26 @@ bool decode_tc_supported(const nvkv_cache &c, int T, int Hq) {
   return c.head_dim == kD && R >= 1 && R <= 48 && encode_fn() != nullptr;
 }
 
-cudaError_t launch_decode_tc(const nvkv_cache &c, const nvkv_seqs &s, const void *q, int T,
-                             int Hq, float sm_scale, int S, float *ws_o, float *ws_lse,
-                             cudaStream_t stream) {
+// The pool as a 2-D byte tensor of 128-byte rows; one 36-row box is one
+// page's kv-head block (head_dim 256).  Shared with the prefill kernel.
+bool make_pool_tmap(const nvkv_cache &c, CUtensorMap *map) {
   EncodeTiledFn enc = encode_fn();
-  if (!enc) return cudaErrorNotSupported;
-  // The pool as a 2-D byte tensor of 128-byte rows; one box = one page's
-  // kv-head block (36 rows).
-  CUtensorMap map;
+  if (!enc) return false;
   const cuuint64_t rows = (cuuint64_t)c.num_pages * c.num_kv_heads * kRowsPerHead;
   const cuuint64_t dims[2] = {128, rows};
   const cuuint64_t strides[1] = {128};
   const cuuint32_t box[2] = {128, kRowsPerHead};
   const cuuint32_t estr[2] = {1, 1};
-  CUresult r = enc(&map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, c.pool, dims, strides, box, estr,
-                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-  if (r != CUDA_SUCCESS) return cudaErrorInvalidValue;
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, c.pool, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+cudaError_t launch_decode_tc(const nvkv_cache &c, const nvkv_seqs &s, const void *q, int T,
+                             int Hq, float sm_scale, int S, float *ws_o, float *ws_lse,
+                             cudaStream_t stream) {
+  CUtensorMap map;
+  if (!make_pool_tmap(c, &map)) return cudaErrorNotSupported;
   const int R = T * (Hq / c.num_kv_heads);
   const float qscale = sm_scale * 1.4426950408889634f;
   if (R <= 16) return launch_n<16>(map, c, s, q, T, Hq, qscale, S, ws_o, ws_lse, stream);

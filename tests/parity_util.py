@@ -52,6 +52,9 @@ def all_rows(wl: Workload):
 
 
 def sample_rows(wl: Workload, n: int, seed: int = 0):
+    """n distinct rows (all of them when the workload has no more than n)."""
+    if wl.batch * wl.T * wl.num_q_heads <= n:
+        return all_rows(wl)
     rng = np.random.default_rng(seed)
     rows = set()
     # always the last query of every sequence and the first and last head

@@ -1,15 +1,18 @@
 """GPU parity of chunked-prefill attention (nvkv_prefill_attn) against the
 float64 oracle: a chunk of new queries, appended first, attends causally to
-the whole cache of its sequence."""
+the whole cache of its sequence.  head_dim 256 runs on the tensor-core
+kernel, head_dim 128 on the CUDA-core kernel; NVKV_DECODE_KERNEL=simt forces
+the latter for cross-checks."""
 import zlib
 
+import numpy as np
 import pytest
 import torch
 
 from nvfp4_quantized_kv_b200 import workload as W
 from nvfp4_quantized_kv_b200.harness import DeviceWorkload
 
-from parity_util import all_rows, assert_close, gpu_rows, oracle_outputs, sample_rows
+from parity_util import ATOL, RTOL, all_rows, assert_close, gpu_rows, oracle_outputs, sample_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -18,6 +21,8 @@ SMALL = [
     ("chunk_from_empty", 1, 8, 2, 128, 64, [0]),
     ("chunk_ragged", 2, 24, 4, 256, 37, [300, 5]),
     ("chunk_long", 1, 12, 2, 256, 200, [1500]),
+    ("chunk_tiny_tail", 3, 24, 4, 256, 1, [0, 63, 64]),
+    ("chunk_mtiles", 1, 24, 4, 256, 90, [700]),
 ]
 
 
@@ -31,10 +36,47 @@ def run(wl):
     return dw
 
 
+def seed_of(name):
+    return zlib.crc32(name.encode()) % 1000
+
+
 @pytest.mark.parametrize("case", SMALL, ids=[c[0] for c in SMALL])
 def test_prefill_small(case):
     name, b, hq, hkv, d, T, ctx = case
-    wl = W.small(name, b, hq, hkv, d, T, ctx, mode="prefill", seed=zlib.crc32(name.encode()) % 1000)
+    wl = W.small(name, b, hq, hkv, d, T, ctx, mode="prefill", seed=seed_of(name))
     dw = run(wl)
-    rows = all_rows(wl) if len(all_rows(wl)) <= 2000 else sample_rows(wl, 400, seed=3)
+    rows = all_rows(wl) if len(all_rows(wl)) <= 2500 else sample_rows(wl, 400, seed=3)
     assert_close(gpu_rows(dw.out, wl, rows), oracle_outputs(wl, rows), name)
+
+
+@pytest.mark.parametrize("case", [c for c in SMALL if c[4] == 256], ids=[c[0] for c in SMALL if c[4] == 256])
+def test_prefill_kernels_agree(case, monkeypatch):
+    name, b, hq, hkv, d, T, ctx = case
+    wl = W.small(name, b, hq, hkv, d, T, ctx, mode="prefill", seed=seed_of(name) + 1)
+    rows = sample_rows(wl, 200, seed=4)
+    ref = oracle_outputs(wl, rows)
+    for kernel in ("default", "simt"):
+        if kernel == "simt":
+            monkeypatch.setenv("NVKV_DECODE_KERNEL", "simt")
+        dw = run(wl)
+        assert_close(gpu_rows(dw.out, wl, rows), ref, f"{name}/{kernel}")
+
+
+def test_chunked_prefill_config_sampled():
+    """65536 cached tokens + a 2048-token chunk, 24/4 heads, head_dim 256."""
+    wl = W.chunked_prefill()
+    dw = run(wl)
+    rows = [(0, 0, 0), (0, 0, 23), (0, 2047, 0), (0, 2047, 17), (0, 1024, 5), (0, 21, 6),
+            (0, 22, 11), (0, 1500, 12)]
+    assert_close(gpu_rows(dw.out, wl, rows), oracle_outputs(wl, rows), wl.name)
+
+
+def test_prefill_tail_matches_decode_verify():
+    """The last T positions of a prefill chunk are an MTP-verify block: both
+    entry points must agree on the same cache and queries."""
+    ctx, T = 1000, 6
+    wp = W.small("tail", 2, 24, 4, 256, T, [ctx, 333], mode="prefill", seed=9)
+    wd = W.small("tail", 2, 24, 4, 256, T, [ctx, 333], mode="decode", seed=9)
+    a = run(wp).out.float()
+    b = run(wd).out.float()
+    assert ((a - b).abs() <= 2 * (ATOL + RTOL * b.abs())).all()
