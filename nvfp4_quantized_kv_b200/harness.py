@@ -29,12 +29,24 @@ def bf16_tensor(bits: np.ndarray, device) -> torch.Tensor:
 
 class DeviceWorkload:
     def __init__(self, wl: Workload, device="cuda", fill: int | None = 0xA5, num_splits: int = 0,
-                 err_word: bool = True):
+                 err_word: bool = True, cache_from: "DeviceWorkload | None" = None):
+        """cache_from: reuse the (already filled) pool of another workload
+        with the same cached context -- same seed, lengths, heads and page
+        table -- under a different step shape (T=1 decode and T=6 verify)."""
         self.wl = wl
         self.device = torch.device(device)
         self.num_splits = num_splits
-        self.cache = Cache.allocate(wl.num_pages, wl.num_kv_heads, wl.head_dim, self.device, fill)
         self.page_table_np = wl.page_table()
+        if cache_from is not None:
+            o = cache_from.wl
+            if (o.seed, list(o.ctx), o.num_kv_heads, o.head_dim, o.num_pages) != \
+                    (wl.seed, list(wl.ctx), wl.num_kv_heads, wl.head_dim, wl.num_pages) or \
+                    not np.array_equal(cache_from.page_table_np, self.page_table_np):
+                raise ValueError("cache_from: the two workloads do not share a cached context")
+            self.cache = cache_from.cache
+        else:
+            self.cache = Cache.allocate(wl.num_pages, wl.num_kv_heads, wl.head_dim, self.device,
+                                        fill)
         self.page_table = _h2d(self.page_table_np, self.device)
         self.kv_lens = _h2d(wl.kv_lens, self.device)
         self.err = torch.zeros(1, dtype=torch.int32, device=self.device) if err_word else None
