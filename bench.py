@@ -40,6 +40,7 @@ if ROOT not in sys.path:
 
 METRIC = "NVFP4 KV-read GB/s (% of HBM peak) and decode tokens/s at 3x~470k ctx"
 FALLBACK_HBM_GBS = 6650.0
+REF_BUDGET_S = 90.0  # oracle seconds of a whole --impl reference run
 DATASHEET_HBM_GBS = 8000.0
 
 # DRAM traffic of one decode-attention launch, from one ncu capture of the
@@ -129,14 +130,27 @@ class ClockSampler:
                 "samples": len(sm)}
 
 
-def oracle_sample(wl, rows_max=6, ctx_cap=None):
+def max_over_ranks(x: float, device) -> float:
+    """The largest value of x over all ranks (the slowest rank's time); x on
+    a single process."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def oracle_sample(wl, rows_max=6, ctx_cap=None, kv=None):
     """Time the float64 oracle on one (sequence 0, kv-head 0) pair: all its
-    query rows over its whole visible cache.  Returns (GB/s in the metric's
-    unit, seconds, threads, description)."""
+    query rows over its visible cache (the first ctx_cap positions when
+    capped; kv = the pre-generated rows of those positions).  Returns (GB/s
+    in the metric's unit, seconds, threads, description)."""
     import oracle
     b, h = 0, 0
     kv_len = int(wl.kv_lens[b]) if ctx_cap is None else min(int(wl.kv_lens[b]), ctx_cap)
-    k, v = wl.kv_rows(b, 0, kv_len)
+    k, v = kv if kv is not None else wl.kv_rows(b, 0, kv_len)
     q = wl.queries()
     G = wl.group
     jobs = []
@@ -151,8 +165,8 @@ def oracle_sample(wl, rows_max=6, ctx_cap=None):
     oracle.attention_rows(jobs, wl.num_kv_heads, wl.head_dim, wl.sm_scale, threads)
     dt = time.perf_counter() - t0
     kv_bytes = kv_len * wl.head_dim * 2 * (1 / 2 + 1 / 16)  # one kv-head, K and V, NVFP4
-    desc = (f"sequence 0 ({kv_len} tokens), kv-head 0, {len(jobs)} query rows (all rows of that "
-            f"pair), float64 oracle, {min(threads, len(jobs))} threads busy")
+    desc = (f"sequence 0 ({kv_len} of {int(wl.kv_lens[b])} tokens), kv-head 0, {len(jobs)} query "
+            f"rows (all rows of that pair), float64 oracle, {min(threads, len(jobs))} threads busy")
     return kv_bytes / dt / 1e9, dt, min(threads, len(jobs)), desc
 
 
@@ -162,12 +176,20 @@ def run_reference(args):
         return
     wl = W.long_context(T=args.T)
     cap = args.ref_ctx
+    if cap is None:
+        # Size the per-step sample so that all warm-up and timed steps take
+        # about REF_BUDGET_S of oracle time: calibrate on 4096 positions.
+        probe = oracle_sample(wl, ctx_cap=4096)
+        per_step = REF_BUDGET_S / (args.steps + args.warmup)
+        cap = int(4096 * per_step / max(probe[1], 1e-6))
+        cap = max(256, min(cap, int(wl.kv_lens[0])))
+    kv = wl.kv_rows(0, 0, min(cap, int(wl.kv_lens[0])))
     vals = []
     for _ in range(args.warmup):
-        oracle_sample(wl, ctx_cap=cap)
+        oracle_sample(wl, ctx_cap=cap, kv=kv)
     secs = 0.0
     for _ in range(args.steps):
-        v, dt, threads, desc = oracle_sample(wl, ctx_cap=cap)
+        v, dt, threads, desc = oracle_sample(wl, ctx_cap=cap, kv=kv)
         vals.append(v)
         secs += dt
     value = statistics.mean(vals)
@@ -268,11 +290,7 @@ def main():
         torch.cuda.synchronize(dev)
         if world > 1:
             dist.barrier()
-        ms = t_start.elapsed_time(t_end) / K
-        if world > 1:
-            tt = torch.tensor([ms], dtype=torch.float64, device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ms = float(tt.item())
+        ms = max_over_ranks(t_start.elapsed_time(t_end) / K, dev)
         return (ms, statistics.mean(e[0].elapsed_time(e[1]) for e in ev),
                 statistics.mean(e[1].elapsed_time(e[2]) for e in ev),
                 statistics.mean(e[2].elapsed_time(e[3]) for e in ev))
@@ -286,6 +304,11 @@ def main():
     err = dw.err_bits()
 
     kv_bytes = wl.kv_bytes_per_step()
+    l2_bytes = torch.cuda.get_device_properties(dev).L2_cache_size
+    l2_note = (f"inputs larger than L2 ({kv_bytes / 1e9:.2f} GB of KV per step, L2 "
+               f"{l2_bytes / 1e6:.0f} MB): no flush needed" if kv_bytes > l2_bytes else
+               f"inputs SMALLER than L2 ({kv_bytes / 1e6:.0f} MB of KV, L2 {l2_bytes / 1e6:.0f} MB):"
+               f" a profiling size, not a benchmark value")
     value = world * kv_bytes / (ms * 1e-3) / 1e9
     tokens_per_s = world * wl.batch * wl.T / (ms * 1e-3)
     peak, peak_kind = hbm_peak()
@@ -323,11 +346,7 @@ def main():
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize(dev)
-    e2e_ms = e0.elapsed_time(e1) / args.e2e_steps
-    if world > 1:
-        tt = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        e2e_ms = float(tt.item())
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / args.e2e_steps, dev)
     h2d = h_k.numel() * 2 + h_v.numel() * 2 + h_q.numel() * 2
     d2h = h_out.numel() * 2
 
@@ -396,7 +415,7 @@ def main():
                        "T": wl.T, "q_heads": wl.num_q_heads, "kv_heads": wl.num_kv_heads,
                        "head_dim": wl.head_dim, "page_tokens": 16, "num_splits": S,
                        "kv_bytes_per_step": kv_bytes,
-                       "l2": f"inputs larger than L2 ({kv_bytes / 1e9:.2f} GB of KV per step)",
+                       "l2": l2_note,
                        "parallelism": f"replicas{world}" if world > 1 else "single-gpu"},
             "hbm_frac": value / world / peak,
             "hbm_frac_datasheet": value / world / DATASHEET_HBM_GBS,

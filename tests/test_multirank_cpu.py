@@ -1,0 +1,76 @@
+"""Host logic of multi-process runs, on CPU with the gloo backend: the
+max-over-ranks time reduction bench.py applies at N > 1, and the reference
+arm's rank rule (rank 0 alone runs and prints)."""
+import os
+import socket
+import subprocess
+import sys
+
+import pytest
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+sys.path.insert(0, ROOT)
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, out):
+    os.environ["MASTER_ADDR"] = "127.0.0.1"
+    os.environ["MASTER_PORT"] = str(port)
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    try:
+        import bench
+        # rank r took (r + 1) * 1.5 ms: everyone must report the slowest
+        got = bench.max_over_ranks((rank + 1) * 1.5, torch.device("cpu"))
+        out[rank] = got
+        dist.barrier()
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_max_over_ranks_gloo(world):
+    port = _free_port()
+    ctx = mp.get_context("spawn")
+    mgr = ctx.Manager()
+    out = mgr.dict()
+    procs = [ctx.Process(target=_worker, args=(r, world, port, out)) for r in range(world)]
+    for p in procs:
+        p.start()
+    for p in procs:
+        p.join(120)
+        assert p.exitcode == 0
+    assert dict(out) == {r: world * 1.5 for r in range(world)}
+
+
+def test_max_over_ranks_single_process():
+    import bench
+    assert bench.max_over_ranks(2.5, torch.device("cpu")) == 2.5
+
+
+def test_reference_arm_nonzero_rank_is_silent():
+    env = dict(os.environ, RANK="1", WORLD_SIZE="2", LOCAL_RANK="1")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--gpus", "2", "--steps", "1", "--warmup", "3"],
+                       capture_output=True, text=True, timeout=300, env=env, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    assert r.stdout.strip() == ""
+
+
+def test_decode_traffic_tracks_the_captured_source(tmp_path, monkeypatch):
+    import bench
+    kv = 1_000_000
+    t = bench.decode_traffic(kv)
+    cap = bench.DECODE_CAPTURE
+    if t is not None:  # the source is the captured one: traffic scales with the KV bytes
+        assert t == pytest.approx(kv * (cap["dram_bytes_read"] + cap["dram_bytes_write"]) /
+                                  cap["kv_bytes"])
+    monkeypatch.setitem(cap, "sha256", "0" * 64)
+    assert bench.decode_traffic(kv) is None
