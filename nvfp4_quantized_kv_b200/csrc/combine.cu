@@ -43,24 +43,34 @@ combine_kernel(const int32_t *__restrict__ kv_lens, int B, int Hkv, int T, int H
   if (units > 0) {
     const int64_t c0 = range_of_unit(pair_start, U, S);
     const int64_t c1 = range_of_unit(pair_start + units - 1, U, S);
-    // A range that owns no unit (possible when U < S) wrote nothing.
+    // A range that owns no unit (possible only when U < S) wrote nothing.
+    const bool all_own_units = U >= S;
+    // The lse of up to 32 ranges at a time, one per lane; their max.
     float L = -INFINITY;
-    for (int64_t c = c0; c <= c1; ++c) {
-      if (range_begin(c, U, S) == range_begin(c + 1, U, S)) continue;
-      L = fmaxf(L, ws_lse[(size_t)(c + bh) * R + r]);
+    for (int64_t cb = c0; cb <= c1; cb += 32) {
+      const int64_t c = cb + lane;
+      if (c <= c1 && (all_own_units || range_begin(c, U, S) != range_begin(c + 1, U, S)))
+        L = fmaxf(L, ws_lse[(size_t)(c + bh) * R + r]);
     }
+    L = warp_max(L);
     if (L > -INFINITY) {
-      for (int64_t c = c0; c <= c1; ++c) {
-        if (range_begin(c, U, S) == range_begin(c + 1, U, S)) continue;
-        const size_t slot = (size_t)(c + bh);
-        const float lse = ws_lse[slot * R + r];
-        if (lse == -INFINITY) continue;
-        const float w = exp2f(lse - L);
-        wsum += w;
-        const float *o = ws_o + (slot * R + r) * (size_t)D + lane * dpl;
+      for (int64_t cb = c0; cb <= c1; cb += 32) {
+        const int64_t c = cb + lane;
+        float w = 0.f;  // weight of range c; 0 for ranges without keys of this row
+        if (c <= c1 && (all_own_units || range_begin(c, U, S) != range_begin(c + 1, U, S))) {
+          const float lse = ws_lse[(size_t)(c + bh) * R + r];
+          if (lse > -INFINITY) w = exp2f(lse - L);
+        }
+        const int n = c1 - cb + 1 < 32 ? (int)(c1 - cb + 1) : 32;
+        for (int k = 0; k < n; ++k) {
+          const float wk = __shfl_sync(0xffffffffu, w, k);
+          if (wk == 0.f) continue;  // warp-uniform
+          wsum += wk;
+          const float *o = ws_o + ((size_t)(cb + k + bh) * R + r) * (size_t)D + lane * dpl;
 #pragma unroll
-        for (int i = 0; i < 8; ++i)
-          if (i < dpl) acc[i] = fmaf(w, o[i], acc[i]);
+          for (int i = 0; i < 8; ++i)
+            if (i < dpl) acc[i] = fmaf(wk, o[i], acc[i]);
+        }
       }
     }
   }

@@ -80,3 +80,27 @@ def test_prefill_tail_matches_decode_verify():
     a = run(wp).out.float()
     b = run(wd).out.float()
     assert ((a - b).abs() <= 2 * (ATOL + RTOL * b.abs())).all()
+
+
+@pytest.mark.parametrize("kernel", ["default", "simt"])
+def test_prefill_reports_bad_page(kernel, monkeypatch):
+    """A page id outside the pool is reported through the error word; its
+    keys read as absent and nothing outside the pool is touched."""
+    import nvfp4_quantized_kv_b200 as nv
+    if kernel == "simt":
+        monkeypatch.setenv("NVKV_DECODE_KERNEL", "simt")
+    dev = torch.device("cuda")
+    hkv, hq, d, n = 2, 12, 256, 20
+    cache = nv.Cache.allocate(2, hkv, d, dev, fill=0)
+    pt = torch.tensor([[0, 9]], dtype=torch.int32, device=dev)  # page 9 does not exist
+    lens = torch.tensor([n], dtype=torch.int32, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    seqs = nv.Seqs(pt, lens, n, err)
+    q = torch.zeros((n, hq, d), dtype=torch.bfloat16, device=dev)
+    cu = torch.tensor([0, n], dtype=torch.int32, device=dev)
+    out = torch.empty((n, hq, d), dtype=torch.bfloat16, device=dev)
+    nv.nvkv_prefill_attn(cache, seqs, q, cu, n, n, hq, 0.0625, out)
+    torch.cuda.synchronize()
+    assert int(err.item()) & nv.DEVERR_PAGE_ID
+    assert torch.isfinite(out.float()).all()
+    assert (out == 0).all()  # an all-zero pool dequantises to 0
