@@ -146,6 +146,27 @@ __device__ __forceinline__ float2 f16x2_to_float2(uint32_t v) {
   return __half22float2(*reinterpret_cast<__half2 *>(&v));
 }
 
+// Packed fp32 pair arithmetic (one instruction for both lanes of the pair).
+__device__ __forceinline__ float2 add_f32x2(float2 a, float2 b) {
+  float2 d;
+  asm("{\n\t.reg .b64 ra, rb, rd;\n\t"
+      "mov.b64 ra, {%2, %3};\n\tmov.b64 rb, {%4, %5};\n\t"
+      "add.rn.f32x2 rd, ra, rb;\n\t"
+      "mov.b64 {%0, %1}, rd;\n\t}"
+      : "=f"(d.x), "=f"(d.y)
+      : "f"(a.x), "f"(a.y), "f"(b.x), "f"(b.y));
+  return d;
+}
+// (2^a, 2^b) as an f16 pair (a in the low half) with one exponential
+// instruction for both: the arguments are rounded to f16 first, so this is
+// for softmax weights that end up in f16 anyway.  2^-inf = +0.
+__device__ __forceinline__ uint32_t ex2_f16x2(float a, float b) {
+  uint32_t h, r;
+  asm("cvt.rn.f16x2.f32 %0, %2, %1;" : "=r"(h) : "f"(a), "f"(b));
+  asm("ex2.approx.f16x2 %0, %1;" : "=r"(r) : "r"(h));
+  return r;
+}
+
 // Warp reductions.
 __device__ __forceinline__ float warp_max(float v) {
 #pragma unroll

@@ -419,13 +419,20 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int H
       tc_fence_after();
       const uint32_t scol = tl + kColS + slot * 64;
       float x[64];
-#pragma unroll
-      for (int c16 = 0; c16 < 4; ++c16) {
-        uint32_t rr[16];
-        tmem_ld16(scol + c16 * 16, rr);
+      {
+        uint32_t r0[16], r1[16], r2[16], r3[16];
+        tmem_ld16(scol, r0);
+        tmem_ld16(scol + 16, r1);
+        tmem_ld16(scol + 32, r2);
+        tmem_ld16(scol + 48, r3);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) x[16 * c16 + e] = __uint_as_float(rr[e]);
+        for (int e = 0; e < 16; ++e) {
+          x[e] = __uint_as_float(r0[e]);
+          x[16 + e] = __uint_as_float(r1[e]);
+          x[32 + e] = __uint_as_float(r2[e]);
+          x[48 + e] = __uint_as_float(r3[e]);
+        }
       }
       const int key0 = j * kTileTokens;
       float tmax = -INFINITY;
@@ -464,16 +471,19 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int H
         l *= alpha;
         m = tmax;
       }
+      // Weights in f16, two per exponential instruction; masked keys are
+      // -inf and give 0 (a row with no visible key yet keeps m = -inf: it
+      // subtracts 0 instead).  The denominator sums the same f16 weights.
+      const float ms = m == -INFINITY ? 0.f : m;
       uint32_t pw[32];
+      float2 lv = make_float2(0.f, 0.f);
 #pragma unroll
       for (int e = 0; e < 32; ++e) {
-        const float p0 = x[2 * e] == -INFINITY ? 0.f : exp2f(x[2 * e] - m);
-        const float p1 = x[2 * e + 1] == -INFINITY ? 0.f : exp2f(x[2 * e + 1] - m);
-        __half2 hh = __floats2half2_rn(p0, p1);
-        const float2 back = __half22float2(hh);  // the denominator sums the f16 weights
-        l += back.x + back.y;
-        pw[e] = *reinterpret_cast<uint32_t *>(&hh);
+        const float2 dd = add_f32x2(make_float2(x[2 * e], x[2 * e + 1]), make_float2(-ms, -ms));
+        pw[e] = ex2_f16x2(dd.x, dd.y);
+        lv = add_f32x2(lv, f16x2_to_float2(pw[e]));
       }
+      l += lv.x + lv.y;
       // P overwrites the first 32 columns of its own S slot (already read).
       tmem_st16(scol, pw);
       tmem_st16(scol + 16, pw + 16);
