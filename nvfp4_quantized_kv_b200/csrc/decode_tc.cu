@@ -607,10 +607,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
               load_m(c16, m);
 #pragma unroll
               for (int e = 0; e < 8; ++e) {
-                const float d0 = x[2 * e] - m[2 * e], d1 = x[2 * e + 1] - m[2 * e + 1];
-                up |= (d0 > kLazyRescale) | (d1 > kLazyRescale);
-                __half2 hv2 = __floats2half2_rn(exp2f(d0), exp2f(d1));  // exp2(-inf) = 0
-                h2[8 * c16 + e] = *reinterpret_cast<uint32_t *>(&hv2);
+                const float2 dd = add_f32x2(make_float2(x[2 * e], x[2 * e + 1]),
+                                            make_float2(-m[2 * e], -m[2 * e + 1]));
+                up |= (dd.x > kLazyRescale) | (dd.y > kLazyRescale);
+                h2[8 * c16 + e] = ex2_f16x2(dd.x, dd.y);  // 2^-inf = 0
               }
             } else {
 #pragma unroll
@@ -687,9 +687,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
                 load_m(c16, m);
 #pragma unroll
                 for (int e = 0; e < 8; ++e) {
-                  __half2 hv2 = __floats2half2_rn(exp2f(x[2 * e] - m[2 * e]),
-                                                  exp2f(x[2 * e + 1] - m[2 * e + 1]));
-                  h2[8 * c16 + e] = *reinterpret_cast<uint32_t *>(&hv2);
+                  const float2 dd = add_f32x2(make_float2(x[2 * e], x[2 * e + 1]),
+                                              make_float2(-m[2 * e], -m[2 * e + 1]));
+                  h2[8 * c16 + e] = ex2_f16x2(dd.x, dd.y);
                 }
               }
             }
@@ -713,9 +713,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
             // the denominator sums the same f16 weights the PV uses
 #pragma unroll
             for (int e = 0; e < 8; ++e) {
-              const float2 back = __half22float2(*reinterpret_cast<const __half2 *>(&h2[8 * c16 + e]));
-              l_part[16 * c16 + 2 * e] += back.x;
-              l_part[16 * c16 + 2 * e + 1] += back.y;
+              const float2 lp = add_f32x2(
+                  make_float2(l_part[16 * c16 + 2 * e], l_part[16 * c16 + 2 * e + 1]),
+                  f16x2_to_float2(h2[8 * c16 + e]));
+              l_part[16 * c16 + 2 * e] = lp.x;
+              l_part[16 * c16 + 2 * e + 1] = lp.y;
             }
           }
           fence_proxy_async_smem();
