@@ -50,9 +50,9 @@ DATASHEET_HBM_GBS = 8000.0
 # the kernel source changes the figure no longer applies and is reported null.
 DECODE_CAPTURE = {
     "source": "nvfp4_quantized_kv_b200/csrc/decode_tc.cu",
-    "sha256": "aaad2426e55390cf91b887b5633080315d46b8b64bba258bbbe35338eeb4dda3",
-    "dram_bytes_read": 207614464,
-    "dram_bytes_write": 6113792,
+    "sha256": "7e9f4688de9c8156cefdb358ad323dfca36bb75c952e32e52d37abe676e035c0",
+    "dram_bytes_read": 207602944,
+    "dram_bytes_write": 4987136,
     "kv_bytes": 207363456,
 }
 

@@ -68,7 +68,9 @@ constexpr uint32_t kColO = 256;   // 256: O (row lanes, fp32 d)
 // Shared memory.
 constexpr int kOffK = kStages * kStageBytes;
 constexpr int kOffV = kOffK + 2 * kKTileBytes;
-constexpr int kOffPages = kOffV + 2 * kVTileBytes;           // int[stages][4]
+constexpr int kVscBytes = kTilePages * 16 * 8 * 4;            // V scales of a tile as f16 pairs
+constexpr int kOffVsc = kOffV + 2 * kVTileBytes;              // 2 tables (tile parity)
+constexpr int kOffPages = kOffVsc + 2 * kVscBytes;            // int[stages][4]
 constexpr int kOffFlags = kOffPages + kStages * kTilePages * 4;
 constexpr int kOffBars = kOffFlags + 16;
 constexpr int kNumBars = 2 * kStages + 2 * 5 + 2;  // full, empty; kready, vready, sready, pready, pvdone; qready, final
@@ -125,6 +127,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int H
   uint8_t *stages = smem;
   uint8_t *ktiles = smem + kOffK;
   uint8_t *vtiles = smem + kOffV;
+  uint32_t *vsc = reinterpret_cast<uint32_t *>(smem + kOffVsc);  // [2][page][group][8]
   int32_t *spages = reinterpret_cast<int32_t *>(smem + kOffPages);
   volatile int *flags = reinterpret_cast<volatile int *>(smem + kOffFlags);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBars);
@@ -270,6 +273,19 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int H
       const int4 pg4 = *reinterpret_cast<const int4 *>(spages + stage * kTilePages);
       const int pgs[4] = {pg4.x, pg4.y, pg4.z, pg4.w};
       const int tok0 = j * kTileTokens;
+      {
+        // This tile's V scales, converted once: thread t takes 4 consecutive
+        // tokens of one (page, group); the 16 V^T rows of a group share them.
+        // (Absent pages convert stale bytes that are never used.)
+        const int p = t >> 6, g = (t >> 2) & 15, q4 = t & 3;
+        const int srow = 34 + (g >> 3);
+        const uint32_t raw = *reinterpret_cast<const uint32_t *>(
+            stg + p * kPagePitch + srow * 128 + (((g & 7) ^ (srow & 7)) << 4) + 4 * q4);
+        uint32_t t2[2];
+        e4m3x4_to_f16x2x2(raw, t2);
+        *reinterpret_cast<uint2 *>(vsc + ((slot * kTilePages + p) * 16 + g) * 8 + 2 * q4) =
+            make_uint2(t2[0], t2[1]);
+      }
       // K tile slot: its previous tile's QK must be done.
       if (j >= 2) {
         wait_bar(&sready[slot], ((j >> 1) + 1) & 1, flags, err);
@@ -317,6 +333,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int H
       fence_proxy_async_smem();
       __syncwarp();
       if (lane == 0) mbar_arrive(&kready[slot]);
+      // The scale table of this tile is complete once every dequantising
+      // thread is here; all of them finished reading the table of tile j-2
+      // before arriving here for tile j-1.
+      named_barrier(1, kDeqWarps * 32);
       // V^T tile slot: its previous tile's PV must be done.
       if (j >= 2) {
         wait_bar(&pvdone[slot], ((j >> 1) + 1) & 1, flags, err);
@@ -327,8 +347,6 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int H
         const int g = d >> 4;
         const int vrow = 18 + (d >> 4);
         const int vchunk = ((d & 15) >> 1) ^ (vrow & 7);
-        const int srow = 34 + (g >> 3);
-        const int schunk = (g & 7) ^ (srow & 7);
         uint8_t *vt = vtiles + slot * kVTileBytes + (d >> 3) * 128 + (d & 7) * 16;
 #pragma unroll
         for (int p = 0; p < kTilePages; ++p) {
@@ -338,17 +356,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int H
             const uint8_t *pg = stg + p * kPagePitch;
             const uint2 cw =
                 *reinterpret_cast<const uint2 *>(pg + vrow * 128 + vchunk * 16 + (d & 1) * 8);
-            const uint4 s4 = *reinterpret_cast<const uint4 *>(pg + srow * 128 + schunk * 16);
-            uint32_t c0[4], c1[4], sp[8];
+            const uint4 *tb =
+                reinterpret_cast<const uint4 *>(vsc + ((slot * kTilePages + p) * 16 + g) * 8);
+            const uint4 sa = tb[0], sb = tb[1];
+            const uint32_t sp[8] = {sa.x, sa.y, sa.z, sa.w, sb.x, sb.y, sb.z, sb.w};
+            uint32_t c0[4], c1[4];
             e2m1x8_to_f16x2x4(cw.x, c0);
             e2m1x8_to_f16x2x4(cw.y, c1);
-            {
-              uint32_t t2[2];
-              e4m3x4_to_f16x2x2(s4.x, t2); sp[0] = t2[0]; sp[1] = t2[1];
-              e4m3x4_to_f16x2x2(s4.y, t2); sp[2] = t2[0]; sp[3] = t2[1];
-              e4m3x4_to_f16x2x2(s4.z, t2); sp[4] = t2[0]; sp[5] = t2[1];
-              e4m3x4_to_f16x2x2(s4.w, t2); sp[6] = t2[0]; sp[7] = t2[1];
-            }
 #pragma unroll
             for (int i = 0; i < 8; ++i) o8[i] = hmul2_u32(i < 4 ? c0[i] : c1[i - 4], sp[i]);
             if (ptok + kPageTokens - 1 > pos_last) {  // zero the tokens past the last query
