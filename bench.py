@@ -50,7 +50,7 @@ DATASHEET_HBM_GBS = 8000.0
 # the kernel source changes the figure no longer applies and is reported null.
 DECODE_CAPTURE = {
     "source": "nvfp4_quantized_kv_b200/csrc/decode_tc.cu",
-    "sha256": "7e9f4688de9c8156cefdb358ad323dfca36bb75c952e32e52d37abe676e035c0",
+    "sha256": "854b03576476adc3f282c87bc6e05aba24cbfa0a10be5865340f81de9378f374",
     "dram_bytes_read": 207602944,
     "dram_bytes_write": 4987136,
     "kv_bytes": 207363456,

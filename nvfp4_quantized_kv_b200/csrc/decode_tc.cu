@@ -20,10 +20,10 @@
 //    (2 x 128 d x 128 tokens) are the A operands, written straight from
 //    registers into Tensor Memory; the G*T query rows (Q, then P) are the
 //    small N side of the MMA, in shared memory.  S^T and O^T accumulate in
-//    Tensor Memory in fp32, and so does the softmax denominator: one more
-//    MMA of an all-ones A tile against P^T sums P over the tokens, with the
-//    same f16 P the value sums use.  Dequantisation is exact in f16
-//    (E2M1 x E4M3 has at most 6 significant bits).
+//    Tensor Memory in fp32; each softmax thread keeps per-row partial sums
+//    of the same f16 P the value sums use, reduced once per segment.
+//    Dequantisation is exact in f16 (E2M1 x E4M3 has at most 6 significant
+//    bits).
 //  * 16 dequantising warps (4 per SM sub-partition): each converts a quarter
 //    of the K tile (one token per thread, 32 d per QK phase) and of the V^T
 //    tile (one d row per thread, 64 tokens).  4 dedicated softmax warps run
