@@ -219,6 +219,7 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-prefill", action="store_true", help="skip the chunked-prefill line")
+    ap.add_argument("--no-spill", action="store_true", help="skip the page spill/restore line")
     ap.add_argument("--no-verify", action="store_true",
                     help="skip the T=6 MTP-verify line (measured on the T=1 pool)")
     ap.add_argument("--ctx", type=str, default=None,
@@ -350,6 +351,37 @@ def main():
     h2d = h_k.numel() * 2 + h_v.numel() * 2 + h_q.numel() * 2
     d2h = h_out.numel() * 2
 
+    # ---- host KV spill / restore of pool pages through a pinned arena ----
+    spill = None
+    if not args.no_spill:
+        pb = nv.nvkv_page_bytes(wl.num_kv_heads, wl.head_dim)
+        n_sp = min(4096, wl.num_pages)
+        sp_pages = torch.from_numpy(np.random.default_rng([wl.seed, 17]).choice(
+            wl.num_pages, size=n_sp, replace=False).astype(np.int32)).to(dev)
+        sp_slots = torch.arange(n_sp, dtype=torch.int32, device=dev)
+        arena = torch.empty(n_sp * pb, dtype=torch.uint8).pin_memory()
+        for _ in range(3):  # spill then restore the same pairs: the pool is unchanged
+            nv.nvkv_pages_spill(dw.cache, sp_pages, sp_slots, arena, dw.err, stream)
+            nv.nvkv_pages_restore(dw.cache, sp_pages, sp_slots, arena, dw.err, stream)
+        se = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+        reps = 5
+        torch.cuda.synchronize(dev)
+        se[0].record(stream)
+        for _ in range(reps):
+            nv.nvkv_pages_spill(dw.cache, sp_pages, sp_slots, arena, dw.err, stream)
+        se[1].record(stream)
+        for _ in range(reps):
+            nv.nvkv_pages_restore(dw.cache, sp_pages, sp_slots, arena, dw.err, stream)
+        se[2].record(stream)
+        torch.cuda.synchronize(dev)
+        d2h = se[0].elapsed_time(se[1]) / reps
+        h2d = se[1].elapsed_time(se[2]) / reps
+        spill = {"pages": n_sp, "bytes": n_sp * pb, "arena": "pinned host",
+                 "spill_ms": d2h, "spill_gbs": n_sp * pb / (d2h * 1e-3) / 1e9,
+                 "restore_ms": h2d, "restore_gbs": n_sp * pb / (h2d * 1e-3) / 1e9,
+                 "device_errors": dw.err_bits()}
+        del arena
+
     # ---- MTP verify (T=6) on the same cached context ----
     verify = None
     if args.T == 1 and not args.no_verify:
@@ -430,6 +462,7 @@ def main():
             "clocks": clk,
             "device_errors": err,
             "verify_T6": verify,
+            "spill": spill,
             "prefill": prefill,
             "cpu_baseline": cpu,
         }

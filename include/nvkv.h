@@ -192,6 +192,31 @@ nvkv_status nvkv_prefill_attn(const nvkv_cache *cache, const nvkv_seqs *seqs, co
                               int32_t num_q_heads, float sm_scale, void *out,
                               nvkv_stream_t stream);
 
+/* Host KV spill and restore ("gzenz/ninfer" README, "Context cache and
+ * eviction": when device KV runs out, evicted continuations move to a pinned
+ * host arena and move back when their cache is reused; placement in the
+ * arena is scatter-gather, so fragmentation never blocks a spill).
+ *   arena: num_slots page-sized slots, nvkv_page_bytes(Hkv, D) bytes each
+ *          (slot s at arena + s * page_bytes), 16-byte aligned, in pinned
+ *          host memory (cudaHostAlloc / cudaHostRegister, e.g. a torch
+ *          pin_memory tensor) or in device memory.  Pageable host memory is
+ *          refused with NVKV_ERR_INVALID_ARG before anything is launched.
+ *   nvkv_pages_spill:   pool page page_ids[i] -> arena slot slot_ids[i]
+ *   nvkv_pages_restore: arena slot slot_ids[i] -> pool page page_ids[i]
+ *          for i < n; a page moves whole (every kv-head), bit-exact.
+ *   page_ids, slot_ids: int32 [n], device or pinned host memory, read by
+ *          the kernel; a pair with an out-of-range id is skipped and sets
+ *          NVKV_DEVERR_PAGE_ID in *err_word (device int, optional).  Pairs
+ *          must not share a destination.
+ * One kernel per call on `stream` (pinned host memory is read and written
+ * through its device-visible address, no staging copy); n = 0 is a no-op. */
+nvkv_status nvkv_pages_spill(const nvkv_cache *cache, const int32_t *page_ids,
+                             const int32_t *slot_ids, int32_t n, void *arena, int64_t num_slots,
+                             int32_t *err_word, nvkv_stream_t stream);
+nvkv_status nvkv_pages_restore(const nvkv_cache *cache, const int32_t *page_ids,
+                               const int32_t *slot_ids, int32_t n, const void *arena,
+                               int64_t num_slots, int32_t *err_word, nvkv_stream_t stream);
+
 /* Static description of a status code. */
 const char *nvkv_status_string(nvkv_status status);
 

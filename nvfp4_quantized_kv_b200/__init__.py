@@ -74,6 +74,8 @@ def library():
             "nvkv_prefill_attn": (ctypes.c_int, [cp, sp, vp, vp, i32, i32, i32, f32, vp, vp]),
             "nvkv_decode_static_scratch_bytes": (sz, []),
             "nvkv_decode_attn_static": (ctypes.c_int, [cp, sp, vp, i32, i32, f32, i32, vp, vp]),
+            "nvkv_pages_spill": (ctypes.c_int, [cp, vp, vp, i32, vp, ctypes.c_int64, vp, vp]),
+            "nvkv_pages_restore": (ctypes.c_int, [cp, vp, vp, i32, vp, ctypes.c_int64, vp, vp]),
             "nvkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         }
         for name, (res, args) in sig.items():
@@ -226,3 +228,42 @@ def nvkv_decode_attn_static(cache: Cache, seqs: Seqs, q: torch.Tensor, T: int, n
         ctypes.byref(cache._c), ctypes.byref(seqs._c), _dev(q, torch.bfloat16, "q"), int(T),
         int(num_q_heads), float(sm_scale), int(num_splits), _dev(out, torch.bfloat16, "out"),
         _stream(stream)), "nvkv_decode_attn_static")
+
+
+def _dev_or_pinned(t: torch.Tensor, dtype: torch.dtype, name: str) -> int:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if not (t.is_cuda or t.is_pinned()):
+        raise ValueError(f"{name} must be on a CUDA device or in pinned host memory")
+    return t.data_ptr()
+
+
+def _pages_args(cache: Cache, page_ids, slot_ids, arena, err_word):
+    n = page_ids.numel()
+    if slot_ids.numel() != n:
+        raise ValueError("page_ids and slot_ids must have the same length")
+    pb = nvkv_page_bytes(cache.num_kv_heads, cache.head_dim)
+    return (ctypes.byref(cache._c), _dev_or_pinned(page_ids, torch.int32, "page_ids"),
+            _dev_or_pinned(slot_ids, torch.int32, "slot_ids"), int(n),
+            _dev_or_pinned(arena, torch.uint8, "arena"), arena.numel() // pb,
+            _dev(err_word, torch.int32, "err_word") if err_word is not None else None)
+
+
+def nvkv_pages_spill(cache: Cache, page_ids: torch.Tensor, slot_ids: torch.Tensor,
+                     arena: torch.Tensor, err_word: torch.Tensor | None = None, stream=None) -> None:
+    """Pool page page_ids[i] -> arena slot slot_ids[i] (arena: uint8, device
+    or pinned host, a whole number of page-sized slots)."""
+    _check(library().nvkv_pages_spill(*_pages_args(cache, page_ids, slot_ids, arena, err_word),
+                                      _stream(stream)), "nvkv_pages_spill")
+
+
+def nvkv_pages_restore(cache: Cache, page_ids: torch.Tensor, slot_ids: torch.Tensor,
+                       arena: torch.Tensor, err_word: torch.Tensor | None = None,
+                       stream=None) -> None:
+    """Arena slot slot_ids[i] -> pool page page_ids[i]."""
+    _check(library().nvkv_pages_restore(*_pages_args(cache, page_ids, slot_ids, arena, err_word),
+                                        _stream(stream)), "nvkv_pages_restore")

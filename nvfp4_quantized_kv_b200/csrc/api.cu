@@ -22,6 +22,8 @@ cudaError_t launch_combine(const nvkv_seqs &, const void *, const void *, int, i
                            void *, cudaStream_t);
 cudaError_t launch_prefill_simt(const nvkv_cache &, const nvkv_seqs &, const void *,
                                 const int32_t *, int, int, float, void *, cudaStream_t);
+cudaError_t launch_page_copy(const uint8_t *, int64_t, uint8_t *, int64_t, const int32_t *,
+                             const int32_t *, int, int64_t, int32_t *, cudaStream_t);
 }  // namespace nvkv
 
 using namespace nvkv;
@@ -76,6 +78,42 @@ WorkspaceLayout layout(int batch, int T, int Hq, int Hkv, int D, int S) {
 }
 
 nvkv_status cuda_status(cudaError_t e) { return e == cudaSuccess ? NVKV_OK : NVKV_ERR_CUDA; }
+
+// The address through which a kernel reaches p: device (or managed) memory
+// as it is, pinned host memory through its mapped device address; nullptr
+// for anything a kernel cannot touch (pageable host memory, unknown).
+const void *device_view(const void *p) {
+  cudaPointerAttributes a;
+  if (cudaPointerGetAttributes(&a, p) != cudaSuccess) {
+    cudaGetLastError();  // clear the (non-sticky) error of the failed query
+    return nullptr;
+  }
+  if (a.type == cudaMemoryTypeDevice || a.type == cudaMemoryTypeManaged) return p;
+  if (a.type == cudaMemoryTypeHost) return a.devicePointer;
+  return nullptr;
+}
+
+nvkv_status pages_move(const nvkv_cache *cache, const int32_t *page_ids, const int32_t *slot_ids,
+                       int32_t n, const void *arena, int64_t num_slots, int32_t *err_word,
+                       nvkv_stream_t stream, bool spill) {
+  const nvkv_status st = check_cache(cache);
+  if (st != NVKV_OK) return st;
+  if (n < 0 || num_slots <= 0 || !page_ids || !slot_ids || !arena || !aligned16(arena))
+    return NVKV_ERR_INVALID_ARG;
+  if (n == 0) return NVKV_OK;
+  const void *pid = device_view(page_ids), *sid = device_view(slot_ids), *ar = device_view(arena);
+  if (!pid || !sid || !ar || !aligned16(ar)) return NVKV_ERR_INVALID_ARG;
+  const int64_t pb = (int64_t)nvkv_page_bytes(cache->num_kv_heads, cache->head_dim);
+  uint8_t *pool = cache->pool;
+  uint8_t *arena_b = const_cast<uint8_t *>(static_cast<const uint8_t *>(ar));
+  const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  const int32_t *p32 = static_cast<const int32_t *>(pid), *s32 = static_cast<const int32_t *>(sid);
+  return cuda_status(spill ? launch_page_copy(pool, cache->num_pages, arena_b, num_slots, p32, s32,
+                                              n, pb, err_word, s)
+                           : launch_page_copy(arena_b, num_slots, pool, cache->num_pages, s32,
+                                              p32, n, pb, err_word, s));
+}
+
 
 // NVKV_DECODE_KERNEL=simt forces the CUDA-core decode and prefill kernels
 // (used by the tests to cross-check the two kernel families on the same
@@ -208,6 +246,18 @@ nvkv_status nvkv_prefill_attn(const nvkv_cache *cache, const nvkv_seqs *seqs, co
                                          sm_scale, out, st_));
   return cuda_status(
       launch_prefill_simt(*cache, *seqs, q, cu_q, total_q, num_q_heads, sm_scale, out, st_));
+}
+
+nvkv_status nvkv_pages_spill(const nvkv_cache *cache, const int32_t *page_ids,
+                             const int32_t *slot_ids, int32_t n, void *arena, int64_t num_slots,
+                             int32_t *err_word, nvkv_stream_t stream) {
+  return pages_move(cache, page_ids, slot_ids, n, arena, num_slots, err_word, stream, true);
+}
+
+nvkv_status nvkv_pages_restore(const nvkv_cache *cache, const int32_t *page_ids,
+                               const int32_t *slot_ids, int32_t n, const void *arena,
+                               int64_t num_slots, int32_t *err_word, nvkv_stream_t stream) {
+  return pages_move(cache, page_ids, slot_ids, n, arena, num_slots, err_word, stream, false);
 }
 
 const char *nvkv_status_string(nvkv_status status) {

@@ -146,3 +146,23 @@ def test_split_plan_partitions_units(lib, seed):
     used = {c + bh for c, bh in slots}
     assert len(used) == len(slots)
     assert max(used, default=0) <= S + B * hkv - 2
+
+
+def test_pages_spill_restore_reject_bad_arguments_without_launch(lib):
+    c = cache()
+    B = ctypes.byref
+    for f in (lib.nvkv_pages_spill, lib.nvkv_pages_restore):
+        assert f(None, 0x10, 0x20, 1, 0x1000, 4, None, None) == nv.ERR_INVALID_ARG
+        assert f(B(c), 0x10, 0x20, -1, 0x1000, 4, None, None) == nv.ERR_INVALID_ARG
+        assert f(B(c), None, 0x20, 1, 0x1000, 4, None, None) == nv.ERR_INVALID_ARG
+        assert f(B(c), 0x10, None, 1, 0x1000, 4, None, None) == nv.ERR_INVALID_ARG
+        assert f(B(c), 0x10, 0x20, 1, None, 4, None, None) == nv.ERR_INVALID_ARG
+        assert f(B(c), 0x10, 0x20, 1, 0x1008, 4, None, None) == nv.ERR_INVALID_ARG  # unaligned arena
+        assert f(B(c), 0x10, 0x20, 1, 0x1000, 0, None, None) == nv.ERR_INVALID_ARG  # no slots
+        assert f(B(c), 0x10, 0x20, 0, 0x1000, 4, None, None) == nv.OK  # nothing to move
+        # pointers no kernel can reach (here: not CUDA memory at all) are refused
+        buf = (ctypes.c_uint8 * 4096)()
+        ids = (ctypes.c_int32 * 1)()
+        a = (ctypes.addressof(buf) + 15) & ~15
+        assert f(B(c), ctypes.addressof(ids), ctypes.addressof(ids), 1, a, 1, None, None) == \
+            nv.ERR_INVALID_ARG
