@@ -76,6 +76,14 @@ def lib():
             L.oracle_append.argtypes = [vp, i32, i32, vp, i32, vp, i32, vp, vp, vp]
             L.oracle_pool_read_row.restype = None
             L.oracle_pool_read_row.argtypes = [vp, i32, i32, vp, i32, i32, i32, vp]
+            L.oracle_rope_table.restype = None
+            L.oracle_rope_table.argtypes = [i32, i32, d, d, vp]
+            L.oracle_rope_rotate_f32.restype = None
+            L.oracle_rope_rotate_f32.argtypes = [vp, i32, i32, vp, vp]
+            L.oracle_quantize_group_f32.restype = None
+            L.oracle_quantize_group_f32.argtypes = [vp, vp, vp]
+            L.oracle_append_rope.restype = None
+            L.oracle_append_rope.argtypes = [vp, i32, i32, vp, i32, vp, i32, vp, vp, vp, i32, vp, i32]
             L.oracle_attention_rows.restype = None
             L.oracle_attention_rows.argtypes = [i32, vp, vp, i32, i32, vp, vp, vp, d, vp, vp, vp, i32]
             L.oracle_attention_pool.restype = None
@@ -254,3 +262,46 @@ def attention_pool(pool: np.ndarray, num_kv_heads: int, head_dim: int, jobs, sm_
                                 _ptr(psum), int(nthreads or os.cpu_count() or 1))
     del keep
     return out, lse, psum
+
+
+# --------------------------------------------------------------------------
+# rotary position embedding of K fused with quantise-append
+# --------------------------------------------------------------------------
+def rope_table(max_pos: int, rotary_dim: int, base: float, scale: float) -> np.ndarray:
+    """float32 [max_pos][rotary_dim/2][2]: (cos, sin) of
+    (pos / scale) * base^(-2i / rotary_dim), from double."""
+    cs = np.zeros((max_pos, rotary_dim // 2, 2), np.float32)
+    lib().oracle_rope_table(int(max_pos), int(rotary_dim), float(base), float(scale), _ptr(cs))
+    return cs
+
+
+def rope_rotate_f32(row_bits, rotary_dim: int, cs_pos) -> np.ndarray:
+    """One bf16 row (uint16 bits [D]) rotated in float by one table row."""
+    row = _u16(row_bits).reshape(-1)
+    cs_pos = np.ascontiguousarray(cs_pos, np.float32).reshape(-1)
+    out = np.zeros(row.shape[0], np.float32)
+    lib().oracle_rope_rotate_f32(_ptr(row), int(row.shape[0]), int(rotary_dim), _ptr(cs_pos),
+                                 _ptr(out))
+    return out
+
+
+def quantize_group_f32(x) -> tuple[np.ndarray, int]:
+    """16 float32 values -> (16 E2M1 codes, E4M3 scale byte)."""
+    x = np.ascontiguousarray(x, np.float32).reshape(16)
+    codes = np.zeros(16, np.uint8)
+    sb = np.zeros(1, np.uint8)
+    lib().oracle_quantize_group_f32(_ptr(x), _ptr(codes), _ptr(sb))
+    return codes, int(sb[0])
+
+
+def append_rope(pool: np.ndarray, Hkv: int, D: int, page_table, kv_lens, k_new_bits, v_new_bits,
+                cu_new, rotary_dim: int, cs) -> None:
+    """oracle.append with K rotated at its position by table cs (in place)."""
+    pt = np.ascontiguousarray(page_table, np.int32)
+    lens = np.ascontiguousarray(kv_lens, np.int32)
+    cu = np.ascontiguousarray(cu_new, np.int32)
+    k, v = _u16(k_new_bits), _u16(v_new_bits)
+    cs = np.ascontiguousarray(cs, np.float32)
+    lib().oracle_append_rope(_ptr(pool), int(Hkv), int(D), _ptr(pt), int(pt.shape[1]), _ptr(lens),
+                             int(pt.shape[0]), _ptr(k), _ptr(v), _ptr(cu), int(rotary_dim), _ptr(cs),
+                             int(cs.shape[0]))

@@ -307,6 +307,117 @@ void oracle_pool_read_row(const uint8_t *pool, int Hkv, int D, const int32_t *pa
 }
 
 /* ------------------------------------------------------------------------ */
+/* Rotary position embedding of K, fused with quantise-append               */
+/* ------------------------------------------------------------------------ */
+/* "gzenz/ninfer" README, "Fork changes vs upstream" -> "Context and model":
+ * YaRN context extension, stated there as linear RoPE scaling (positions
+ * divided by a scaling factor).  The pages fix nothing else; the readings:
+ * the first rotary_dim elements of a head rotate, element i paired with
+ * element i + rotary_dim/2 (i < rotary_dim/2), by the angle
+ * (pos / scale) * base^(-2i / rotary_dim); the remaining elements pass
+ * through.  V is not rotated. */
+
+/* (cos, sin) of the angle for positions 0 .. max_pos-1 and pairs
+ * 0 .. rotary_dim/2-1, computed in double and rounded once to float:
+ * cs[(pos * rotary_dim/2 + i) * 2 + {0, 1}]. */
+void oracle_rope_table(int max_pos, int rotary_dim, double base, double scale, float *cs) {
+    int h = rotary_dim / 2;
+    for (int p = 0; p < max_pos; ++p)
+        for (int i = 0; i < h; ++i) {
+            double inv_freq = pow(base, -2.0 * i / rotary_dim);
+            double a = ((double)p / scale) * inv_freq;
+            cs[((size_t)p * h + i) * 2 + 0] = (float)cos(a);
+            cs[((size_t)p * h + i) * 2 + 1] = (float)sin(a);
+        }
+}
+
+/* Rotate one bf16 row of D elements in float, in the stated operation
+ * order (the fused append kernel's): with c, s the float table entries,
+ *   x' = fma(x, c, -(y * s)),   y' = fma(y, c, x * s),
+ * each product y*s and x*s rounded to float, fma rounded once. */
+void oracle_rope_rotate_f32(const uint16_t *row, int D, int rotary_dim, const float *cs_pos,
+                            float *out) {
+    int h = rotary_dim / 2;
+    for (int d = 0; d < D; ++d) out[d] = (float)oracle_bf16_value(row[d]);
+    for (int i = 0; i < h; ++i) {
+        float c = cs_pos[2 * i], sn = cs_pos[2 * i + 1];
+        float x = (float)oracle_bf16_value(row[i]), y = (float)oracle_bf16_value(row[i + h]);
+        float ys = y * sn, xs = x * sn;
+        out[i] = fmaf(x, c, -ys);
+        out[i + h] = fmaf(y, c, xs);
+    }
+}
+
+/* Quantise one group of 16 float values.  The scale is taken from the
+ * float quotient amax / 6 rounded to E4M3 (what the kernel computes); for
+ * normal values this is the decision of the exact quotient too (amax lies on
+ * a grid 4-8 float ulps of amax/6 wide, so an inexact float quotient is at
+ * least 2/3 ulp away from any E4M3 midpoint).  Codes: as for bf16 groups; an
+ * inexact x / scale is at least 2^-24 (relative) away from an E2M1
+ * midpoint, far more than the double rounding error. */
+void oracle_quantize_group_f32(const float x[16], uint8_t codes[16], uint8_t *scale_byte) {
+    float amax = 0.0f;
+    for (int i = 0; i < 16; ++i) {
+        float a = fabsf(x[i]);
+        if (a > amax) amax = a;
+    }
+    float q = amax / 6.0f;
+    uint8_t sb = oracle_e4m3_round((double)q);
+    double scale = oracle_e4m3_value(sb);
+    *scale_byte = sb;
+    for (int i = 0; i < 16; ++i) {
+        if (scale == 0.0) {
+            codes[i] = 0;
+            continue;
+        }
+        int idx = oracle_e2m1_round_index(fabs((double)x[i]) / scale);
+        int neg = signbit(x[i]) ? 1 : 0;
+        codes[i] = (uint8_t)((idx == 0) ? 0 : ((neg << 3) | idx));
+    }
+}
+
+/* Append with K rotated at its position (table cs as from
+ * oracle_rope_table, max_pos rows); V as oracle_append. */
+void oracle_append_rope(uint8_t *pool, int Hkv, int D, const int32_t *page_table,
+                        int max_pages_per_seq, const int32_t *kv_lens, int batch,
+                        const uint16_t *k_new, const uint16_t *v_new, const int32_t *cu_new,
+                        int rotary_dim, const float *cs, int max_pos) {
+    float krot[512];
+    uint8_t codes[16], sb;
+    int nib;
+    for (int b = 0; b < batch; ++b) {
+        int n = cu_new[b + 1] - cu_new[b];
+        const int32_t *page_row = page_table + (size_t)b * max_pages_per_seq;
+        for (int i = 0; i < n; ++i) {
+            int row = cu_new[b] + i;
+            int pos = kv_lens[b] - n + i;
+            if (pos >= max_pos) continue;  /* no table row: the kernel skips it too */
+            int page = page_row[pos / 16], s = pos % 16;
+            for (int hh = 0; hh < Hkv; ++hh) {
+                const uint16_t *kr = k_new + ((size_t)row * Hkv + hh) * D;
+                const uint16_t *vr = v_new + ((size_t)row * Hkv + hh) * D;
+                oracle_rope_rotate_f32(kr, D, rotary_dim, cs + (size_t)pos * (rotary_dim / 2) * 2,
+                                       krot);
+                for (int g = 0; g < D / 16; ++g) {
+                    oracle_quantize_group_f32(krot + 16 * g, codes, &sb);
+                    for (int e = 0; e < 16; ++e) {
+                        size_t off = pool_offset_kcode(page, hh, s, 16 * g + e, Hkv, D, &nib);
+                        put_nibble(pool, off, nib, codes[e]);
+                    }
+                    pool[pool_offset_kscale(page, hh, s, g, Hkv, D)] = sb;
+                    oracle_quantize_group(vr + 16 * g, codes, &sb);
+                    for (int e = 0; e < 16; ++e) {
+                        size_t off = pool_offset_vcode(page, hh, s, 16 * g + e, Hkv, D, &nib);
+                        put_nibble(pool, off, nib, codes[e]);
+                    }
+                    pool[pool_offset_vscale(page, hh, s, g, Hkv, D)] = sb;
+                }
+            }
+        }
+    }
+}
+
+/* ------------------------------------------------------------------------ */
 /* Attention                                                                 */
 /* ------------------------------------------------------------------------ */
 
