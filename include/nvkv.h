@@ -192,6 +192,32 @@ nvkv_status nvkv_prefill_attn(const nvkv_cache *cache, const nvkv_seqs *seqs, co
                               int32_t num_q_heads, float sm_scale, void *out,
                               nvkv_stream_t stream);
 
+/* Rotary position embedding of K fused with the quantise-append: the YaRN
+ * context extension of the "gzenz/ninfer" README, "Fork changes vs
+ * upstream" -> "Context and model", stated there as linear RoPE scaling
+ * (--rope-scaling-factor).  The pages fix no base, rotary width or pairing;
+ * this library's reading: the first rotary_dim elements of each K head
+ * rotate, element i paired with element i + rotary_dim/2, by the angle
+ * (pos / scale) * base^(-2i / rotary_dim); V and the other elements are
+ * stored unrotated (queries are rotated by the caller with the same table).
+ *
+ * nvkv_rope_table fills cs (device float [max_pos][rotary_dim/2][2], 8-byte
+ * aligned) with (cos, sin) of those angles, computed in double and rounded
+ * once to float.  rotary_dim > 0 and a multiple of 32; base, scale > 0.
+ *
+ * nvkv_append_rope is nvkv_append with each K row rotated at its position
+ * by row pos of rope_cs (max_pos rows) before quantisation, in float:
+ * x' = fma(x, c, -(y*s)), y' = fma(y, c, x*s) (products rounded to float).
+ * 0 < rotary_dim <= head_dim, rotary_dim % 32 == 0.  A new row whose
+ * position has no table row (pos >= max_pos) is not written (neither K nor
+ * V) and sets NVKV_DEVERR_LENGTH. */
+nvkv_status nvkv_rope_table(float *cs, int32_t max_pos, int32_t rotary_dim, double base,
+                            double scale, nvkv_stream_t stream);
+nvkv_status nvkv_append_rope(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *k_new,
+                             const void *v_new, const int32_t *cu_new, int32_t total_new,
+                             int32_t max_new, const float *rope_cs, int32_t max_pos,
+                             int32_t rotary_dim, nvkv_stream_t stream);
+
 /* Host KV spill and restore ("gzenz/ninfer" README, "Context cache and
  * eviction": when device KV runs out, evicted continuations move to a pinned
  * host arena and move back when their cache is reused; placement in the

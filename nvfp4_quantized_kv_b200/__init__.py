@@ -74,6 +74,8 @@ def library():
             "nvkv_prefill_attn": (ctypes.c_int, [cp, sp, vp, vp, i32, i32, i32, f32, vp, vp]),
             "nvkv_decode_static_scratch_bytes": (sz, []),
             "nvkv_decode_attn_static": (ctypes.c_int, [cp, sp, vp, i32, i32, f32, i32, vp, vp]),
+            "nvkv_rope_table": (ctypes.c_int, [vp, i32, i32, ctypes.c_double, ctypes.c_double, vp]),
+            "nvkv_append_rope": (ctypes.c_int, [cp, sp, vp, vp, vp, i32, i32, vp, i32, i32, vp]),
             "nvkv_pages_spill": (ctypes.c_int, [cp, vp, vp, i32, vp, ctypes.c_int64, vp, vp]),
             "nvkv_pages_restore": (ctypes.c_int, [cp, vp, vp, i32, vp, ctypes.c_int64, vp, vp]),
             "nvkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
@@ -186,6 +188,28 @@ def nvkv_append(cache: Cache, seqs: Seqs, k_new: torch.Tensor, v_new: torch.Tens
         ctypes.byref(cache._c), ctypes.byref(seqs._c), _dev(k_new, torch.bfloat16, "k_new"),
         _dev(v_new, torch.bfloat16, "v_new"), _dev(cu_new, torch.int32, "cu_new"), int(total_new),
         int(max_new), _stream(stream)), "nvkv_append")
+
+
+def nvkv_rope_table(cs: torch.Tensor, rotary_dim: int, base: float, scale: float,
+                    stream=None) -> None:
+    """Fill cs (float32 CUDA [max_pos][rotary_dim/2][2]) with (cos, sin) of
+    (pos / scale) * base^(-2i / rotary_dim)."""
+    if cs.dim() != 3 or cs.shape[1] * 2 != rotary_dim or cs.shape[2] != 2:
+        raise ValueError("cs must be [max_pos][rotary_dim/2][2]")
+    _check(library().nvkv_rope_table(_dev(cs, torch.float32, "cs"), int(cs.shape[0]),
+                                     int(rotary_dim), float(base), float(scale), _stream(stream)),
+           "nvkv_rope_table")
+
+
+def nvkv_append_rope(cache: Cache, seqs: Seqs, k_new: torch.Tensor, v_new: torch.Tensor,
+                     cu_new: torch.Tensor, total_new: int, max_new: int, rope_cs: torch.Tensor,
+                     rotary_dim: int, stream=None) -> None:
+    """nvkv_append with K rotated at its position by the rope_cs table."""
+    _check(library().nvkv_append_rope(
+        ctypes.byref(cache._c), ctypes.byref(seqs._c), _dev(k_new, torch.bfloat16, "k_new"),
+        _dev(v_new, torch.bfloat16, "v_new"), _dev(cu_new, torch.int32, "cu_new"), int(total_new),
+        int(max_new), _dev(rope_cs, torch.float32, "rope_cs"), int(rope_cs.shape[0]),
+        int(rotary_dim), _stream(stream)), "nvkv_append_rope")
 
 
 def nvkv_decode_attn(cache: Cache, seqs: Seqs, q: torch.Tensor, T: int, num_q_heads: int,

@@ -9,7 +9,8 @@
 
 namespace nvkv {
 cudaError_t launch_append(const nvkv_cache &, const nvkv_seqs &, const void *, const void *,
-                          const int32_t *, int, int, cudaStream_t);
+                          const int32_t *, int, int, const float *, int, int, cudaStream_t);
+cudaError_t launch_rope_table(float *, int, int, double, double, cudaStream_t);
 cudaError_t launch_decode_simt(const nvkv_cache &, const nvkv_seqs &, const void *, int, int,
                                float, int, float *, float *, cudaStream_t);
 bool decode_tc_supported(const nvkv_cache &, int, int);
@@ -189,6 +190,35 @@ nvkv_status nvkv_append(const nvkv_cache *cache, const nvkv_seqs *seqs, const vo
   if (!k_new || !v_new || !cu_new || !aligned16(k_new) || !aligned16(v_new))
     return NVKV_ERR_INVALID_ARG;
   return cuda_status(launch_append(*cache, *seqs, k_new, v_new, cu_new, total_new, max_new,
+                                   nullptr, 0, 0, reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvkv_status nvkv_rope_table(float *cs, int32_t max_pos, int32_t rotary_dim, double base,
+                            double scale, nvkv_stream_t stream) {
+  if (!cs || (reinterpret_cast<uintptr_t>(cs) & 7u) || max_pos <= 0 || rotary_dim <= 0 ||
+      rotary_dim % 32 != 0 || !(base > 0.0) || !(scale > 0.0) || !std::isfinite(base) ||
+      !std::isfinite(scale))
+    return NVKV_ERR_INVALID_ARG;
+  return cuda_status(launch_rope_table(cs, max_pos, rotary_dim, base, scale,
+                                       reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvkv_status nvkv_append_rope(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *k_new,
+                             const void *v_new, const int32_t *cu_new, int32_t total_new,
+                             int32_t max_new, const float *rope_cs, int32_t max_pos,
+                             int32_t rotary_dim, nvkv_stream_t stream) {
+  nvkv_status st = check_cache(cache);
+  if (st != NVKV_OK) return st;
+  if ((st = check_seqs(seqs)) != NVKV_OK) return st;
+  if (total_new < 0 || max_new < 0) return NVKV_ERR_INVALID_ARG;
+  if (!rope_cs || (reinterpret_cast<uintptr_t>(rope_cs) & 7u) || max_pos <= 0 ||
+      rotary_dim <= 0 || rotary_dim % 32 != 0 || rotary_dim > cache->head_dim)
+    return NVKV_ERR_INVALID_ARG;
+  if (total_new == 0 || max_new == 0) return NVKV_OK;
+  if (!k_new || !v_new || !cu_new || !aligned16(k_new) || !aligned16(v_new))
+    return NVKV_ERR_INVALID_ARG;
+  return cuda_status(launch_append(*cache, *seqs, k_new, v_new, cu_new, total_new, max_new,
+                                   rope_cs, rotary_dim, max_pos,
                                    reinterpret_cast<cudaStream_t>(stream)));
 }
 

@@ -166,3 +166,23 @@ def test_pages_spill_restore_reject_bad_arguments_without_launch(lib):
         a = (ctypes.addressof(buf) + 15) & ~15
         assert f(B(c), ctypes.addressof(ids), ctypes.addressof(ids), 1, a, 1, None, None) == \
             nv.ERR_INVALID_ARG
+
+
+def test_rope_calls_reject_bad_arguments_without_launch(lib):
+    c, s = cache(), seqs()
+    B = ctypes.byref
+    t = lib.nvkv_rope_table
+    assert t(None, 16, 64, 1e4, 1.0, None) == nv.ERR_INVALID_ARG
+    assert t(0x1004, 16, 64, 1e4, 1.0, None) == nv.ERR_INVALID_ARG   # not 8-byte aligned
+    assert t(0x1000, 0, 64, 1e4, 1.0, None) == nv.ERR_INVALID_ARG
+    assert t(0x1000, 16, 48, 1e4, 1.0, None) == nv.ERR_INVALID_ARG   # not a multiple of 32
+    assert t(0x1000, 16, 64, -1.0, 1.0, None) == nv.ERR_INVALID_ARG
+    assert t(0x1000, 16, 64, 1e4, 0.0, None) == nv.ERR_INVALID_ARG
+    a = lib.nvkv_append_rope
+    ok = (0x10, 0x20, 0x30, 1, 1)
+    assert a(B(c), B(s), *ok, None, 16, 64, None) == nv.ERR_INVALID_ARG
+    assert a(B(c), B(s), *ok, 0x1000, 16, 0, None) == nv.ERR_INVALID_ARG
+    assert a(B(c), B(s), *ok, 0x1000, 16, 160, None) == nv.ERR_INVALID_ARG  # > head_dim 128
+    assert a(B(c), B(s), *ok, 0x1000, 16, 40, None) == nv.ERR_INVALID_ARG
+    assert a(B(c), B(s), *ok, 0x1000, 0, 64, None) == nv.ERR_INVALID_ARG
+    assert a(B(c), B(s), 0x10, 0x20, 0x30, 0, 0, 0x1000, 16, 64, None) == nv.OK  # nothing new
