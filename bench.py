@@ -41,6 +41,11 @@ if ROOT not in sys.path:
 METRIC = "NVFP4 KV-read GB/s (% of HBM peak) and decode tokens/s at 3x~470k ctx"
 FALLBACK_HBM_GBS = 6650.0
 REF_BUDGET_S = 90.0  # oracle seconds of a whole --impl reference run
+# Rotary embedding for the fused RoPE + append line: the scaling factor of the
+# pages' 555k-context example; the base is this library's reading (the pages
+# give none).
+ROPE_SCALE = 2.12
+ROPE_BASE = 1.0e7
 DATASHEET_HBM_GBS = 8000.0
 
 # DRAM traffic of one decode-attention launch, from one ncu capture of the
@@ -403,6 +408,7 @@ def main():
 
     # ---- chunked prefill (65536 cached + 2048 new tokens), tensor-core kernel ----
     prefill = None
+    rope = None
     if not args.no_prefill:
         del dw
         torch.cuda.empty_cache()
@@ -430,6 +436,47 @@ def main():
                    "flop_per_call": flops, "bound": "tensor", "peak_tflops": tf_peak,
                    "peak_kind": tf_kind, "frac": flops / (p_ms * 1e-3) / 1e12 / tf_peak,
                    "device_errors": pdw.err_bits()}
+        # ---- fused RoPE + quantise-append of the same 2048-row chunk ----
+        # (after the prefill timing: it rewrites the chunk's K rotated, then
+        # the plain append writes it back unrotated)
+        try:
+            r = pw.head_dim
+            rows = pw.batch * pw.T
+            cs = torch.empty((int(pw.kv_lens.max()), r // 2, 2), dtype=torch.float32, device=dev)
+            nv.nvkv_rope_table(cs, r, ROPE_BASE, ROPE_SCALE, stream)
+
+            def rope_once():
+                nv.nvkv_append_rope(pdw.cache, pdw.seqs, pdw.k_new, pdw.v_new, pdw.cu_new, rows,
+                                    pw.T, cs, r, stream)
+
+            def plain_once():
+                nv.nvkv_append(pdw.cache, pdw.seqs, pdw.k_new, pdw.v_new, pdw.cu_new, rows, pw.T,
+                               stream)
+
+            for _ in range(3):
+                rope_once()
+                plain_once()
+            re_ = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            torch.cuda.synchronize(dev)
+            re_[0].record(stream)
+            for _ in range(10):
+                rope_once()
+            re_[1].record(stream)
+            for _ in range(10):
+                plain_once()
+            re_[2].record(stream)
+            torch.cuda.synchronize(dev)
+            t_rope = re_[0].elapsed_time(re_[1]) / 10
+            t_plain = re_[1].elapsed_time(re_[2]) / 10
+            # algorithmic bytes: bf16 K and V in, NVFP4 K and V out
+            io = rows * pw.num_kv_heads * pw.head_dim * (2 * 2 + 2 * 0.5625)
+            rope = {"rows": rows, "rotary_dim": r, "base": ROPE_BASE, "scale": ROPE_SCALE,
+                    "ms": t_rope, "gbs": io / (t_rope * 1e-3) / 1e9, "plain_append_ms": t_plain,
+                    "plain_append_gbs": io / (t_plain * 1e-3) / 1e9,
+                    "device_errors": pdw.err_bits()}
+            del cs
+        except Exception as exc:  # a failure here must not cost the headline line
+            rope = {"error": repr(exc)[:300]}
         del pdw
 
     cpu = None
@@ -464,6 +511,7 @@ def main():
             "verify_T6": verify,
             "spill": spill,
             "prefill": prefill,
+            "rope_append": rope,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
