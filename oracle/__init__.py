@@ -84,6 +84,22 @@ def lib():
             L.oracle_quantize_group_f32.argtypes = [vp, vp, vp]
             L.oracle_append_rope.restype = None
             L.oracle_append_rope.argtypes = [vp, i32, i32, vp, i32, vp, i32, vp, vp, vp, i32, vp, i32]
+            L.oracle_k8_quantize_row.restype = None
+            L.oracle_k8_quantize_row.argtypes = [vp, i32, vp, vp]
+            L.oracle_k8_dequant.restype = d
+            L.oracle_k8_dequant.argtypes = [i32, ctypes.c_float]
+            L.oracle_k8v4_page_bytes.restype = ctypes.c_size_t
+            L.oracle_k8v4_page_bytes.argtypes = [i32, i32]
+            L.oracle_append_k8v4.restype = None
+            L.oracle_append_k8v4.argtypes = [vp, i32, i32, vp, i32, vp, i32, vp, vp, vp]
+            L.oracle_k8v4_read_row.restype = None
+            L.oracle_k8v4_read_row.argtypes = [vp, i32, i32, vp, i32, i32, i32, vp]
+            for fn in (L.oracle_attention_rows_k8v4, L.oracle_attention_pool_k8v4):
+                fn.restype = None
+            L.oracle_attention_rows_k8v4.argtypes = [i32, vp, vp, i32, i32, vp, vp, vp, d, vp, vp,
+                                                     vp, i32]
+            L.oracle_attention_pool_k8v4.argtypes = [i32, vp, i32, i32, vp, vp, vp, vp, d, vp, vp,
+                                                     vp, i32]
             L.oracle_attention_rows.restype = None
             L.oracle_attention_rows.argtypes = [i32, vp, vp, i32, i32, vp, vp, vp, d, vp, vp, vp, i32]
             L.oracle_attention_pool.restype = None
@@ -202,8 +218,9 @@ def _ptr_array(arrs) -> np.ndarray:
 
 
 def attention_rows(jobs, num_kv_heads: int, head_dim: int, sm_scale: float,
-                   nthreads: int | None = None):
-    """Exact softmax attention for a list of output rows over a logical cache.
+                   nthreads: int | None = None, k8: bool = False):
+    """Exact softmax attention for a list of output rows over a logical cache
+    (K in NVFP4, or in the 8-bit row format of the K8V4 cache when k8).
 
     jobs: iterable of (k_rows, v_rows, h, n_visible, q) with k_rows / v_rows
     the sequence's bf16 bits [rows][Hkv][D] in position order, h the kv-head,
@@ -229,17 +246,17 @@ def attention_rows(jobs, num_kv_heads: int, head_dim: int, sm_scale: float,
     out = np.zeros((n, head_dim), np.float64)
     lse = np.zeros(n, np.float64)
     psum = np.zeros(n, np.float64)
-    lib().oracle_attention_rows(n, _ptr(kp), _ptr(vp_), num_kv_heads, head_dim, _ptr(hs),
-                                _ptr(nv), _ptr(qp), float(sm_scale), _ptr(out), _ptr(lse),
-                                _ptr(psum), int(nthreads or os.cpu_count() or 1))
+    fn = lib().oracle_attention_rows_k8v4 if k8 else lib().oracle_attention_rows
+    fn(n, _ptr(kp), _ptr(vp_), num_kv_heads, head_dim, _ptr(hs), _ptr(nv), _ptr(qp),
+       float(sm_scale), _ptr(out), _ptr(lse), _ptr(psum), int(nthreads or os.cpu_count() or 1))
     del keep
     return out, lse, psum
 
 
 def attention_pool(pool: np.ndarray, num_kv_heads: int, head_dim: int, jobs, sm_scale: float,
-                   nthreads: int | None = None):
-    """As attention_rows, but the cache is a pool image; jobs are
-    (page_row, h, n_visible, q)."""
+                   nthreads: int | None = None, k8: bool = False):
+    """As attention_rows, but the cache is a pool image (the K8V4 layout when
+    k8); jobs are (page_row, h, n_visible, q)."""
     jobs = list(jobs)
     n = len(jobs)
     keep, prs, qs = [], [], []
@@ -257,9 +274,9 @@ def attention_pool(pool: np.ndarray, num_kv_heads: int, head_dim: int, jobs, sm_
     out = np.zeros((n, head_dim), np.float64)
     lse = np.zeros(n, np.float64)
     psum = np.zeros(n, np.float64)
-    lib().oracle_attention_pool(n, _ptr(pool), num_kv_heads, head_dim, _ptr(pp), _ptr(hs),
-                                _ptr(nv), _ptr(qp), float(sm_scale), _ptr(out), _ptr(lse),
-                                _ptr(psum), int(nthreads or os.cpu_count() or 1))
+    fn = lib().oracle_attention_pool_k8v4 if k8 else lib().oracle_attention_pool
+    fn(n, _ptr(pool), num_kv_heads, head_dim, _ptr(pp), _ptr(hs), _ptr(nv), _ptr(qp),
+       float(sm_scale), _ptr(out), _ptr(lse), _ptr(psum), int(nthreads or os.cpu_count() or 1))
     del keep
     return out, lse, psum
 
@@ -305,3 +322,44 @@ def append_rope(pool: np.ndarray, Hkv: int, D: int, page_table, kv_lens, k_new_b
     lib().oracle_append_rope(_ptr(pool), int(Hkv), int(D), _ptr(pt), int(pt.shape[1]), _ptr(lens),
                              int(pt.shape[0]), _ptr(k), _ptr(v), _ptr(cu), int(rotary_dim), _ptr(cs),
                              int(cs.shape[0]))
+
+
+# --------------------------------------------------------------------------
+# K8V4 cache: 8-bit K rows (E4M3 codes, one float scale per row), NVFP4 V
+# --------------------------------------------------------------------------
+def k8_quantize_row(x_bits) -> tuple[np.ndarray, float]:
+    """One K row (bf16 bits [D]) -> (E4M3 code bytes [D], float32 scale)."""
+    x = _u16(x_bits).reshape(-1)
+    codes = np.zeros(x.shape[0], np.uint8)
+    sc = np.zeros(1, np.float32)
+    lib().oracle_k8_quantize_row(_ptr(x), int(x.shape[0]), _ptr(codes), _ptr(sc))
+    return codes, float(sc[0])
+
+
+def k8_dequant(code: int, scale: float) -> float:
+    return lib().oracle_k8_dequant(int(code), float(np.float32(scale)))
+
+
+def k8v4_page_bytes(num_kv_heads: int, head_dim: int) -> int:
+    return int(lib().oracle_k8v4_page_bytes(num_kv_heads, head_dim))
+
+
+def append_k8v4(pool: np.ndarray, num_kv_heads: int, head_dim: int, page_table, kv_lens, k_new,
+                v_new, cu_new) -> None:
+    """oracle.append for a K8V4 pool image (in place)."""
+    assert pool.dtype == np.uint8 and pool.flags["C_CONTIGUOUS"]
+    pt = np.ascontiguousarray(page_table, np.int32)
+    kl = np.ascontiguousarray(kv_lens, np.int32)
+    cu = np.ascontiguousarray(cu_new, np.int32)
+    k, v = _u16(k_new), _u16(v_new)
+    lib().oracle_append_k8v4(_ptr(pool), num_kv_heads, head_dim, _ptr(pt), pt.shape[1], _ptr(kl),
+                             kl.shape[0], _ptr(k), _ptr(v), _ptr(cu))
+
+
+def k8v4_read_row(pool: np.ndarray, num_kv_heads: int, head_dim: int, page_row, pos: int, h: int,
+                  is_v: bool) -> np.ndarray:
+    pr = np.ascontiguousarray(page_row, np.int32)
+    out = np.zeros(head_dim, np.float64)
+    lib().oracle_k8v4_read_row(_ptr(pool), num_kv_heads, head_dim, _ptr(pr), int(pos), int(h),
+                               int(bool(is_v)), _ptr(out))
+    return out

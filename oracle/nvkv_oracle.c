@@ -435,14 +435,25 @@ typedef struct {
     double *out;   /* [D] */
     double *lse;   /* natural-log sum of exp of the scores, may be NULL */
     double *psum;  /* sum of the normalised weights, may be NULL */
+    int k8;        /* K8V4 cache: K in the 8-bit row format (0: NVFP4 K) */
 } oracle_job;
+
+void oracle_k8v4_read_row(const uint8_t *pool, int Hkv, int D, const int32_t *page_row, int pos,
+                          int h, int is_v, double *out);
+void oracle_k8_qdq_row(const uint16_t *x, int D, double *out);
 
 static void load_row(const oracle_job *jb, int j, int is_v, double *dst) {
     if (jb->pool) {
-        oracle_pool_read_row(jb->pool, jb->Hkv, jb->D, jb->page_row, j, jb->h, is_v, dst);
+        if (jb->k8)
+            oracle_k8v4_read_row(jb->pool, jb->Hkv, jb->D, jb->page_row, j, jb->h, is_v, dst);
+        else
+            oracle_pool_read_row(jb->pool, jb->Hkv, jb->D, jb->page_row, j, jb->h, is_v, dst);
     } else {
         const uint16_t *src = (is_v ? jb->v_rows : jb->k_rows) + ((size_t)j * jb->Hkv + jb->h) * jb->D;
-        oracle_qdq_row(src, jb->D, dst);
+        if (jb->k8 && !is_v)
+            oracle_k8_qdq_row(src, jb->D, dst);
+        else
+            oracle_qdq_row(src, jb->D, dst);
     }
 }
 
@@ -557,6 +568,165 @@ void oracle_attention_pool(int njobs, const uint8_t *pool, int Hkv, int D,
         jobs[i].out = out + (size_t)i * D;
         jobs[i].lse = lse ? lse + i : NULL;
         jobs[i].psum = psum ? psum + i : NULL;
+    }
+    run_jobs(jobs, njobs, nthreads);
+    free(jobs);
+}
+
+/* ------------------------------------------------------------------------ */
+/* K8V4 cache: 8-bit K, NVFP4 V                                              */
+/* ------------------------------------------------------------------------ */
+/* "knoopx/ninfer" README, "Capabilities and limits": the engine stores KV
+ * as BF16, INT8, FP8, NVFP4 or K8V4; the same README's note on its published
+ * measurements names an "FP8 E4M3 row-256" KV.  Reading: K8V4 keeps V in
+ * NVFP4 (as above) and K in that 8-bit format, one float scale per K row of
+ * one token and one kv-head (D elements):
+ *   scale = float(amax / 448)  (float division, round to nearest even),
+ *   code  = E4M3 nearest to float(x / scale)  (float division, then E4M3
+ *           rounding with ties to the even mantissa, saturating at 448),
+ *   scale 0 (an all-zero row) gives codes 0; a magnitude that rounds to 0 is
+ *   code 0 (no negative zero).
+ * Both quotients are taken in float, as a kernel computes them, so the
+ * decisions are the kernel's; the value is E4M3(code) * scale.            */
+void oracle_k8_quantize_row(const uint16_t *x, int D, uint8_t *codes, float *scale) {
+    float amax = 0.0f;
+    for (int d = 0; d < D; ++d) {
+        float a = fabsf((float)oracle_bf16_value(x[d]));
+        if (a > amax) amax = a;
+    }
+    float sc = amax / 448.0f;
+    *scale = sc;
+    for (int d = 0; d < D; ++d) {
+        if (sc == 0.0f) {
+            codes[d] = 0;
+            continue;
+        }
+        float q = (float)oracle_bf16_value(x[d]) / sc;
+        uint8_t mag = oracle_e4m3_round(fabs((double)q));
+        codes[d] = (mag == 0) ? 0 : (uint8_t)((signbit(q) ? 0x80 : 0) | mag);
+    }
+}
+
+double oracle_k8_dequant(int code, float scale) {
+    return oracle_e4m3_value(code) * (double)scale;
+}
+
+void oracle_k8_qdq_row(const uint16_t *x, int D, double *out) {
+    uint8_t codes[512];
+    float sc;
+    oracle_k8_quantize_row(x, D, codes, &sc);
+    for (int d = 0; d < D; ++d) out[d] = oracle_k8_dequant(codes[d], sc);
+}
+
+/* K8V4 page layout: page p, kv-head h block of 25*D + 64 bytes at
+ * (p * Hkv + h) * (25*D + 64):
+ *   [0, 16D)            K codes [16 slots][D], one E4M3 byte per element
+ *   [16D, 16D+64)       K scales [16 slots], IEEE binary32, little-endian
+ *   [16D+64, 24D+64)    V codes [D][8]: byte (d, i) holds slot 2i in its low
+ *                       nibble and slot 2i+1 in its high nibble
+ *   [24D+64, 25D+64)    V scales [D/16][16 slots]                          */
+size_t oracle_k8v4_page_bytes(int Hkv, int D) { return (size_t)Hkv * (25 * (size_t)D + 64); }
+
+static size_t k8v4_base(int page, int h, int Hkv, int D) {
+    return ((size_t)page * Hkv + h) * (25 * (size_t)D + 64);
+}
+
+void oracle_append_k8v4(uint8_t *pool, int Hkv, int D, const int32_t *page_table,
+                        int max_pages_per_seq, const int32_t *kv_lens, int batch,
+                        const uint16_t *k_new, const uint16_t *v_new, const int32_t *cu_new) {
+    uint8_t kc[512], codes[16], sb;
+    float ks;
+    for (int b = 0; b < batch; ++b) {
+        int n = cu_new[b + 1] - cu_new[b];
+        const int32_t *page_row = page_table + (size_t)b * max_pages_per_seq;
+        for (int i = 0; i < n; ++i) {
+            int row = cu_new[b] + i;
+            int pos = kv_lens[b] - n + i;
+            int page = page_row[pos / 16], s = pos % 16;
+            for (int h = 0; h < Hkv; ++h) {
+                size_t base = k8v4_base(page, h, Hkv, D);
+                const uint16_t *kr = k_new + ((size_t)row * Hkv + h) * D;
+                const uint16_t *vr = v_new + ((size_t)row * Hkv + h) * D;
+                oracle_k8_quantize_row(kr, D, kc, &ks);
+                memcpy(pool + base + (size_t)s * D, kc, (size_t)D);
+                memcpy(pool + base + 16 * (size_t)D + 4 * (size_t)s, &ks, 4);
+                for (int g = 0; g < D / 16; ++g) {
+                    oracle_quantize_group(vr + 16 * g, codes, &sb);
+                    for (int e = 0; e < 16; ++e) {
+                        int d = 16 * g + e;
+                        size_t off = base + 16 * (size_t)D + 64 + (size_t)d * 8 + (size_t)(s >> 1);
+                        put_nibble(pool, off, s & 1, codes[e]);
+                    }
+                    pool[base + 24 * (size_t)D + 64 + (size_t)g * 16 + s] = sb;
+                }
+            }
+        }
+    }
+}
+
+void oracle_k8v4_read_row(const uint8_t *pool, int Hkv, int D, const int32_t *page_row, int pos,
+                          int h, int is_v, double *out) {
+    int page = page_row[pos / 16], s = pos % 16;
+    size_t base = k8v4_base(page, h, Hkv, D);
+    if (!is_v) {
+        float ks;
+        memcpy(&ks, pool + base + 16 * (size_t)D + 4 * (size_t)s, 4);
+        for (int d = 0; d < D; ++d) out[d] = oracle_k8_dequant(pool[base + (size_t)s * D + d], ks);
+        return;
+    }
+    for (int d = 0; d < D; ++d) {
+        int code = get_nibble(pool, base + 16 * (size_t)D + 64 + (size_t)d * 8 + (size_t)(s >> 1),
+                              s & 1);
+        int sb = pool[base + 24 * (size_t)D + 64 + (size_t)(d / 16) * 16 + s];
+        out[d] = oracle_dequant(code, sb);
+    }
+}
+
+/* Attention over a K8V4 cache: as oracle_attention_rows / _pool with K in
+ * the 8-bit row format. */
+void oracle_attention_rows_k8v4(int njobs, const uint16_t *const *k_seq,
+                                const uint16_t *const *v_seq, int Hkv, int D, const int32_t *h,
+                                const int32_t *n_visible, const uint16_t *const *q,
+                                double sm_scale, double *out, double *lse, double *psum,
+                                int nthreads) {
+    oracle_job *jobs = (oracle_job *)calloc((size_t)njobs, sizeof(oracle_job));
+    for (int i = 0; i < njobs; ++i) {
+        jobs[i].k_rows = k_seq[i];
+        jobs[i].v_rows = v_seq[i];
+        jobs[i].Hkv = Hkv;
+        jobs[i].D = D;
+        jobs[i].h = h[i];
+        jobs[i].n_visible = n_visible[i];
+        jobs[i].q = q[i];
+        jobs[i].sm_scale = sm_scale;
+        jobs[i].out = out + (size_t)i * D;
+        jobs[i].lse = lse ? lse + i : NULL;
+        jobs[i].psum = psum ? psum + i : NULL;
+        jobs[i].k8 = 1;
+    }
+    run_jobs(jobs, njobs, nthreads);
+    free(jobs);
+}
+
+void oracle_attention_pool_k8v4(int njobs, const uint8_t *pool, int Hkv, int D,
+                                const int32_t *const *page_rows, const int32_t *h,
+                                const int32_t *n_visible, const uint16_t *const *q,
+                                double sm_scale, double *out, double *lse, double *psum,
+                                int nthreads) {
+    oracle_job *jobs = (oracle_job *)calloc((size_t)njobs, sizeof(oracle_job));
+    for (int i = 0; i < njobs; ++i) {
+        jobs[i].pool = pool;
+        jobs[i].page_row = page_rows[i];
+        jobs[i].Hkv = Hkv;
+        jobs[i].D = D;
+        jobs[i].h = h[i];
+        jobs[i].n_visible = n_visible[i];
+        jobs[i].q = q[i];
+        jobs[i].sm_scale = sm_scale;
+        jobs[i].out = out + (size_t)i * D;
+        jobs[i].lse = lse ? lse + i : NULL;
+        jobs[i].psum = psum ? psum + i : NULL;
+        jobs[i].k8 = 1;
     }
     run_jobs(jobs, njobs, nthreads);
     free(jobs);
