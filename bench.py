@@ -225,6 +225,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--no-prefill", action="store_true", help="skip the chunked-prefill line")
     ap.add_argument("--no-spill", action="store_true", help="skip the page spill/restore line")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="skip the CUDA-graph replay line (a step captured once, replayed)")
     ap.add_argument("--no-verify", action="store_true",
                     help="skip the T=6 MTP-verify line (measured on the T=1 pool)")
     ap.add_argument("--ctx", type=str, default=None,
@@ -485,6 +487,47 @@ def main():
         cpu = {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc,
                "seconds": dt}
 
+    # ---- decode step captured in a CUDA Graph and replayed (the serving mode
+    # of the pages' engine), on its own 3 x 60k context, last so that nothing
+    # measured above can depend on it ----
+    graph = None
+    if not args.no_graph:
+        try:
+            gw = W.long_context(T=1, ctx=(60000, 60000, 60000))
+            gdw = DeviceWorkload(gw, dev, fill=None, num_splits=args.num_splits)
+            gdw.fill_context()
+            gdw.load_step_inputs()
+            for _ in range(3):
+                gdw.step()
+            torch.cuda.synchronize(dev)
+            direct_out = gdw.out.clone()
+            cg = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(cg):
+                gdw.step()
+            cg.replay()
+            torch.cuda.synchronize(dev)
+            same = bool(torch.equal(gdw.out, direct_out))
+            reps = 200
+            ge = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            cur = torch.cuda.current_stream(dev)
+            ge[0].record(cur)
+            for _ in range(reps):
+                gdw.step()
+            ge[1].record(cur)
+            for _ in range(reps):
+                cg.replay()
+            ge[2].record(cur)
+            torch.cuda.synchronize(dev)
+            d_ms = ge[0].elapsed_time(ge[1]) / reps
+            r_ms = ge[1].elapsed_time(ge[2]) / reps
+            kvb = gw.kv_bytes_per_step()
+            graph = {"workload": gw.name, "direct_ms": d_ms, "replay_ms": r_ms,
+                     "direct_gbs": kvb / (d_ms * 1e-3) / 1e9, "replay_gbs": kvb / (r_ms * 1e-3) / 1e9,
+                     "replay_equals_direct": same, "device_errors": gdw.err_bits()}
+            del cg, gdw
+        except Exception as exc:  # a failure here must not cost the lines above
+            graph = {"error": repr(exc)[:300]}
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
@@ -512,6 +555,7 @@ def main():
             "spill": spill,
             "prefill": prefill,
             "rope_append": rope,
+            "cuda_graph": graph,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
