@@ -47,6 +47,7 @@ REF_BUDGET_S = 90.0  # oracle seconds of a whole --impl reference run
 ROPE_SCALE = 2.12
 ROPE_BASE = 1.0e7
 DATASHEET_HBM_GBS = 8000.0
+DATASHEET_BF16_TFLOPS = 2250.0  # dense
 
 # DRAM traffic of one decode-attention launch, from one ncu capture of the
 # kernel source with this SHA-256 (profiles/decode_tc_long_ctx_3x60k_T1_full.md:
@@ -437,6 +438,7 @@ def main():
         prefill = {"workload": pw.name, "ms": p_ms, "tflops": flops / (p_ms * 1e-3) / 1e12,
                    "flop_per_call": flops, "bound": "tensor", "peak_tflops": tf_peak,
                    "peak_kind": tf_kind, "frac": flops / (p_ms * 1e-3) / 1e12 / tf_peak,
+                   "frac_datasheet": flops / (p_ms * 1e-3) / 1e12 / DATASHEET_BF16_TFLOPS,
                    "device_errors": pdw.err_bits()}
         # ---- fused RoPE + quantise-append of the same 2048-row chunk ----
         # (after the prefill timing: it rewrites the chunk's K rotated, then
