@@ -382,11 +382,12 @@ def main():
             nv.nvkv_pages_restore(dw.cache, sp_pages, sp_slots, arena, dw.err, stream)
         se[2].record(stream)
         torch.cuda.synchronize(dev)
-        d2h = se[0].elapsed_time(se[1]) / reps
-        h2d = se[1].elapsed_time(se[2]) / reps
+        spill_ms = se[0].elapsed_time(se[1]) / reps
+        restore_ms = se[1].elapsed_time(se[2]) / reps
         spill = {"pages": n_sp, "bytes": n_sp * pb, "arena": "pinned host",
-                 "spill_ms": d2h, "spill_gbs": n_sp * pb / (d2h * 1e-3) / 1e9,
-                 "restore_ms": h2d, "restore_gbs": n_sp * pb / (h2d * 1e-3) / 1e9,
+                 "spill_ms": spill_ms, "spill_gbs": n_sp * pb / (spill_ms * 1e-3) / 1e9,
+                 "restore_ms": restore_ms,
+                 "restore_gbs": n_sp * pb / (restore_ms * 1e-3) / 1e9,
                  "device_errors": dw.err_bits()}
         del arena
 

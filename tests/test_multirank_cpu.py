@@ -74,3 +74,42 @@ def test_decode_traffic_tracks_the_captured_source(tmp_path, monkeypatch):
                                   cap["kv_bytes"])
     monkeypatch.setitem(cap, "sha256", "0" * 64)
     assert bench.decode_traffic(kv) is None
+
+
+def test_reference_arm_rank0_prints_one_contract_line():
+    import json
+    env = dict(os.environ, RANK="0", WORLD_SIZE="1", LOCAL_RANK="0")
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference",
+                        "--steps", "2", "--warmup", "3", "--ref-ctx", "512"],
+                       capture_output=True, text=True, timeout=300, env=env, cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["steps"] == 2 and d["warmup"] == 3
+    assert d["value"] > 0 and d["unit"] == "GB/s" and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0,
+                        "d2h_bytes_per_step": 0}
+    assert "512 of" in d["config"]["sample"]
+
+
+def test_bench_e2e_byte_counts_are_assigned_once():
+    """The e2e line reports the bytes copied each step; no later measurement
+    in the same function may reuse those names for something else."""
+    import ast
+    tree = ast.parse(open(os.path.join(ROOT, "bench.py")).read())
+    main = next(n for n in tree.body if isinstance(n, ast.FunctionDef) and n.name == "main")
+    stores = []
+
+    def visit(node):  # main's own scope: nested functions have their own
+        for c in ast.iter_child_nodes(node):
+            if isinstance(c, (ast.FunctionDef, ast.Lambda)):
+                continue
+            if isinstance(c, ast.Name) and isinstance(c.ctx, ast.Store):
+                stores.append(c.id)
+            visit(c)
+
+    visit(main)
+    for name in ("h2d", "d2h", "value", "ms", "kv_bytes", "e2e_ms", "decode_gbs"):
+        assert stores.count(name) == 1, name
