@@ -243,6 +243,45 @@ nvkv_status nvkv_pages_restore(const nvkv_cache *cache, const int32_t *page_ids,
                                const int32_t *slot_ids, int32_t n, const void *arena,
                                int64_t num_slots, int32_t *err_word, nvkv_stream_t stream);
 
+/* K8V4 cache: 8-bit K, NVFP4 V.  The "knoopx/ninfer" README, "Capabilities
+ * and limits", lists K8V4 among its KV storage formats and its note on the
+ * published measurements names an E4M3 "row-256" KV; the pages fix no
+ * layout.  This library's reading: K rows in E4M3 with one fp32 scale per
+ * row of one token and one kv-head, V exactly as in the NVFP4 cache.
+ *   K scale = amax / 448 in fp32 (round to nearest even); K code = the E4M3
+ *   value nearest to x / scale computed in fp32 (ties to the even mantissa,
+ *   saturating at 448); an all-zero row has scale 0 and codes 0; a
+ *   magnitude that rounds to 0 is stored as 0x00.  Value = E4M3(code) * scale.
+ * Page layout: page p starts at pool + p * nvkv_k8v4_page_bytes(Hkv, D);
+ * kv-head h owns the (25*D + 64)-byte block at offset h * (25*D + 64):
+ *   [0,        16D)     K codes  [16 slots][D], one E4M3 byte per element
+ *   [16D,      16D+64)  K scales [16 slots], fp32 little-endian
+ *   [16D+64,   24D+64)  V codes  [D][8], as the NVFP4 V codes
+ *   [24D+64,   25D+64)  V scales [D/16][16 slots], as the NVFP4 V scales
+ * A K8V4 cache is an nvkv_cache whose pool holds num_pages *
+ * nvkv_k8v4_page_bytes() bytes; it is used only with the *_k8v4 calls
+ * (the other calls read and write the NVFP4 layout).  Each call below has
+ * the arguments, layouts, checks and error behaviour of its NVFP4
+ * counterpart:
+ *   nvkv_append_k8v4       ~ nvkv_append
+ *   nvkv_decode_attn_k8v4  ~ nvkv_decode_attn (same workspace size and
+ *                            split plan; merge with nvkv_combine)
+ *   nvkv_prefill_attn_k8v4 ~ nvkv_prefill_attn
+ * The attention calls run on CUDA cores (one warp per query row).
+ * nvkv_k8v4_page_bytes returns 0 for non-positive arguments. */
+size_t nvkv_k8v4_page_bytes(int32_t num_kv_heads, int32_t head_dim);
+nvkv_status nvkv_append_k8v4(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *k_new,
+                             const void *v_new, const int32_t *cu_new, int32_t total_new,
+                             int32_t max_new, nvkv_stream_t stream);
+nvkv_status nvkv_decode_attn_k8v4(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *q,
+                                  int32_t T, int32_t num_q_heads, float sm_scale,
+                                  int32_t num_splits, void *workspace, size_t workspace_bytes,
+                                  nvkv_stream_t stream);
+nvkv_status nvkv_prefill_attn_k8v4(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *q,
+                                   const int32_t *cu_q, int32_t total_q, int32_t max_q,
+                                   int32_t num_q_heads, float sm_scale, void *out,
+                                   nvkv_stream_t stream);
+
 /* Static description of a status code. */
 const char *nvkv_status_string(nvkv_status status);
 

@@ -22,7 +22,9 @@ __all__ = [
     "nvkv_page_bytes", "nvkv_default_num_splits", "nvkv_decode_workspace_bytes",
     "nvkv_split_plan", "nvkv_append", "nvkv_decode_attn", "nvkv_combine",
     "nvkv_prefill_attn", "nvkv_status_string", "nvkv_decode_attn_static",
-    "nvkv_decode_static_scratch_bytes",
+    "nvkv_decode_static_scratch_bytes", "nvkv_rope_table", "nvkv_append_rope",
+    "nvkv_pages_spill", "nvkv_pages_restore", "nvkv_k8v4_page_bytes", "nvkv_append_k8v4",
+    "nvkv_decode_attn_k8v4", "nvkv_prefill_attn_k8v4",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -78,6 +80,10 @@ def library():
             "nvkv_append_rope": (ctypes.c_int, [cp, sp, vp, vp, vp, i32, i32, vp, i32, i32, vp]),
             "nvkv_pages_spill": (ctypes.c_int, [cp, vp, vp, i32, vp, ctypes.c_int64, vp, vp]),
             "nvkv_pages_restore": (ctypes.c_int, [cp, vp, vp, i32, vp, ctypes.c_int64, vp, vp]),
+            "nvkv_k8v4_page_bytes": (sz, [i32, i32]),
+            "nvkv_append_k8v4": (ctypes.c_int, [cp, sp, vp, vp, vp, i32, i32, vp]),
+            "nvkv_decode_attn_k8v4": (ctypes.c_int, [cp, sp, vp, i32, i32, f32, i32, vp, sz, vp]),
+            "nvkv_prefill_attn_k8v4": (ctypes.c_int, [cp, sp, vp, vp, i32, i32, i32, f32, vp, vp]),
             "nvkv_status_string": (ctypes.c_char_p, [ctypes.c_int]),
         }
         for name, (res, args) in sig.items():
@@ -117,24 +123,45 @@ def _stream(stream) -> int:
     return int(stream)
 
 
-class Cache:
-    """The paged NVFP4 pool: ``pool`` is a uint8 CUDA tensor of
-    num_pages * nvkv_page_bytes(num_kv_heads, head_dim) bytes."""
+KV_FORMATS = ("nvfp4", "k8v4")
 
-    def __init__(self, pool: torch.Tensor, num_pages: int, num_kv_heads: int, head_dim: int):
+
+def _page_bytes_of(kv_format: str, num_kv_heads: int, head_dim: int) -> int:
+    if kv_format == "nvfp4":
+        return nvkv_page_bytes(num_kv_heads, head_dim)
+    if kv_format == "k8v4":
+        return nvkv_k8v4_page_bytes(num_kv_heads, head_dim)
+    raise ValueError(f"kv_format must be one of {KV_FORMATS}, got {kv_format!r}")
+
+
+class Cache:
+    """The paged pool: ``pool`` is a uint8 CUDA tensor of num_pages pages of
+    nvkv_page_bytes(num_kv_heads, head_dim) bytes (kv_format "nvfp4") or
+    nvkv_k8v4_page_bytes(...) bytes ("k8v4": 8-bit K, NVFP4 V).  A K8V4
+    cache is used only with the *_k8v4 calls."""
+
+    def __init__(self, pool: torch.Tensor, num_pages: int, num_kv_heads: int, head_dim: int,
+                 kv_format: str = "nvfp4"):
         self.pool, self.num_pages, self.num_kv_heads, self.head_dim = pool, num_pages, num_kv_heads, head_dim
-        need = num_pages * nvkv_page_bytes(num_kv_heads, head_dim)
+        self.kv_format = kv_format
+        need = num_pages * _page_bytes_of(kv_format, num_kv_heads, head_dim)
         if pool.numel() < need:
             raise ValueError(f"pool has {pool.numel()} bytes, needs {need}")
         self._c = _CacheC(_dev(pool, torch.uint8, "pool"), num_pages, num_kv_heads, head_dim)
 
     @staticmethod
-    def allocate(num_pages: int, num_kv_heads: int, head_dim: int, device="cuda", fill=None):
-        n = num_pages * nvkv_page_bytes(num_kv_heads, head_dim)
+    def allocate(num_pages: int, num_kv_heads: int, head_dim: int, device="cuda", fill=None,
+                 kv_format: str = "nvfp4"):
+        n = num_pages * _page_bytes_of(kv_format, num_kv_heads, head_dim)
         pool = torch.empty(n, dtype=torch.uint8, device=device)
         if fill is not None:
             pool.fill_(fill)
-        return Cache(pool, num_pages, num_kv_heads, head_dim)
+        return Cache(pool, num_pages, num_kv_heads, head_dim, kv_format)
+
+
+def _fmt(cache: "Cache", want: str, what: str) -> None:
+    if cache.kv_format != want:
+        raise ValueError(f"{what} needs a {want} cache, got a {cache.kv_format} cache")
 
 
 class Seqs:
@@ -184,6 +211,7 @@ def nvkv_split_plan(kv_lens_host, num_kv_heads: int, num_splits: int):
 
 def nvkv_append(cache: Cache, seqs: Seqs, k_new: torch.Tensor, v_new: torch.Tensor,
                 cu_new: torch.Tensor, total_new: int, max_new: int, stream=None) -> None:
+    _fmt(cache, "nvfp4", "nvkv_append")
     _check(library().nvkv_append(
         ctypes.byref(cache._c), ctypes.byref(seqs._c), _dev(k_new, torch.bfloat16, "k_new"),
         _dev(v_new, torch.bfloat16, "v_new"), _dev(cu_new, torch.int32, "cu_new"), int(total_new),
@@ -205,6 +233,7 @@ def nvkv_append_rope(cache: Cache, seqs: Seqs, k_new: torch.Tensor, v_new: torch
                      cu_new: torch.Tensor, total_new: int, max_new: int, rope_cs: torch.Tensor,
                      rotary_dim: int, stream=None) -> None:
     """nvkv_append with K rotated at its position by the rope_cs table."""
+    _fmt(cache, "nvfp4", "nvkv_append_rope")
     _check(library().nvkv_append_rope(
         ctypes.byref(cache._c), ctypes.byref(seqs._c), _dev(k_new, torch.bfloat16, "k_new"),
         _dev(v_new, torch.bfloat16, "v_new"), _dev(cu_new, torch.int32, "cu_new"), int(total_new),
@@ -215,6 +244,7 @@ def nvkv_append_rope(cache: Cache, seqs: Seqs, k_new: torch.Tensor, v_new: torch
 def nvkv_decode_attn(cache: Cache, seqs: Seqs, q: torch.Tensor, T: int, num_q_heads: int,
                      sm_scale: float, num_splits: int, workspace: torch.Tensor,
                      stream=None) -> None:
+    _fmt(cache, "nvfp4", "nvkv_decode_attn")
     _check(library().nvkv_decode_attn(
         ctypes.byref(cache._c), ctypes.byref(seqs._c), _dev(q, torch.bfloat16, "q"), int(T),
         int(num_q_heads), float(sm_scale), int(num_splits), _dev(workspace, torch.uint8, "workspace"),
@@ -233,6 +263,7 @@ def nvkv_combine(seqs: Seqs, workspace: torch.Tensor, T: int, num_q_heads: int,
 def nvkv_prefill_attn(cache: Cache, seqs: Seqs, q: torch.Tensor, cu_q: torch.Tensor,
                       total_q: int, max_q: int, num_q_heads: int, sm_scale: float,
                       out: torch.Tensor, stream=None) -> None:
+    _fmt(cache, "nvfp4", "nvkv_prefill_attn")
     _check(library().nvkv_prefill_attn(
         ctypes.byref(cache._c), ctypes.byref(seqs._c), _dev(q, torch.bfloat16, "q"),
         _dev(cu_q, torch.int32, "cu_q"), int(total_q), int(max_q), int(num_q_heads),
@@ -248,6 +279,7 @@ def nvkv_decode_attn_static(cache: Cache, seqs: Seqs, q: torch.Tensor, T: int, n
                             stream=None) -> None:
     """Decode attention + combine with the library's own device scratch (no
     workspace argument, nothing allocated); see include/nvkv.h."""
+    _fmt(cache, "nvfp4", "nvkv_decode_attn_static")
     _check(library().nvkv_decode_attn_static(
         ctypes.byref(cache._c), ctypes.byref(seqs._c), _dev(q, torch.bfloat16, "q"), int(T),
         int(num_q_heads), float(sm_scale), int(num_splits), _dev(out, torch.bfloat16, "out"),
@@ -267,6 +299,7 @@ def _dev_or_pinned(t: torch.Tensor, dtype: torch.dtype, name: str) -> int:
 
 
 def _pages_args(cache: Cache, page_ids, slot_ids, arena, err_word):
+    _fmt(cache, "nvfp4", "nvkv_pages_spill / nvkv_pages_restore")
     n = page_ids.numel()
     if slot_ids.numel() != n:
         raise ValueError("page_ids and slot_ids must have the same length")
@@ -291,3 +324,39 @@ def nvkv_pages_restore(cache: Cache, page_ids: torch.Tensor, slot_ids: torch.Ten
     """Arena slot slot_ids[i] -> pool page page_ids[i]."""
     _check(library().nvkv_pages_restore(*_pages_args(cache, page_ids, slot_ids, arena, err_word),
                                         _stream(stream)), "nvkv_pages_restore")
+
+
+# ---- K8V4 cache (8-bit K rows with one fp32 scale per row, NVFP4 V) --------
+
+def nvkv_k8v4_page_bytes(num_kv_heads: int, head_dim: int) -> int:
+    return int(library().nvkv_k8v4_page_bytes(num_kv_heads, head_dim))
+
+
+def nvkv_append_k8v4(cache: Cache, seqs: Seqs, k_new: torch.Tensor, v_new: torch.Tensor,
+                     cu_new: torch.Tensor, total_new: int, max_new: int, stream=None) -> None:
+    _fmt(cache, "k8v4", "nvkv_append_k8v4")
+    _check(library().nvkv_append_k8v4(
+        ctypes.byref(cache._c), ctypes.byref(seqs._c), _dev(k_new, torch.bfloat16, "k_new"),
+        _dev(v_new, torch.bfloat16, "v_new"), _dev(cu_new, torch.int32, "cu_new"), int(total_new),
+        int(max_new), _stream(stream)), "nvkv_append_k8v4")
+
+
+def nvkv_decode_attn_k8v4(cache: Cache, seqs: Seqs, q: torch.Tensor, T: int, num_q_heads: int,
+                          sm_scale: float, num_splits: int, workspace: torch.Tensor,
+                          stream=None) -> None:
+    """Split-K partial results over a K8V4 cache; merge with nvkv_combine."""
+    _fmt(cache, "k8v4", "nvkv_decode_attn_k8v4")
+    _check(library().nvkv_decode_attn_k8v4(
+        ctypes.byref(cache._c), ctypes.byref(seqs._c), _dev(q, torch.bfloat16, "q"), int(T),
+        int(num_q_heads), float(sm_scale), int(num_splits), _dev(workspace, torch.uint8, "workspace"),
+        workspace.numel(), _stream(stream)), "nvkv_decode_attn_k8v4")
+
+
+def nvkv_prefill_attn_k8v4(cache: Cache, seqs: Seqs, q: torch.Tensor, cu_q: torch.Tensor,
+                           total_q: int, max_q: int, num_q_heads: int, sm_scale: float,
+                           out: torch.Tensor, stream=None) -> None:
+    _fmt(cache, "k8v4", "nvkv_prefill_attn_k8v4")
+    _check(library().nvkv_prefill_attn_k8v4(
+        ctypes.byref(cache._c), ctypes.byref(seqs._c), _dev(q, torch.bfloat16, "q"),
+        _dev(cu_q, torch.int32, "cu_q"), int(total_q), int(max_q), int(num_q_heads),
+        float(sm_scale), _dev(out, torch.bfloat16, "out"), _stream(stream)), "nvkv_prefill_attn_k8v4")

@@ -11,8 +11,10 @@ namespace nvkv {
 cudaError_t launch_append(const nvkv_cache &, const nvkv_seqs &, const void *, const void *,
                           const int32_t *, int, int, const float *, int, int, cudaStream_t);
 cudaError_t launch_rope_table(float *, int, int, double, double, cudaStream_t);
+cudaError_t launch_append_k8v4(const nvkv_cache &, const nvkv_seqs &, const void *, const void *,
+                               const int32_t *, int, int, cudaStream_t);
 cudaError_t launch_decode_simt(const nvkv_cache &, const nvkv_seqs &, const void *, int, int,
-                               float, int, float *, float *, cudaStream_t);
+                               float, int, float *, float *, cudaStream_t, bool);
 bool decode_tc_supported(const nvkv_cache &, int, int);
 cudaError_t launch_decode_tc(const nvkv_cache &, const nvkv_seqs &, const void *, int, int, float,
                              int, float *, float *, cudaStream_t);
@@ -22,7 +24,7 @@ cudaError_t launch_prefill_tc(const nvkv_cache &, const nvkv_seqs &, const void 
 cudaError_t launch_combine(const nvkv_seqs &, const void *, const void *, int, int, int, int, int,
                            void *, cudaStream_t);
 cudaError_t launch_prefill_simt(const nvkv_cache &, const nvkv_seqs &, const void *,
-                                const int32_t *, int, int, float, void *, cudaStream_t);
+                                const int32_t *, int, int, float, void *, cudaStream_t, bool);
 cudaError_t launch_page_copy(const uint8_t *, int64_t, uint8_t *, int64_t, const int32_t *,
                              const int32_t *, int, int64_t, int32_t *, cudaStream_t);
 }  // namespace nvkv
@@ -115,6 +117,45 @@ nvkv_status pages_move(const nvkv_cache *cache, const int32_t *page_ids, const i
                                               p32, n, pb, err_word, s));
 }
 
+
+// Checks shared by the decode entry points of both cache formats; on
+// success `a` holds the resolved split count and the workspace regions.
+struct DecodeArgs {
+  int S = 0;
+  float *ws_o = nullptr, *ws_lse = nullptr;
+};
+
+nvkv_status check_decode(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *q, int32_t T,
+                         int32_t num_q_heads, float sm_scale, int32_t num_splits, void *workspace,
+                         size_t workspace_bytes, DecodeArgs &a) {
+  nvkv_status st = check_cache(cache);
+  if (st != NVKV_OK) return st;
+  if ((st = check_seqs(seqs)) != NVKV_OK) return st;
+  if ((st = check_heads(num_q_heads, cache->num_kv_heads, cache->head_dim, T)) != NVKV_OK) return st;
+  if (!q || !aligned16(q) || !std::isfinite(sm_scale) || num_splits < 0) return NVKV_ERR_INVALID_ARG;
+  a.S = resolve_splits(num_splits);
+  const WorkspaceLayout w = layout(seqs->batch, T, num_q_heads, cache->num_kv_heads,
+                                   cache->head_dim, a.S);
+  if (!workspace || !aligned16(workspace) || workspace_bytes < w.total) return NVKV_ERR_WORKSPACE;
+  a.ws_o = static_cast<float *>(workspace);
+  a.ws_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) + w.lse_off);
+  return NVKV_OK;
+}
+
+// Checks shared by the prefill entry points (NVKV_OK with total_q == 0
+// means there is nothing to launch).
+nvkv_status check_prefill(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *q,
+                          const int32_t *cu_q, int32_t total_q, int32_t max_q,
+                          int32_t num_q_heads, float sm_scale, const void *out) {
+  nvkv_status st = check_cache(cache);
+  if (st != NVKV_OK) return st;
+  if ((st = check_seqs(seqs)) != NVKV_OK) return st;
+  if (num_q_heads <= 0 || num_q_heads % cache->num_kv_heads != 0) return NVKV_ERR_INVALID_ARG;
+  if (total_q < 0 || max_q < 0 || !std::isfinite(sm_scale)) return NVKV_ERR_INVALID_ARG;
+  if (total_q == 0) return NVKV_OK;
+  if (!q || !cu_q || !out || !aligned16(q) || !aligned16(out)) return NVKV_ERR_INVALID_ARG;
+  return NVKV_OK;
+}
 
 // NVKV_DECODE_KERNEL=simt forces the CUDA-core decode and prefill kernels
 // (used by the tests to cross-check the two kernel families on the same
@@ -225,23 +266,16 @@ nvkv_status nvkv_append_rope(const nvkv_cache *cache, const nvkv_seqs *seqs, con
 nvkv_status nvkv_decode_attn(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *q,
                              int32_t T, int32_t num_q_heads, float sm_scale, int32_t num_splits,
                              void *workspace, size_t workspace_bytes, nvkv_stream_t stream) {
-  nvkv_status st = check_cache(cache);
+  DecodeArgs a;
+  const nvkv_status st = check_decode(cache, seqs, q, T, num_q_heads, sm_scale, num_splits,
+                                      workspace, workspace_bytes, a);
   if (st != NVKV_OK) return st;
-  if ((st = check_seqs(seqs)) != NVKV_OK) return st;
-  if ((st = check_heads(num_q_heads, cache->num_kv_heads, cache->head_dim, T)) != NVKV_OK) return st;
-  if (!q || !aligned16(q) || !std::isfinite(sm_scale) || num_splits < 0) return NVKV_ERR_INVALID_ARG;
-  const int S = resolve_splits(num_splits);
-  const WorkspaceLayout w = layout(seqs->batch, T, num_q_heads, cache->num_kv_heads,
-                                   cache->head_dim, S);
-  if (!workspace || !aligned16(workspace) || workspace_bytes < w.total) return NVKV_ERR_WORKSPACE;
-  float *ws_o = static_cast<float *>(workspace);
-  float *ws_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) + w.lse_off);
   cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
   if (!force_simt() && decode_tc_supported(*cache, T, num_q_heads))
     return cuda_status(
-        launch_decode_tc(*cache, *seqs, q, T, num_q_heads, sm_scale, S, ws_o, ws_lse, st_));
-  return cuda_status(
-      launch_decode_simt(*cache, *seqs, q, T, num_q_heads, sm_scale, S, ws_o, ws_lse, st_));
+        launch_decode_tc(*cache, *seqs, q, T, num_q_heads, sm_scale, a.S, a.ws_o, a.ws_lse, st_));
+  return cuda_status(launch_decode_simt(*cache, *seqs, q, T, num_q_heads, sm_scale, a.S, a.ws_o,
+                                        a.ws_lse, st_, false));
 }
 
 nvkv_status nvkv_combine(const nvkv_seqs *seqs, const void *workspace, int32_t T,
@@ -263,19 +297,57 @@ nvkv_status nvkv_prefill_attn(const nvkv_cache *cache, const nvkv_seqs *seqs, co
                               const int32_t *cu_q, int32_t total_q, int32_t max_q,
                               int32_t num_q_heads, float sm_scale, void *out,
                               nvkv_stream_t stream) {
-  nvkv_status st = check_cache(cache);
-  if (st != NVKV_OK) return st;
-  if ((st = check_seqs(seqs)) != NVKV_OK) return st;
-  if (num_q_heads <= 0 || num_q_heads % cache->num_kv_heads != 0) return NVKV_ERR_INVALID_ARG;
-  if (total_q < 0 || max_q < 0 || !std::isfinite(sm_scale)) return NVKV_ERR_INVALID_ARG;
-  if (total_q == 0) return NVKV_OK;
-  if (!q || !cu_q || !out || !aligned16(q) || !aligned16(out)) return NVKV_ERR_INVALID_ARG;
+  const nvkv_status st =
+      check_prefill(cache, seqs, q, cu_q, total_q, max_q, num_q_heads, sm_scale, out);
+  if (st != NVKV_OK || total_q == 0) return st;
   cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
   if (!force_simt() && prefill_tc_supported(*cache))
     return cuda_status(launch_prefill_tc(*cache, *seqs, q, cu_q, total_q, max_q, num_q_heads,
                                          sm_scale, out, st_));
-  return cuda_status(
-      launch_prefill_simt(*cache, *seqs, q, cu_q, total_q, num_q_heads, sm_scale, out, st_));
+  return cuda_status(launch_prefill_simt(*cache, *seqs, q, cu_q, total_q, num_q_heads, sm_scale,
+                                         out, st_, false));
+}
+
+size_t nvkv_k8v4_page_bytes(int32_t num_kv_heads, int32_t head_dim) {
+  if (num_kv_heads <= 0 || head_dim <= 0) return 0;
+  return (size_t)num_kv_heads * (25 * (size_t)head_dim + 64);
+}
+
+nvkv_status nvkv_append_k8v4(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *k_new,
+                             const void *v_new, const int32_t *cu_new, int32_t total_new,
+                             int32_t max_new, nvkv_stream_t stream) {
+  nvkv_status st = check_cache(cache);
+  if (st != NVKV_OK) return st;
+  if ((st = check_seqs(seqs)) != NVKV_OK) return st;
+  if (total_new < 0 || max_new < 0) return NVKV_ERR_INVALID_ARG;
+  if (total_new == 0 || max_new == 0) return NVKV_OK;
+  if (!k_new || !v_new || !cu_new || !aligned16(k_new) || !aligned16(v_new))
+    return NVKV_ERR_INVALID_ARG;
+  return cuda_status(launch_append_k8v4(*cache, *seqs, k_new, v_new, cu_new, total_new, max_new,
+                                        reinterpret_cast<cudaStream_t>(stream)));
+}
+
+nvkv_status nvkv_decode_attn_k8v4(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *q,
+                                  int32_t T, int32_t num_q_heads, float sm_scale,
+                                  int32_t num_splits, void *workspace, size_t workspace_bytes,
+                                  nvkv_stream_t stream) {
+  DecodeArgs a;
+  const nvkv_status st = check_decode(cache, seqs, q, T, num_q_heads, sm_scale, num_splits,
+                                      workspace, workspace_bytes, a);
+  if (st != NVKV_OK) return st;
+  return cuda_status(launch_decode_simt(*cache, *seqs, q, T, num_q_heads, sm_scale, a.S, a.ws_o,
+                                        a.ws_lse, reinterpret_cast<cudaStream_t>(stream), true));
+}
+
+nvkv_status nvkv_prefill_attn_k8v4(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *q,
+                                   const int32_t *cu_q, int32_t total_q, int32_t max_q,
+                                   int32_t num_q_heads, float sm_scale, void *out,
+                                   nvkv_stream_t stream) {
+  const nvkv_status st =
+      check_prefill(cache, seqs, q, cu_q, total_q, max_q, num_q_heads, sm_scale, out);
+  if (st != NVKV_OK || total_q == 0) return st;
+  return cuda_status(launch_prefill_simt(*cache, *seqs, q, cu_q, total_q, num_q_heads, sm_scale,
+                                         out, reinterpret_cast<cudaStream_t>(stream), true));
 }
 
 nvkv_status nvkv_pages_spill(const nvkv_cache *cache, const int32_t *page_ids,

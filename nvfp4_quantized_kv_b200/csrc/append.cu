@@ -206,6 +206,138 @@ cudaError_t launch_append(const nvkv_cache &c, const nvkv_seqs &s, const void *k
   return cudaGetLastError();
 }
 
+// ---------------------------------------------------------------------------
+// K8V4 cache (the "knoopx/ninfer" README, "Capabilities and limits", lists
+// K8V4 among its KV storage formats; the same README's note on its published
+// measurements names an E4M3 "row-256" KV).  K: one float scale per row of
+// one token and one kv-head, scale = amax / 448 (fp32 division), and one
+// E4M3 byte per element, the E4M3 value nearest to x / scale (fp32
+// division, ties to the even mantissa, saturating at 448; a magnitude that
+// rounds to zero is stored as +0; an all-zero row has scale 0 and codes 0).
+// V: NVFP4 groups exactly as in the NVFP4 cache.
+//
+// Work item = (sequence b, slot pair, kv-head h, group g) as in
+// append_kernel.  The D/16 items of one (pair, h) are adjacent lanes of one
+// warp (D/16 is 8 or 16 and divides the block size), so the row maximum of
+// K is a shuffle reduction over those lanes.  Every lane of a warp takes
+// part in the shuffles: lanes without work contribute 0 and write nothing,
+// and the only early exits are uniform over the block.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t e4m3_byte(float q) {
+  const uint32_t c = __nv_cvt_float_to_fp8(q, __NV_SATFINITE, __NV_E4M3);
+  return (c & 0x7fu) ? c : 0u;
+}
+
+__global__ void __launch_bounds__(256)
+append_k8v4_kernel(uint8_t *__restrict__ pool, int num_pages, int Hkv, int D,
+                   const int32_t *__restrict__ page_table, int max_pages,
+                   const int32_t *__restrict__ kv_lens, int max_kv_len,
+                   const __nv_bfloat16 *__restrict__ k_new,
+                   const __nv_bfloat16 *__restrict__ v_new, const int32_t *__restrict__ cu_new,
+                   int total_new, int max_new, int max_pairs, int32_t *err) {
+  const int b = blockIdx.y;
+  const int groups = D / kGroup;
+  const int per_pair = Hkv * groups;
+  const int item = blockIdx.x * blockDim.x + threadIdx.x;
+  const int pair = item / per_pair;
+  const int h = (item % per_pair) / groups;
+  const int g = item % groups;
+
+  // Checks of the sequence: the same for every thread of the block.
+  const int row0 = cu_new[b];
+  const int n = cu_new[b + 1] - row0;
+  const int len = kv_lens[b];
+  if (n <= 0) return;
+  const int first = len - n;
+  if (row0 < 0 || row0 + n > total_new || n > max_new || first < 0 || len > max_kv_len ||
+      len > max_pages * kPageTokens) {
+    if (item == 0) report(err, NVKV_DEVERR_LENGTH);
+    return;
+  }
+
+  const int pos_even = 2 * ((first >> 1) + pair);
+  bool live = item < max_pairs * per_pair && pos_even < len;
+  int page = 0;
+  if (live) {
+    page = page_table[(size_t)b * max_pages + pos_even / kPageTokens];
+    if (page < 0 || page >= num_pages) {
+      report(err, NVKV_DEVERR_PAGE_ID);
+      live = false;
+    }
+  }
+  const int slot_even = pos_even % kPageTokens;
+  uint8_t *blk = pool + ((size_t)page * Hkv + h) * k8_head_bytes(D);
+
+  bool is_new[2];
+  size_t src[2];
+  float kx[2][16];
+  float amax[2] = {0.f, 0.f};
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    const int pos = pos_even + k;
+    is_new[k] = live && pos >= first && pos < len;
+    src[k] = ((size_t)(row0 + pos - first) * Hkv + h) * D + g * kGroup;
+    if (is_new[k]) {
+      load16_f32(k_new + src[k], kx[k]);
+    } else {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) kx[k][i] = 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < 16; ++i) amax[k] = fmaxf(amax[k], fabsf(kx[k][i]));
+  }
+  for (int o = 1; o < groups; o <<= 1) {  // row maximum over the row's D/16 lanes
+    amax[0] = fmaxf(amax[0], __shfl_xor_sync(0xffffffffu, amax[0], o));
+    amax[1] = fmaxf(amax[1], __shfl_xor_sync(0xffffffffu, amax[1], o));
+  }
+
+  GroupQ vq[2];
+#pragma unroll
+  for (int k = 0; k < 2; ++k) {
+    if (!is_new[k]) continue;
+    const int slot = slot_even + k;
+    const float sc = __fdiv_rn(amax[k], 448.0f);
+    uint32_t w[4] = {0u, 0u, 0u, 0u};
+    if (sc != 0.f) {
+#pragma unroll
+      for (int i = 0; i < 16; ++i) w[i >> 2] |= e4m3_byte(__fdiv_rn(kx[k][i], sc)) << (8 * (i & 3));
+    }
+    *reinterpret_cast<uint4 *>(blk + (size_t)slot * D + g * kGroup) =
+        make_uint4(w[0], w[1], w[2], w[3]);
+    if (g == 0) *reinterpret_cast<float *>(blk + k8_ks_off(D) + 4 * slot) = sc;
+    vq[k] = quantize16(v_new + src[k]);
+    blk[k8_vs_off(D) + g * kPageTokens + slot] = vq[k].scale;
+  }
+  if (!live) return;
+  // V code bytes (d, slot_even/2) for the 16 elements of group g.
+  uint8_t *vc = blk + k8_vc_off(D) + (size_t)(g * kGroup) * 8 + slot_even / 2;
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    uint8_t *p = vc + i * 8;
+    const uint32_t lo = is_new[0] ? ((i < 8 ? vq[0].codes_lo : vq[0].codes_hi) >> (4 * (i & 7))) & 15u
+                                  : *p & 15u;
+    const uint32_t hi = is_new[1] ? ((i < 8 ? vq[1].codes_lo : vq[1].codes_hi) >> (4 * (i & 7))) & 15u
+                                  : *p >> 4;
+    *p = static_cast<uint8_t>(lo | (hi << 4));
+  }
+}
+
+cudaError_t launch_append_k8v4(const nvkv_cache &c, const nvkv_seqs &s, const void *k_new,
+                               const void *v_new, const int32_t *cu_new, int total_new,
+                               int max_new, cudaStream_t stream) {
+  const int max_pairs = max_new / 2 + 1;
+  const int per_pair = c.num_kv_heads * (c.head_dim / kGroup);
+  const long items = (long)max_pairs * per_pair;
+  const int threads = 256;
+  dim3 grid((unsigned)((items + threads - 1) / threads), (unsigned)s.batch);
+  append_k8v4_kernel<<<grid, threads, 0, stream>>>(
+      c.pool, c.num_pages, c.num_kv_heads, c.head_dim, s.page_table, s.max_pages_per_seq,
+      s.kv_lens, s.max_kv_len, static_cast<const __nv_bfloat16 *>(k_new),
+      static_cast<const __nv_bfloat16 *>(v_new), cu_new, total_new, max_new, max_pairs,
+      s.err_word);
+  return cudaGetLastError();
+}
+
 namespace {
 
 // (cos, sin) of (pos / scale) * base^(-2i / rotary_dim), in double, rounded

@@ -15,18 +15,79 @@
 // tokens a warp reads the K codes of the page (two lanes per token, half of
 // head_dim each), forms the 16 scores, updates the online softmax, then
 // each lane accumulates D/32 output channels from the transposed V codes.
+//
+// The same kernels serve the K8V4 cache (the "knoopx/ninfer" README lists it
+// among its KV storage formats): K rows of one E4M3 byte per element with
+// one float scale per row, V as in the NVFP4 cache.  Only the K score and
+// the block offsets differ; the softmax and the value sums are shared.
 #include "nvkv_common.cuh"
 
 namespace nvkv {
 
 constexpr int kSimtWarps = 8;
 
+// Partial score of K row `slot` of a page block: the dot product of the
+// half `half` of head_dim with the same half of the query row qr.
+//
+// NVFP4 block: 4-bit codes, one E4M3 scale per 16 elements.
+__device__ __forceinline__ float k_half_score(Nvfp4Layout, const uint8_t *blk, int D, int slot,
+                                              int half, const float *qr) {
+  const uint8_t *kc = blk + kc_off(D) + slot * (D / 2) + half * (D / 4);
+  const uint8_t *ks = blk + ks_off(D) + slot * (D / 16) + half * (D / 32);
+  const float *qh = qr + half * (D / 2);
+  float s = 0.f;
+  for (int c16 = 0; c16 < D / 64; ++c16) {  // 16 bytes = 32 elements = 2 groups
+    uint4 w4 = *reinterpret_cast<const uint4 *>(kc + 16 * c16);
+    uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+    for (int gg = 0; gg < 2; ++gg) {
+      float part = 0.f;
+#pragma unroll
+      for (int bi = 0; bi < 8; ++bi) {
+        const int byte_idx = gg * 8 + bi;
+        uint32_t byte = (w[byte_idx >> 2] >> (8 * (byte_idx & 3))) & 0xffu;
+        float2 v = f16x2_to_float2(e2m1x2_to_f16x2(byte));
+        const int d = 32 * c16 + 2 * byte_idx;
+        part = fmaf(v.x, qh[d], part);
+        part = fmaf(v.y, qh[d + 1], part);
+      }
+      s = fmaf(part, e4m3_to_float(ks[2 * c16 + gg]), s);
+    }
+  }
+  return s;
+}
 
+// K8V4 block: one E4M3 byte per element, one float scale per row.
+__device__ __forceinline__ float k_half_score(K8v4Layout, const uint8_t *blk, int D, int slot,
+                                              int half, const float *qr) {
+  const uint8_t *kc = blk + slot * D + half * (D / 2);
+  const float row_scale = *reinterpret_cast<const float *>(blk + k8_ks_off(D) + 4 * slot);
+  const float *qh = qr + half * (D / 2);
+  float part = 0.f;
+  for (int c16 = 0; c16 < D / 32; ++c16) {  // 16 bytes = 16 elements
+    uint4 w4 = *reinterpret_cast<const uint4 *>(kc + 16 * c16);
+    uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
+#pragma unroll
+    for (int wi = 0; wi < 4; ++wi) {
+      uint32_t h2[2];
+      e4m3x4_to_f16x2x2(w[wi], h2);  // h2[k] = elements 2k, 2k+1 of the word
+      const float2 a = f16x2_to_float2(h2[0]), b = f16x2_to_float2(h2[1]);
+      const int d = 16 * c16 + 4 * wi;
+      part = fmaf(a.x, qh[d], part);
+      part = fmaf(a.y, qh[d + 1], part);
+      part = fmaf(b.x, qh[d + 2], part);
+      part = fmaf(b.y, qh[d + 3], part);
+    }
+  }
+  return part * row_scale;
+}
 
 // Online softmax of one query row (qr: fp32, pre-scaled to base-2 scores)
-// over keys [jb, je) of one sequence / kv-head, jb a multiple of 16.  The
-// calling warp returns the running max m, the sum l of 2^(s - m) and, per
-// lane, the unnormalised value sums of channels [lane*D/32, (lane+1)*D/32).
+// over keys [jb, je) of one sequence / kv-head, jb a multiple of 16, in a
+// pool of layout L.  The calling warp returns the running max m, the sum l
+// of 2^(s - m) and, per lane, the unnormalised value sums of channels
+// [lane*D/32, (lane+1)*D/32).
+template <class L>
 __device__ __forceinline__ void attend_rows_simt(const uint8_t *__restrict__ pool, int num_pages,
                                                  int Hkv, int D, int h,
                                                  const int32_t *__restrict__ pt, int jb, int je,
@@ -44,34 +105,11 @@ __device__ __forceinline__ void attend_rows_simt(const uint8_t *__restrict__ poo
       if (lane == 0) report(err, NVKV_DEVERR_PAGE_ID);
       continue;
     }
-    const uint8_t *blk = pool + (size_t)page * Hkv * head_bytes(D) + (size_t)h * head_bytes(D);
+    const uint8_t *blk = pool + (size_t)page * Hkv * L::head(D) + (size_t)h * L::head(D);
     // ---- scores: lane -> (slot, half of head_dim) ----
     const int slot = lane & 15, half = lane >> 4;
     const bool valid = (p0 + slot) < je;
-    float s = 0.f;
-    {
-      const uint8_t *kc = blk + kc_off(D) + slot * (D / 2) + half * (D / 4);
-      const uint8_t *ks = blk + ks_off(D) + slot * (D / 16) + half * (D / 32);
-      const float *qh = qr + half * (D / 2);
-      for (int c16 = 0; c16 < D / 64; ++c16) {  // 16 bytes = 32 elements = 2 groups
-        uint4 w4 = *reinterpret_cast<const uint4 *>(kc + 16 * c16);
-        uint32_t w[4] = {w4.x, w4.y, w4.z, w4.w};
-#pragma unroll
-        for (int gg = 0; gg < 2; ++gg) {
-          float part = 0.f;
-#pragma unroll
-          for (int bi = 0; bi < 8; ++bi) {
-            const int byte_idx = gg * 8 + bi;
-            uint32_t byte = (w[byte_idx >> 2] >> (8 * (byte_idx & 3))) & 0xffu;
-            float2 v = f16x2_to_float2(e2m1x2_to_f16x2(byte));
-            const int d = 32 * c16 + 2 * byte_idx;
-            part = fmaf(v.x, qh[d], part);
-            part = fmaf(v.y, qh[d + 1], part);
-          }
-          s = fmaf(part, e4m3_to_float(ks[2 * c16 + gg]), s);
-        }
-      }
-    }
+    float s = k_half_score(L{}, blk, D, slot, half, qr);
     s += __shfl_xor_sync(0xffffffffu, s, 16);
     const float s_eff = valid ? s : -INFINITY;
     const float m_new = fmaxf(m, warp_max(s_eff));
@@ -82,7 +120,7 @@ __device__ __forceinline__ void attend_rows_simt(const uint8_t *__restrict__ poo
     // ---- values: lane -> channels [lane*dpl, lane*dpl + dpl) ----
     const int d0 = lane * dpl;
     const int g = d0 / kGroup;
-    uint4 sc4 = *reinterpret_cast<const uint4 *>(blk + vs_off(D) + g * kPageTokens);
+    uint4 sc4 = *reinterpret_cast<const uint4 *>(blk + L::vs(D) + g * kPageTokens);
     uint32_t sc[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
     float wgt[16];
 #pragma unroll
@@ -94,7 +132,7 @@ __device__ __forceinline__ void attend_rows_simt(const uint8_t *__restrict__ poo
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
       if (i >= dpl) break;
-      const uint2 cw = *reinterpret_cast<const uint2 *>(blk + vc_off(D) + (size_t)(d0 + i) * 8);
+      const uint2 cw = *reinterpret_cast<const uint2 *>(blk + L::vc(D) + (size_t)(d0 + i) * 8);
       uint32_t cws[2] = {cw.x, cw.y};
       float a = acc[i] * alpha;
 #pragma unroll
@@ -109,6 +147,7 @@ __device__ __forceinline__ void attend_rows_simt(const uint8_t *__restrict__ poo
   }
 }
 
+template <class L>
 __global__ void __launch_bounds__(kSimtWarps * 32)
 decode_simt_kernel(const uint8_t *__restrict__ pool, int num_pages, int Hkv, int D,
                    const int32_t *__restrict__ page_table, int max_pages,
@@ -154,7 +193,8 @@ decode_simt_kernel(const uint8_t *__restrict__ pool, int num_pages, int Hkv, int
       const int n_vis = kv_len - T + t + 1;  // keys 0 .. n_vis-1 are visible
       const int jb = tok_begin, je = bad_len ? jb : min(tok_end, n_vis);
       float m, l, acc[8];
-      attend_rows_simt(pool, num_pages, Hkv, D, h, pt, jb, je, qs + (size_t)r * D, m, l, acc, err);
+      attend_rows_simt<L>(pool, num_pages, Hkv, D, h, pt, jb, je, qs + (size_t)r * D, m, l, acc,
+                          err);
       // ---- partial result of this split for row r ----
       float *o = ws_o + (slot * R + r) * (size_t)D;
       const float inv = l > 0.f ? 1.f / l : 0.f;
@@ -165,16 +205,18 @@ decode_simt_kernel(const uint8_t *__restrict__ pool, int num_pages, int Hkv, int
   }
 }
 
+// k8: the pool is in the K8V4 layout (else NVFP4).
 cudaError_t launch_decode_simt(const nvkv_cache &c, const nvkv_seqs &s, const void *q, int T,
                                int Hq, float sm_scale, int S, float *ws_o, float *ws_lse,
-                               cudaStream_t stream) {
+                               cudaStream_t stream, bool k8) {
   const int R = T * (Hq / c.num_kv_heads);
   const size_t smem = (size_t)R * c.head_dim * sizeof(float);
-  cudaError_t e = cudaFuncSetAttribute(decode_simt_kernel,
-                                       cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  auto kernel = k8 ? decode_simt_kernel<K8v4Layout> : decode_simt_kernel<Nvfp4Layout>;
+  cudaError_t e =
+      cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   const float qscale = sm_scale * 1.4426950408889634f;  // scores in base 2
-  decode_simt_kernel<<<S, kSimtWarps * 32, smem, stream>>>(
+  kernel<<<S, kSimtWarps * 32, smem, stream>>>(
       c.pool, c.num_pages, c.num_kv_heads, c.head_dim, s.page_table, s.max_pages_per_seq,
       s.kv_lens, s.batch, s.max_kv_len, static_cast<const __nv_bfloat16 *>(q), T, Hq, qscale, S,
       ws_o, ws_lse, s.err_word);
@@ -184,6 +226,7 @@ cudaError_t launch_decode_simt(const nvkv_cache &c, const nvkv_seqs &s, const vo
 // Chunked prefill on CUDA cores: one warp per (chunk row, query head), over
 // the row's whole visible prefix (keys 0 .. its position).  Used for chunks
 // the tensor-core prefill kernel does not take.
+template <class L>
 __global__ void __launch_bounds__(kSimtWarps * 32)
 prefill_simt_kernel(const uint8_t *__restrict__ pool, int num_pages, int Hkv, int D,
                     const int32_t *__restrict__ page_table, int max_pages,
@@ -212,8 +255,8 @@ prefill_simt_kernel(const uint8_t *__restrict__ pool, int num_pages, int Hkv, in
     je = 0;
   }
   float m, l, acc[8];
-  attend_rows_simt(pool, num_pages, Hkv, D, h, page_table + (size_t)b * max_pages, 0, je, qr, m,
-                   l, acc, err);
+  attend_rows_simt<L>(pool, num_pages, Hkv, D, h, page_table + (size_t)b * max_pages, 0, je, qr,
+                      m, l, acc, err);
   const int dpl = D / 32;
   const float inv = l > 0.f ? 1.f / l : 0.f;
   __nv_bfloat16 *dst = out + ((size_t)row * Hq + hq) * D + lane * dpl;
@@ -222,12 +265,13 @@ prefill_simt_kernel(const uint8_t *__restrict__ pool, int num_pages, int Hkv, in
 
 cudaError_t launch_prefill_simt(const nvkv_cache &c, const nvkv_seqs &s, const void *q,
                                 const int32_t *cu_q, int total_q, int Hq, float sm_scale,
-                                void *out, cudaStream_t stream) {
+                                void *out, cudaStream_t stream, bool k8) {
   const long warps = (long)total_q * Hq;
   const long blocks = (warps + kSimtWarps - 1) / kSimtWarps;
   const size_t smem = (size_t)kSimtWarps * c.head_dim * sizeof(float);
   const float qscale = sm_scale * 1.4426950408889634f;
-  prefill_simt_kernel<<<(unsigned)blocks, kSimtWarps * 32, smem, stream>>>(
+  auto kernel = k8 ? prefill_simt_kernel<K8v4Layout> : prefill_simt_kernel<Nvfp4Layout>;
+  kernel<<<(unsigned)blocks, kSimtWarps * 32, smem, stream>>>(
       c.pool, c.num_pages, c.num_kv_heads, c.head_dim, s.page_table, s.max_pages_per_seq,
       s.kv_lens, s.batch, s.max_kv_len, static_cast<const __nv_bfloat16 *>(q), cu_q, total_q, Hq,
       qscale, static_cast<__nv_bfloat16 *>(out), s.err_word);

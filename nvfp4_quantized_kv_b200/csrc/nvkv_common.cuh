@@ -26,6 +26,30 @@ __host__ __device__ constexpr int vc_off(int D) { return 9 * D; }
 __host__ __device__ constexpr int vs_off(int D) { return 17 * D; }
 __host__ __device__ constexpr int head_bytes(int D) { return 18 * D; }
 
+// Byte offsets inside one kv-head block of a K8V4 page (25*D + 64 bytes):
+// K codes [16 slots][D] (one E4M3 byte per element), K scales [16 slots]
+// (float), then V exactly as in an NVFP4 block: codes [D][8], scales
+// [D/16][16].  Every region starts on a 16-byte boundary (D is 128 or 256).
+__host__ __device__ constexpr int k8_ks_off(int D) { return 16 * D; }
+__host__ __device__ constexpr int k8_vc_off(int D) { return 16 * D + 64; }
+__host__ __device__ constexpr int k8_vs_off(int D) { return 24 * D + 64; }
+__host__ __device__ constexpr int k8_head_bytes(int D) { return 25 * D + 64; }
+
+// The two cache formats as compile-time layouts (the CUDA-core attention
+// kernels are written once for both).
+struct Nvfp4Layout {
+  static constexpr bool kK8 = false;
+  __device__ static int head(int D) { return head_bytes(D); }
+  __device__ static int vc(int D) { return vc_off(D); }
+  __device__ static int vs(int D) { return vs_off(D); }
+};
+struct K8v4Layout {
+  static constexpr bool kK8 = true;
+  __device__ static int head(int D) { return k8_head_bytes(D); }
+  __device__ static int vc(int D) { return k8_vc_off(D); }
+  __device__ static int vs(int D) { return k8_vs_off(D); }
+};
+
 // ---------------------------------------------------------------------------
 // Split plan (see nvkv_decode_workspace_bytes in nvkv.h).  Units of 128
 // tokens of every (b, h) pair, in (b, h, unit) order, are dealt to S ranges:

@@ -11,8 +11,15 @@ from __future__ import annotations
 import numpy as np
 import torch
 
-from . import (Cache, Seqs, nvkv_append, nvkv_combine, nvkv_decode_attn,
-               nvkv_decode_workspace_bytes, nvkv_prefill_attn)
+from . import (Cache, Seqs, nvkv_append, nvkv_append_k8v4, nvkv_combine, nvkv_decode_attn,
+               nvkv_decode_attn_k8v4, nvkv_decode_workspace_bytes, nvkv_prefill_attn,
+               nvkv_prefill_attn_k8v4)
+
+# The calls of each cache format: (append, decode partials, prefill).
+_CALLS = {
+    "nvfp4": (nvkv_append, nvkv_decode_attn, nvkv_prefill_attn),
+    "k8v4": (nvkv_append_k8v4, nvkv_decode_attn_k8v4, nvkv_prefill_attn_k8v4),
+}
 from .workload import Workload
 
 
@@ -29,10 +36,16 @@ def bf16_tensor(bits: np.ndarray, device) -> torch.Tensor:
 
 class DeviceWorkload:
     def __init__(self, wl: Workload, device="cuda", fill: int | None = 0xA5, num_splits: int = 0,
-                 err_word: bool = True, cache_from: "DeviceWorkload | None" = None):
+                 err_word: bool = True, cache_from: "DeviceWorkload | None" = None,
+                 kv_format: str = "nvfp4"):
         """cache_from: reuse the (already filled) pool of another workload
         with the same cached context -- same seed, lengths, heads and page
-        table -- under a different step shape (T=1 decode and T=6 verify)."""
+        table -- under a different step shape (T=1 decode and T=6 verify).
+        kv_format: "nvfp4" (the default) or "k8v4"."""
+        if kv_format not in _CALLS:
+            raise ValueError(f"kv_format must be one of {tuple(_CALLS)}")
+        self.kv_format = kv_format
+        self._append, self._decode, self._prefill = _CALLS[kv_format]
         self.wl = wl
         self.device = torch.device(device)
         self.num_splits = num_splits
@@ -41,12 +54,13 @@ class DeviceWorkload:
             o = cache_from.wl
             if (o.seed, list(o.ctx), o.num_kv_heads, o.head_dim, o.num_pages) != \
                     (wl.seed, list(wl.ctx), wl.num_kv_heads, wl.head_dim, wl.num_pages) or \
-                    not np.array_equal(cache_from.page_table_np, self.page_table_np):
+                    not np.array_equal(cache_from.page_table_np, self.page_table_np) or \
+                    cache_from.kv_format != kv_format:
                 raise ValueError("cache_from: the two workloads do not share a cached context")
             self.cache = cache_from.cache
         else:
             self.cache = Cache.allocate(wl.num_pages, wl.num_kv_heads, wl.head_dim, self.device,
-                                        fill)
+                                        fill, kv_format)
         self.page_table = _h2d(self.page_table_np, self.device)
         self.kv_lens = _h2d(wl.kv_lens, self.device)
         self.err = torch.zeros(1, dtype=torch.int32, device=self.device) if err_word else None
@@ -74,8 +88,8 @@ class DeviceWorkload:
                 lens = torch.tensor([stop], dtype=torch.int32, device=self.device)
                 seqs = Seqs(pt_b, lens, stop, self.err)
                 cu = torch.tensor([0, stop - start], dtype=torch.int32, device=self.device)
-                nvkv_append(self.cache, seqs, bf16_tensor(k, self.device), bf16_tensor(v, self.device),
-                            cu, stop - start, stop - start)
+                self._append(self.cache, seqs, bf16_tensor(k, self.device),
+                             bf16_tensor(v, self.device), cu, stop - start, stop - start)
         torch.cuda.synchronize(self.device)
 
     # ---- step inputs -----------------------------------------------------
@@ -91,19 +105,19 @@ class DeviceWorkload:
     # ---- one step ----------------------------------------------------------
     def append(self, stream=None) -> None:
         wl = self.wl
-        nvkv_append(self.cache, self.seqs, self.k_new, self.v_new, self.cu_new, wl.batch * wl.T,
-                    wl.T, stream)
+        self._append(self.cache, self.seqs, self.k_new, self.v_new, self.cu_new, wl.batch * wl.T,
+                     wl.T, stream)
 
     def attend(self, stream=None) -> None:
         wl = self.wl
         if wl.mode == "decode":
-            nvkv_decode_attn(self.cache, self.seqs, self.q, wl.T, wl.num_q_heads, wl.sm_scale,
-                             self.num_splits, self.workspace, stream)
+            self._decode(self.cache, self.seqs, self.q, wl.T, wl.num_q_heads, wl.sm_scale,
+                         self.num_splits, self.workspace, stream)
             nvkv_combine(self.seqs, self.workspace, wl.T, wl.num_q_heads, wl.num_kv_heads,
                          wl.head_dim, self.num_splits, self.out, stream)
         else:
-            nvkv_prefill_attn(self.cache, self.seqs, self.q, self.cu_new, wl.batch * wl.T, wl.T,
-                              wl.num_q_heads, wl.sm_scale, self.out, stream)
+            self._prefill(self.cache, self.seqs, self.q, self.cu_new, wl.batch * wl.T, wl.T,
+                          wl.num_q_heads, wl.sm_scale, self.out, stream)
 
     def step(self, stream=None) -> None:
         self.append(stream)

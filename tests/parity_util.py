@@ -14,10 +14,11 @@ ATOL = 8e-3
 RTOL = 8e-3
 
 
-def oracle_outputs(wl: Workload, rows, nthreads=None):
+def oracle_outputs(wl: Workload, rows, nthreads=None, k8=False):
     """rows: list of (b, t, hq).  Returns float64 [len(rows)][D]: the exact
     attention of query t of sequence b, head hq, over the sequence's keys
-    0 .. ctx_b + t (all rows of the workload, quantised by the oracle)."""
+    0 .. ctx_b + t (all rows of the workload, quantised by the oracle; K in
+    the K8V4 cache's 8-bit row format when k8)."""
     q = wl.queries()
     G = wl.group
     kv = {}
@@ -27,7 +28,8 @@ def oracle_outputs(wl: Workload, rows, nthreads=None):
     for b, t, hq in rows:
         k, v = kv[b]
         jobs.append((k, v, hq // G, wl.query_position(b, t) + 1, q[b * wl.T + t, hq]))
-    out, _, psum = oracle.attention_rows(jobs, wl.num_kv_heads, wl.head_dim, wl.sm_scale, nthreads)
+    out, _, psum = oracle.attention_rows(jobs, wl.num_kv_heads, wl.head_dim, wl.sm_scale, nthreads,
+                                         k8=k8)
     assert np.all(np.abs(psum - 1) < 1e-9)
     return out
 

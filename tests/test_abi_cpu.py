@@ -186,3 +186,58 @@ def test_rope_calls_reject_bad_arguments_without_launch(lib):
     assert a(B(c), B(s), *ok, 0x1000, 16, 40, None) == nv.ERR_INVALID_ARG
     assert a(B(c), B(s), *ok, 0x1000, 0, 64, None) == nv.ERR_INVALID_ARG
     assert a(B(c), B(s), 0x10, 0x20, 0x30, 0, 0, 0x1000, 16, 64, None) == nv.OK  # nothing new
+
+
+def test_k8v4_page_bytes(lib):
+    import oracle
+    for hkv, d in [(4, 256), (2, 128), (1, 128), (8, 256)]:
+        assert nv.nvkv_k8v4_page_bytes(hkv, d) == hkv * (25 * d + 64) == \
+            oracle.k8v4_page_bytes(hkv, d)
+        assert (25 * d + 64) % 16 == 0  # every kv-head block starts 16-byte aligned
+    assert lib.nvkv_k8v4_page_bytes(0, 128) == 0 and lib.nvkv_k8v4_page_bytes(2, 0) == 0
+
+
+def test_k8v4_calls_reject_bad_arguments_without_launch(lib):
+    B = ctypes.byref
+    c, s = cache(), seqs()
+    a = lib.nvkv_append_k8v4
+    assert a(None, B(s), 0x10, 0x20, 0x30, 1, 1, None) == nv.ERR_INVALID_ARG
+    assert a(B(cache(d=64)), B(s), 0x10, 0x20, 0x30, 1, 1, None) == nv.ERR_UNSUPPORTED
+    assert a(B(c), B(s), 0x18, 0x20, 0x30, 1, 1, None) == nv.ERR_INVALID_ARG  # misaligned
+    assert a(B(c), B(seqs(max_len=65)), 0x10, 0x20, 0x30, 1, 1, None) == nv.ERR_INVALID_ARG
+    assert a(B(c), B(s), None, None, None, 0, 0, None) == nv.OK  # nothing to do
+    c4 = cache(hkv=4, d=256)
+    f = lib.nvkv_decode_attn_k8v4
+    need = lib.nvkv_decode_workspace_bytes(1, 1, 24, 4, 256, 8)
+    assert f(B(c4), B(s), 0x100, 1, 25, 0.1, 8, 0x1000, need, None) == nv.ERR_INVALID_ARG
+    assert f(B(c4), B(s), 0x100, 17, 24, 0.1, 8, 0x1000, need, None) == nv.ERR_UNSUPPORTED
+    assert f(B(c4), B(s), 0x100, 1, 24, float("inf"), 8, 0x1000, need, None) == \
+        nv.ERR_INVALID_ARG
+    assert f(B(c4), B(s), 0x100, 1, 24, 0.1, 8, 0x1000, need - 1, None) == nv.ERR_WORKSPACE
+    assert f(B(c4), B(s), 0x100, 1, 24, 0.1, 8, None, need, None) == nv.ERR_WORKSPACE
+    p = lib.nvkv_prefill_attn_k8v4
+    assert p(B(c4), B(s), 0x100, 0x200, 10, 10, 25, 0.1, 0x300, None) == nv.ERR_INVALID_ARG
+    assert p(B(c4), B(s), None, 0x200, 10, 10, 24, 0.1, 0x300, None) == nv.ERR_INVALID_ARG
+    assert p(B(c4), B(s), 0x100, 0x200, 10, 10, 24, 0.1, 0x308, None) == nv.ERR_INVALID_ARG
+    assert p(B(c4), B(s), None, None, 0, 0, 24, 0.1, None, None) == nv.OK
+
+
+def test_calls_refuse_a_cache_of_the_other_format():
+    """The Python binding keeps the two layouts apart: an NVFP4 call given a
+    K8V4 cache (and the reverse) raises before any argument is marshalled."""
+    import types
+    k8 = types.SimpleNamespace(kv_format="k8v4")
+    fp4 = types.SimpleNamespace(kv_format="nvfp4")
+    for call in (lambda: nv.nvkv_append(k8, None, None, None, None, 1, 1),
+                 lambda: nv.nvkv_decode_attn(k8, None, None, 1, 8, 0.1, 0, None),
+                 lambda: nv.nvkv_prefill_attn(k8, None, None, None, 1, 1, 8, 0.1, None),
+                 lambda: nv.nvkv_decode_attn_static(k8, None, None, 1, 8, 0.1, 0, None),
+                 lambda: nv.nvkv_append_rope(k8, None, None, None, None, 1, 1, None, 64),
+                 lambda: nv.nvkv_pages_spill(k8, None, None, None),
+                 lambda: nv.nvkv_append_k8v4(fp4, None, None, None, None, 1, 1),
+                 lambda: nv.nvkv_decode_attn_k8v4(fp4, None, None, 1, 8, 0.1, 0, None),
+                 lambda: nv.nvkv_prefill_attn_k8v4(fp4, None, None, None, 1, 1, 8, 0.1, None)):
+        with pytest.raises(ValueError, match="cache"):
+            call()
+    with pytest.raises(ValueError):
+        nv._page_bytes_of("int8", 2, 128)
