@@ -228,6 +228,8 @@ def main():
     ap.add_argument("--no-spill", action="store_true", help="skip the page spill/restore line")
     ap.add_argument("--no-graph", action="store_true",
                     help="skip the CUDA-graph replay line (a step captured once, replayed)")
+    ap.add_argument("--no-k8v4", action="store_true",
+                    help="skip the K8V4-cache decode line (3 x 60k context)")
     ap.add_argument("--no-verify", action="store_true",
                     help="skip the T=6 MTP-verify line (measured on the T=1 pool)")
     ap.add_argument("--ctx", type=str, default=None,
@@ -531,6 +533,44 @@ def main():
         except Exception as exc:  # a failure here must not cost the lines above
             graph = {"error": repr(exc)[:300]}
 
+    # ---- the same decode step over a K8V4 cache (E4M3 K rows, NVFP4 V) on
+    # the CUDA-core kernels, on its own 3 x 60k context ----
+    k8 = None
+    if not args.no_k8v4:
+        try:
+            kw = W.long_context(T=1, ctx=(60000, 60000, 60000))
+            kdw = DeviceWorkload(kw, dev, fill=None, num_splits=args.num_splits,
+                                 kv_format="k8v4")
+            kdw.fill_context()
+            kdw.load_step_inputs()
+            for _ in range(3):
+                kdw.step(stream)
+            reps = 50
+            ke = [torch.cuda.Event(enable_timing=True) for _ in range(3)]
+            torch.cuda.synchronize(dev)
+            ke[0].record(stream)
+            for _ in range(reps):
+                kdw.step(stream)
+            ke[1].record(stream)
+            for _ in range(reps):
+                kdw.attend(stream)
+            ke[2].record(stream)
+            torch.cuda.synchronize(dev)
+            step_ms = ke[0].elapsed_time(ke[1]) / reps
+            attend_ms = ke[1].elapsed_time(ke[2]) / reps
+            # K 1 byte per element + an fp32 scale per row, V 4.5 bits per element
+            kvb = sum(int(c) + 1 for c in kw.ctx) * kw.num_kv_heads * (
+                kw.head_dim + 4 + kw.head_dim * 9 // 16)
+            k8 = {"workload": kw.name + "_k8v4", "kernel": "decode_simt (CUDA cores)",
+                  "kv_bytes_per_step": kvb, "step_ms": step_ms,
+                  "step_gbs": kvb / (step_ms * 1e-3) / 1e9, "attend_ms": attend_ms,
+                  "attend_gbs": kvb / (attend_ms * 1e-3) / 1e9,
+                  "attend_frac": kvb / (attend_ms * 1e-3) / 1e9 / peak,
+                  "device_errors": kdw.err_bits()}
+            del kdw
+        except Exception as exc:  # a failure here must not cost the lines above
+            k8 = {"error": repr(exc)[:300]}
+
     if rank == 0:
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
@@ -559,6 +599,7 @@ def main():
             "prefill": prefill,
             "rope_append": rope,
             "cuda_graph": graph,
+            "k8v4_decode": k8,
             "cpu_baseline": cpu,
         }
         print(json.dumps(line), flush=True)
