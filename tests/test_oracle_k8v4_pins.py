@@ -158,3 +158,32 @@ def test_attention_rows_and_pool_forms_agree():
     # K in the 8-bit format differs from NVFP4 K, V is the same format
     c, _, _ = oracle.attention_rows(jobs_r, Hkv, D, 0.088, k8=False)
     assert not np.array_equal(a, c)
+
+
+def test_attention_invariants_with_8bit_keys():
+    """Closed forms of softmax attention that hold whatever the key format:
+    a zero query and equal key rows both give the mean of the dequantised
+    values; one key whose score dominates gives its value row; the lse of a
+    single key is its score, computed here from the 8-bit dequantised row."""
+    rng = np.random.default_rng(35)
+    Hkv, D, n = 2, 128, 33
+    k = _bits(rng.standard_normal((n, Hkv, D)) * 4)
+    v = _bits(rng.standard_normal((n, Hkv, D)))
+    vmean = oracle.qdq_rows(v[:, 1]).mean(axis=0)
+    zero_q = np.zeros(D, np.uint16)
+    out, _, _ = oracle.attention_rows([(k, v, 1, n, zero_q)], Hkv, D, 0.088, k8=True)
+    assert np.allclose(out[0], vmean, rtol=0, atol=1e-13)
+    keq = np.repeat(k[:1], n, axis=0)
+    q = _bits(rng.standard_normal(D))
+    out, _, _ = oracle.attention_rows([(keq, v, 1, n, q)], Hkv, D, 0.088, k8=True)
+    assert np.allclose(out[0], vmean, rtol=0, atol=1e-13)
+    kd = _bits(rng.standard_normal((n, Hkv, D)) * 0.01)
+    kd[13, 0] = _bits(np.full(D, 8.0))
+    qd = _bits(np.full(D, 4.0))
+    out, _, _ = oracle.attention_rows([(kd, v, 0, n, qd)], Hkv, D, 1 / np.sqrt(D), k8=True)
+    assert np.allclose(out[0], oracle.qdq_rows(v[13, 0][None])[0], rtol=0, atol=1e-60)
+    out, lse, _ = oracle.attention_rows([(k, v, 1, 1, q)], Hkv, D, 0.088, k8=True)
+    c, sc = oracle.k8_quantize_row(k[0, 1])
+    krow = np.array([oracle.k8_dequant(int(x), sc) for x in c])
+    qf = _f32(q).astype(np.float64)
+    assert abs(lse[0] - 0.088 * float(np.dot(qf, krow))) < 1e-12
