@@ -11,12 +11,20 @@ Sources (page titles and sections of the pages this path is built from):
     NVFP4 KV cache bullet: 4-bit E2M1 codes plus one E4M3 scale per group
     of 16, here groups along head_dim.
   * "knoopx/ninfer" README, "Capabilities and limits": chunked prefill,
-    batched decode, MTP verify with one to five drafts, one shared KV pool.
+    batched decode, MTP verify with one to five drafts, one shared KV pool;
+    K8V4 among the KV storage formats (8-bit K rows, NVFP4 V).
+  * "gzenz/ninfer" README, "Fork changes vs upstream" -> "Context and
+    model": linear RoPE scaling of the context extension (the rotating
+    append).
 
 Parity of every function here is pinned by ``tests/test_oracle_pins.py``
 (format tables, exhaustive rounding sweeps against an independent
 table-scan formulation and torch's float8 conversion, round-trip
-invariants, closed-form attention cases and pure-Python brute force).
+invariants, closed-form attention cases and pure-Python brute force),
+``tests/test_oracle_rope_pins.py`` (rotary table and rotation: closed-form
+angles, linear scaling, the relative-position property, norms) and
+``tests/test_oracle_k8v4_pins.py`` (8-bit K rows: table scan, error bound,
+layout reader, attention closed forms).
 """
 from __future__ import annotations
 
