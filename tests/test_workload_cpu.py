@@ -76,3 +76,9 @@ def test_kv_bytes_per_step_is_the_metric_closed_form():
     assert wl.kv_bytes_per_step() == int(sum(int(c) + 1 for c in wl.ctx) * 4 * 256 * 1.125)
     w6 = W.long_context(T=6)
     assert w6.kv_bytes_per_step() == int(sum(int(c) + 6 for c in w6.ctx) * 4 * 256 * 1.125)
+
+
+def test_device_workload_refuses_an_unknown_cache_format():
+    from nvfp4_quantized_kv_b200.harness import DeviceWorkload
+    with pytest.raises(ValueError, match="kv_format"):
+        DeviceWorkload(W.tiny_decode(), device="cpu", kv_format="int8")
