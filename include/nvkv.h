@@ -267,6 +267,9 @@ nvkv_status nvkv_pages_restore(const nvkv_cache *cache, const int32_t *page_ids,
  *   nvkv_decode_attn_k8v4  ~ nvkv_decode_attn (same workspace size and
  *                            split plan; merge with nvkv_combine)
  *   nvkv_prefill_attn_k8v4 ~ nvkv_prefill_attn
+ *   nvkv_pages_spill_k8v4, nvkv_pages_restore_k8v4 ~ nvkv_pages_spill,
+ *                            nvkv_pages_restore, with arena slots of
+ *                            nvkv_k8v4_page_bytes() bytes
  * The attention calls run on CUDA cores (one warp per query row).
  * nvkv_k8v4_page_bytes returns 0 for non-positive arguments. */
 size_t nvkv_k8v4_page_bytes(int32_t num_kv_heads, int32_t head_dim);
@@ -281,6 +284,12 @@ nvkv_status nvkv_prefill_attn_k8v4(const nvkv_cache *cache, const nvkv_seqs *seq
                                    const int32_t *cu_q, int32_t total_q, int32_t max_q,
                                    int32_t num_q_heads, float sm_scale, void *out,
                                    nvkv_stream_t stream);
+nvkv_status nvkv_pages_spill_k8v4(const nvkv_cache *cache, const int32_t *page_ids,
+                                  const int32_t *slot_ids, int32_t n, void *arena,
+                                  int64_t num_slots, int32_t *err_word, nvkv_stream_t stream);
+nvkv_status nvkv_pages_restore_k8v4(const nvkv_cache *cache, const int32_t *page_ids,
+                                    const int32_t *slot_ids, int32_t n, const void *arena,
+                                    int64_t num_slots, int32_t *err_word, nvkv_stream_t stream);
 
 /* Static description of a status code. */
 const char *nvkv_status_string(nvkv_status status);

@@ -24,7 +24,8 @@ __all__ = [
     "nvkv_prefill_attn", "nvkv_status_string", "nvkv_decode_attn_static",
     "nvkv_decode_static_scratch_bytes", "nvkv_rope_table", "nvkv_append_rope",
     "nvkv_pages_spill", "nvkv_pages_restore", "nvkv_k8v4_page_bytes", "nvkv_append_k8v4",
-    "nvkv_decode_attn_k8v4", "nvkv_prefill_attn_k8v4",
+    "nvkv_decode_attn_k8v4", "nvkv_prefill_attn_k8v4", "nvkv_pages_spill_k8v4",
+    "nvkv_pages_restore_k8v4",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -81,6 +82,9 @@ def library():
             "nvkv_pages_spill": (ctypes.c_int, [cp, vp, vp, i32, vp, ctypes.c_int64, vp, vp]),
             "nvkv_pages_restore": (ctypes.c_int, [cp, vp, vp, i32, vp, ctypes.c_int64, vp, vp]),
             "nvkv_k8v4_page_bytes": (sz, [i32, i32]),
+            "nvkv_pages_spill_k8v4": (ctypes.c_int, [cp, vp, vp, i32, vp, ctypes.c_int64, vp, vp]),
+            "nvkv_pages_restore_k8v4": (ctypes.c_int, [cp, vp, vp, i32, vp, ctypes.c_int64, vp,
+                                                       vp]),
             "nvkv_append_k8v4": (ctypes.c_int, [cp, sp, vp, vp, vp, i32, i32, vp]),
             "nvkv_decode_attn_k8v4": (ctypes.c_int, [cp, sp, vp, i32, i32, f32, i32, vp, sz, vp]),
             "nvkv_prefill_attn_k8v4": (ctypes.c_int, [cp, sp, vp, vp, i32, i32, i32, f32, vp, vp]),
@@ -299,11 +303,10 @@ def _dev_or_pinned(t: torch.Tensor, dtype: torch.dtype, name: str) -> int:
 
 
 def _pages_args(cache: Cache, page_ids, slot_ids, arena, err_word):
-    _fmt(cache, "nvfp4", "nvkv_pages_spill / nvkv_pages_restore")
     n = page_ids.numel()
     if slot_ids.numel() != n:
         raise ValueError("page_ids and slot_ids must have the same length")
-    pb = nvkv_page_bytes(cache.num_kv_heads, cache.head_dim)
+    pb = _page_bytes_of(cache.kv_format, cache.num_kv_heads, cache.head_dim)
     return (ctypes.byref(cache._c), _dev_or_pinned(page_ids, torch.int32, "page_ids"),
             _dev_or_pinned(slot_ids, torch.int32, "slot_ids"), int(n),
             _dev_or_pinned(arena, torch.uint8, "arena"), arena.numel() // pb,
@@ -313,17 +316,21 @@ def _pages_args(cache: Cache, page_ids, slot_ids, arena, err_word):
 def nvkv_pages_spill(cache: Cache, page_ids: torch.Tensor, slot_ids: torch.Tensor,
                      arena: torch.Tensor, err_word: torch.Tensor | None = None, stream=None) -> None:
     """Pool page page_ids[i] -> arena slot slot_ids[i] (arena: uint8, device
-    or pinned host, a whole number of page-sized slots)."""
-    _check(library().nvkv_pages_spill(*_pages_args(cache, page_ids, slot_ids, arena, err_word),
-                                      _stream(stream)), "nvkv_pages_spill")
+    or pinned host, a whole number of page-sized slots of the cache's
+    format)."""
+    fn = library().nvkv_pages_spill_k8v4 if cache.kv_format == "k8v4" else library().nvkv_pages_spill
+    _check(fn(*_pages_args(cache, page_ids, slot_ids, arena, err_word), _stream(stream)),
+           "nvkv_pages_spill")
 
 
 def nvkv_pages_restore(cache: Cache, page_ids: torch.Tensor, slot_ids: torch.Tensor,
                        arena: torch.Tensor, err_word: torch.Tensor | None = None,
                        stream=None) -> None:
     """Arena slot slot_ids[i] -> pool page page_ids[i]."""
-    _check(library().nvkv_pages_restore(*_pages_args(cache, page_ids, slot_ids, arena, err_word),
-                                        _stream(stream)), "nvkv_pages_restore")
+    fn = (library().nvkv_pages_restore_k8v4 if cache.kv_format == "k8v4"
+          else library().nvkv_pages_restore)
+    _check(fn(*_pages_args(cache, page_ids, slot_ids, arena, err_word), _stream(stream)),
+           "nvkv_pages_restore")
 
 
 # ---- K8V4 cache (8-bit K rows with one fp32 scale per row, NVFP4 V) --------

@@ -96,9 +96,10 @@ const void *device_view(const void *p) {
   return nullptr;
 }
 
+// pb: bytes of one page of the cache's format.
 nvkv_status pages_move(const nvkv_cache *cache, const int32_t *page_ids, const int32_t *slot_ids,
                        int32_t n, const void *arena, int64_t num_slots, int32_t *err_word,
-                       nvkv_stream_t stream, bool spill) {
+                       nvkv_stream_t stream, bool spill, bool k8) {
   const nvkv_status st = check_cache(cache);
   if (st != NVKV_OK) return st;
   if (n < 0 || num_slots <= 0 || !page_ids || !slot_ids || !arena || !aligned16(arena))
@@ -106,7 +107,8 @@ nvkv_status pages_move(const nvkv_cache *cache, const int32_t *page_ids, const i
   if (n == 0) return NVKV_OK;
   const void *pid = device_view(page_ids), *sid = device_view(slot_ids), *ar = device_view(arena);
   if (!pid || !sid || !ar || !aligned16(ar)) return NVKV_ERR_INVALID_ARG;
-  const int64_t pb = (int64_t)nvkv_page_bytes(cache->num_kv_heads, cache->head_dim);
+  const int64_t pb = (int64_t)(k8 ? nvkv_k8v4_page_bytes(cache->num_kv_heads, cache->head_dim)
+                                  : nvkv_page_bytes(cache->num_kv_heads, cache->head_dim));
   uint8_t *pool = cache->pool;
   uint8_t *arena_b = const_cast<uint8_t *>(static_cast<const uint8_t *>(ar));
   const cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
@@ -353,13 +355,26 @@ nvkv_status nvkv_prefill_attn_k8v4(const nvkv_cache *cache, const nvkv_seqs *seq
 nvkv_status nvkv_pages_spill(const nvkv_cache *cache, const int32_t *page_ids,
                              const int32_t *slot_ids, int32_t n, void *arena, int64_t num_slots,
                              int32_t *err_word, nvkv_stream_t stream) {
-  return pages_move(cache, page_ids, slot_ids, n, arena, num_slots, err_word, stream, true);
+  return pages_move(cache, page_ids, slot_ids, n, arena, num_slots, err_word, stream, true, false);
 }
 
 nvkv_status nvkv_pages_restore(const nvkv_cache *cache, const int32_t *page_ids,
                                const int32_t *slot_ids, int32_t n, const void *arena,
                                int64_t num_slots, int32_t *err_word, nvkv_stream_t stream) {
-  return pages_move(cache, page_ids, slot_ids, n, arena, num_slots, err_word, stream, false);
+  return pages_move(cache, page_ids, slot_ids, n, arena, num_slots, err_word, stream, false,
+                    false);
+}
+
+nvkv_status nvkv_pages_spill_k8v4(const nvkv_cache *cache, const int32_t *page_ids,
+                                  const int32_t *slot_ids, int32_t n, void *arena,
+                                  int64_t num_slots, int32_t *err_word, nvkv_stream_t stream) {
+  return pages_move(cache, page_ids, slot_ids, n, arena, num_slots, err_word, stream, true, true);
+}
+
+nvkv_status nvkv_pages_restore_k8v4(const nvkv_cache *cache, const int32_t *page_ids,
+                                    const int32_t *slot_ids, int32_t n, const void *arena,
+                                    int64_t num_slots, int32_t *err_word, nvkv_stream_t stream) {
+  return pages_move(cache, page_ids, slot_ids, n, arena, num_slots, err_word, stream, false, true);
 }
 
 const char *nvkv_status_string(nvkv_status status) {

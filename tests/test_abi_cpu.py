@@ -233,7 +233,6 @@ def test_calls_refuse_a_cache_of_the_other_format():
                  lambda: nv.nvkv_prefill_attn(k8, None, None, None, 1, 1, 8, 0.1, None),
                  lambda: nv.nvkv_decode_attn_static(k8, None, None, 1, 8, 0.1, 0, None),
                  lambda: nv.nvkv_append_rope(k8, None, None, None, None, 1, 1, None, 64),
-                 lambda: nv.nvkv_pages_spill(k8, None, None, None),
                  lambda: nv.nvkv_append_k8v4(fp4, None, None, None, None, 1, 1),
                  lambda: nv.nvkv_decode_attn_k8v4(fp4, None, None, 1, 8, 0.1, 0, None),
                  lambda: nv.nvkv_prefill_attn_k8v4(fp4, None, None, None, 1, 1, 8, 0.1, None)):
@@ -241,3 +240,14 @@ def test_calls_refuse_a_cache_of_the_other_format():
             call()
     with pytest.raises(ValueError):
         nv._page_bytes_of("int8", 2, 128)
+
+
+def test_k8v4_pages_calls_reject_bad_arguments_without_launch(lib):
+    c = cache()
+    B = ctypes.byref
+    for f in (lib.nvkv_pages_spill_k8v4, lib.nvkv_pages_restore_k8v4):
+        assert f(None, 0x10, 0x20, 1, 0x1000, 4, None, None) == nv.ERR_INVALID_ARG
+        assert f(B(c), 0x10, 0x20, -1, 0x1000, 4, None, None) == nv.ERR_INVALID_ARG
+        assert f(B(c), 0x10, 0x20, 1, 0x1008, 4, None, None) == nv.ERR_INVALID_ARG
+        assert f(B(cache(d=64)), 0x10, 0x20, 1, 0x1000, 4, None, None) == nv.ERR_UNSUPPORTED
+        assert f(B(c), 0x10, 0x20, 0, 0x1000, 4, None, None) == nv.OK

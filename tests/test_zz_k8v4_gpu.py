@@ -204,3 +204,39 @@ def test_decode_k8v4_reports_bad_page():
     torch.cuda.synchronize()
     assert int(err.item()) & nv.DEVERR_PAGE_ID
     assert torch.isfinite(out.float()).all()
+
+
+@pytest.mark.parametrize("kind", ["device", "pinned"])
+def test_k8v4_spill_restore_and_attention_after_restore(kind):
+    """Whole K8V4 pages (nvkv_k8v4_page_bytes each) move to arena slots and
+    back bit for bit; attention over a pool whose pages were destroyed and
+    restored equals attention before the spill, bit for bit."""
+    wl = W.small("k8_spill", 2, 24, 4, 256, 1, [700, 300], seed=22)
+    dw = run_step(wl)
+    before = dw.out.clone()
+    pb = nv.nvkv_k8v4_page_bytes(4, 256)
+    used = np.unique(dw.page_table_np[dw.page_table_np >= 0])
+    slots = np.arange(len(used))
+    if kind == "device":
+        arena = torch.full((len(used) * pb,), 0x3C, dtype=torch.uint8, device="cuda")
+        pid = torch.from_numpy(used.astype(np.int32)).cuda()
+        sid = torch.from_numpy(slots.astype(np.int32)).cuda()
+    else:
+        arena = torch.full((len(used) * pb,), 0x3C, dtype=torch.uint8).pin_memory()
+        pid = torch.from_numpy(used.astype(np.int32)).pin_memory()
+        sid = torch.from_numpy(slots.astype(np.int32)).pin_memory()
+    err = torch.zeros(1, dtype=torch.int32, device="cuda")
+    nv.nvkv_pages_spill(dw.cache, pid, sid, arena, err)
+    torch.cuda.synchronize()
+    pool = dw.cache.pool.cpu().numpy().reshape(wl.num_pages, pb)
+    ar = arena.cpu().numpy().reshape(len(used), pb)
+    for p, s in zip(used, slots):
+        assert np.array_equal(ar[s], pool[p])
+    dw.cache.pool.fill_(0x77)
+    nv.nvkv_pages_restore(dw.cache, pid, sid, arena, err)
+    torch.cuda.synchronize()
+    assert np.array_equal(dw.cache.pool.cpu().numpy().reshape(wl.num_pages, pb)[used], pool[used])
+    dw.attend()
+    torch.cuda.synchronize()
+    assert torch.equal(dw.out, before)
+    assert int(err.item()) == 0
