@@ -102,7 +102,9 @@ size_t nvkv_page_bytes(int32_t num_kv_heads, int32_t head_dim);
  *                 rows cu_new[b] .. cu_new[b+1]-1 belong to sequence b and are
  *                 written to positions kv_lens[b]-n_b .. kv_lens[b]-1,
  *                 n_b = cu_new[b+1]-cu_new[b].
- *   total_new:    cu_new[batch] (host copy); max_new >= every n_b (host bound).
+ *   total_new:    cu_new[batch] (host copy); max_new >= every n_b (host bound);
+ *                 NVKV_ERR_UNSUPPORTED when (max_new/2 + 1) * Hkv * D/16
+ *                 exceeds 2^31 - 1 (the kernels' 32-bit work-item index).
  * Writes exactly the code nibbles and scale bytes of those positions; every
  * other pool byte, including the other nibble of a shared V code byte, is
  * left as it was.  Sequences must not share pages written by the same call. */

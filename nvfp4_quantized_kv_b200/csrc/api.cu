@@ -1,6 +1,7 @@
 // api.cu -- the extern "C" boundary of libnvkv (declared in include/nvkv.h):
 // host-side argument checks, workspace carving and kernel dispatch.  Nothing
 // here allocates, synchronises or reads device memory.
+#include <climits>
 #include <cmath>
 #include <cstdlib>
 #include <cstring>
@@ -120,6 +121,13 @@ nvkv_status pages_move(const nvkv_cache *cache, const int32_t *page_ids, const i
 }
 
 
+// The append kernels index their work items (slot pair, kv-head, group of
+// 16) with 32-bit integers: max_new/2 + 1 pairs times Hkv * D/16 items
+// must fit.
+bool append_fits(const nvkv_cache &c, int32_t max_new) {
+  return ((int64_t)max_new / 2 + 1) * c.num_kv_heads * (c.head_dim / kGroup) <= INT32_MAX;
+}
+
 // Checks shared by the decode entry points of both cache formats; on
 // success `a` holds the resolved split count and the workspace regions.
 struct DecodeArgs {
@@ -232,6 +240,7 @@ nvkv_status nvkv_append(const nvkv_cache *cache, const nvkv_seqs *seqs, const vo
   if (total_new == 0 || max_new == 0) return NVKV_OK;
   if (!k_new || !v_new || !cu_new || !aligned16(k_new) || !aligned16(v_new))
     return NVKV_ERR_INVALID_ARG;
+  if (!append_fits(*cache, max_new)) return NVKV_ERR_UNSUPPORTED;
   return cuda_status(launch_append(*cache, *seqs, k_new, v_new, cu_new, total_new, max_new,
                                    nullptr, 0, 0, reinterpret_cast<cudaStream_t>(stream)));
 }
@@ -260,6 +269,7 @@ nvkv_status nvkv_append_rope(const nvkv_cache *cache, const nvkv_seqs *seqs, con
   if (total_new == 0 || max_new == 0) return NVKV_OK;
   if (!k_new || !v_new || !cu_new || !aligned16(k_new) || !aligned16(v_new))
     return NVKV_ERR_INVALID_ARG;
+  if (!append_fits(*cache, max_new)) return NVKV_ERR_UNSUPPORTED;
   return cuda_status(launch_append(*cache, *seqs, k_new, v_new, cu_new, total_new, max_new,
                                    rope_cs, rotary_dim, max_pos,
                                    reinterpret_cast<cudaStream_t>(stream)));
@@ -325,6 +335,7 @@ nvkv_status nvkv_append_k8v4(const nvkv_cache *cache, const nvkv_seqs *seqs, con
   if (total_new == 0 || max_new == 0) return NVKV_OK;
   if (!k_new || !v_new || !cu_new || !aligned16(k_new) || !aligned16(v_new))
     return NVKV_ERR_INVALID_ARG;
+  if (!append_fits(*cache, max_new)) return NVKV_ERR_UNSUPPORTED;
   return cuda_status(launch_append_k8v4(*cache, *seqs, k_new, v_new, cu_new, total_new, max_new,
                                         reinterpret_cast<cudaStream_t>(stream)));
 }

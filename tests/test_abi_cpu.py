@@ -251,3 +251,16 @@ def test_k8v4_pages_calls_reject_bad_arguments_without_launch(lib):
         assert f(B(c), 0x10, 0x20, 1, 0x1008, 4, None, None) == nv.ERR_INVALID_ARG
         assert f(B(cache(d=64)), 0x10, 0x20, 1, 0x1000, 4, None, None) == nv.ERR_UNSUPPORTED
         assert f(B(c), 0x10, 0x20, 0, 0x1000, 4, None, None) == nv.OK
+
+
+def test_appends_refuse_item_counts_beyond_32_bits(lib):
+    """The append kernels index (slot pair, kv-head, group) items with 32-bit
+    integers; a max_new whose item count would overflow is refused."""
+    B = ctypes.byref
+    c, s = cache(hkv=64, d=256), seqs()
+    big = 2 ** 31 - 1  # (big/2 + 1) * 64 * 16 items > 2^31
+    assert lib.nvkv_append(B(c), B(s), 0x10, 0x20, 0x30, 1, big, None) == nv.ERR_UNSUPPORTED
+    assert lib.nvkv_append_k8v4(B(c), B(s), 0x10, 0x20, 0x30, 1, big, None) == \
+        nv.ERR_UNSUPPORTED
+    assert lib.nvkv_append_rope(B(c), B(s), 0x10, 0x20, 0x30, 1, big, 0x1000, 16, 64, None) == \
+        nv.ERR_UNSUPPORTED
