@@ -17,8 +17,8 @@ decode tokens/s (B*T query tokens per layer-call / step time) beside it.
 The same JSON line carries, as sub-objects measured after the timed
 region: the T=6 verify on the same pool, page spill / restore through a
 pinned arena, the chunked prefill (TFLOP/s), the fused RoPE + append, a
-decode step replayed from a CUDA Graph, and the decode over a K8V4 cache;
-each is guarded so that its failure is reported in its own object.
+decode step replayed from a CUDA Graph, and the decode over a K8V4 cache
+(the last three are guarded: a failure is reported in its own object).
 
 Launched with torchrun for N > 1: every rank runs its own replica of the
 workload (the path has no cross-GPU exchange); the reported value is the
