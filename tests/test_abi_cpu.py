@@ -264,3 +264,21 @@ def test_appends_refuse_item_counts_beyond_32_bits(lib):
         nv.ERR_UNSUPPORTED
     assert lib.nvkv_append_rope(B(c), B(s), 0x10, 0x20, 0x30, 1, big, 0x1000, 16, 64, None) == \
         nv.ERR_UNSUPPORTED
+
+
+def test_the_library_is_usable_from_plain_c(lib, tmp_path):
+    """A C program compiled against include/nvkv.h and linked with libnvkv.so
+    runs the size functions, the split plan and the argument checks."""
+    import shutil
+    import subprocess
+    cc = shutil.which("gcc") or shutil.which("cc")
+    if cc is None:
+        pytest.skip("no C compiler")
+    exe = str(tmp_path / "abi_from_c")
+    libdir = os.path.dirname(nv.library_path)
+    subprocess.run([cc, "-std=c11", "-Wall", "-Werror", "-I", os.path.join(ROOT, "include"),
+                    os.path.join(ROOT, "tests", "c", "abi_from_c.c"), "-L", libdir, "-lnvkv",
+                    "-Wl,-rpath," + libdir, "-o", exe], check=True, capture_output=True)
+    r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
+    assert r.returncode == 0, r.stderr
+    assert r.stdout.strip() == "ok"
