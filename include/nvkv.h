@@ -8,7 +8,7 @@
  * elements (here: 16 consecutive head_dim elements of one token and one
  * kv-head) shares one E4M3 scale.  The serving features the calls follow are
  * those listed in the "knoopx/ninfer" README, section "Capabilities and
- * limits": one shared, startup-fixed KV pool serving every active request,
+ * limits": a single KV pool, sized at startup, serving every active request,
  * batched decode replayed from CUDA Graphs, MTP speculative verify with one
  * to five draft tokens (T = drafts + 1 causal queries per sequence), and
  * chunked prefill; one GPU.

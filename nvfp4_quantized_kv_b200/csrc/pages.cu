@@ -1,9 +1,10 @@
 // pages.cu -- host KV spill / restore of whole NVFP4 pages.
 //
-// "gzenz/ninfer" README, "Context cache and eviction": when device KV is
-// full, evicted continuations move to a pinned host arena (device to host)
-// and come back (host to device) when the cache is reused; placement in the
-// arena is scatter-gather, so a fragmented arena never blocks a spill.
+// "gzenz/ninfer" README, "Context cache and eviction": once the device pool
+// runs out, the engine copies the KV of the continuations it evicts into an
+// arena of pinned host memory and copies it back to the device when that
+// cache is used again; the arena is filled scatter-gather, so fragmentation
+// of the arena cannot make a spill fail.
 // Here the arena is an array of page-sized slots and a spill or restore is
 // a list of (pool page, arena slot) pairs: one kernel moves every listed
 // page block in 16-byte words, reading and writing pinned host memory

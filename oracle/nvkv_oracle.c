@@ -25,7 +25,7 @@
  *     - there is no second, per-tensor scale.
  *
  *   Paged pool -- "knoopx/ninfer" README, "Quick start" and "Capabilities and
- *   limits" (one shared, startup-fixed KV pool serving all active requests).
+ *   limits" (a single KV pool, sized at startup, serves all active requests).
  *   Pages hold 16 token slots; the byte layout of a page is this project's
  *   own (the pages are silent), written out in pool_offset_* below.
  *
