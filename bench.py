@@ -254,6 +254,9 @@ def main():
     from nvfp4_quantized_kv_b200 import workload as W
     from nvfp4_quantized_kv_b200.harness import DeviceWorkload
 
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py: the native arm needs a CUDA GPU (B200); "
+                         "--impl reference runs on the host cores")
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local = int(os.environ.get("LOCAL_RANK", "0"))

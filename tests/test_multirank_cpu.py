@@ -113,3 +113,12 @@ def test_bench_e2e_byte_counts_are_assigned_once():
     visit(main)
     for name in ("h2d", "d2h", "value", "ms", "kv_bytes", "e2e_ms", "decode_gbs"):
         assert stores.count(name) == 1, name
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU refusal")
+def test_native_arm_refuses_to_run_without_a_gpu():
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--steps", "1",
+                        "--warmup", "3"], capture_output=True, text=True, timeout=300, cwd=ROOT)
+    assert r.returncode == 1
+    assert "needs a CUDA GPU" in r.stderr
+    assert r.stdout.strip() == ""
