@@ -87,6 +87,36 @@ def test_rotation_preserves_pair_norms():
     assert np.allclose(n0, n1, rtol=1e-6, atol=1e-12)
 
 
+def test_float_rotation_is_within_two_roundings_of_the_exact_rotation():
+    """The float rotation against the rotation evaluated in float64 from the
+    same (float) bf16 inputs and table entries, element by element.  The
+    float evaluation x' = fma(x, c, -(y*s)) rounds twice: the product y*s
+    (at most half an ulp of |y*s|) and the fused multiply-add (at most half
+    an ulp of the result), so |x'_float - x'_exact| <= 2^-24 (|y*s| + |x'|)
+    (half an ulp of v is at most 2^-24 |v| for normal floats); the same holds
+    for y' = fma(y, c, x*s) with x*s.  A wrong pairing, sign or table index
+    misses by far more than this bound."""
+    rng = np.random.default_rng(11)
+    D = 256
+    for r, base, scale in ((256, 1e7, 2.12), (64, 1e4, 1.0), (128, 5e5, 3.0)):
+        cs = oracle.rope_table(3000, r, base, scale)
+        h = r // 2
+        for pos in (0, 1, 17, 999, 2999):
+            bits = _bits(rng.standard_normal(D) * 10.0 ** rng.uniform(-2, 2, D))
+            x = (bits.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+            c = cs[pos, :, 0].astype(np.float64)
+            s = cs[pos, :, 1].astype(np.float64)
+            got = oracle.rope_rotate_f32(bits, r, cs[pos]).astype(np.float64)
+            a, b = x[:h], x[h:r]
+            want_a = a * c - b * s
+            want_b = b * c + a * s
+            bound_a = 2.0 ** -24 * (np.abs(b * s) + np.abs(want_a)) * (1 + 2.0 ** -20) + 2.0 ** -140
+            bound_b = 2.0 ** -24 * (np.abs(a * s) + np.abs(want_b)) * (1 + 2.0 ** -20) + 2.0 ** -140
+            assert (np.abs(got[:h] - want_a) <= bound_a).all()
+            assert (np.abs(got[h:r] - want_b) <= bound_b).all()
+            assert np.array_equal(got[r:], x[r:])
+
+
 def _scan_quantize(x):
     """Independent formulation: the E4M3 value nearest to amax/6 by scanning
     the finite E4M3 values (ties to the even mantissa), then the E2M1 value
