@@ -159,21 +159,27 @@ nvkv_status nvkv_combine(const nvkv_seqs *seqs, const void *workspace, int32_t T
  * same q / out layouts), with the split-K partial results kept in a
  * library-owned device array of nvkv_decode_static_scratch_bytes() bytes
  * (8 MiB) instead of caller memory.  The pages describe no such call; it is
- * here for callers that cannot allocate device memory where they run
- * attention (inside a CUDA Graph capture, under an allocator they do not
- * own, or on a path that must not take allocator locks).  It allocates and
- * frees nothing.
+ * here for callers that cannot call cudaMalloc or any other allocator where
+ * they run attention: runtimes whose device memory belongs to a pool they
+ * may not draw from, plugins inside an application that owns all device
+ * memory, and real-time paths that must not take allocator locks or face an
+ * allocation failure.  It allocates and frees nothing.
  *  - Every GPU that loads the library holds the 8 MiB array until the process
  *    exits.
- *  - Shapes whose nvkv_decode_workspace_bytes() exceeds the array return
+ *  - out must be non-NULL and 16-byte aligned (NVKV_ERR_INVALID_ARG, checked
+ *    before anything is launched).  Shapes whose
+ *    nvkv_decode_workspace_bytes() exceeds the array return
  *    NVKV_ERR_WORKSPACE without launching.
  *  - The first call on each device (with that device current) looks up the
- *    array's device address (cudaGetSymbolAddress) and caches it; make that
- *    first call before any stream capture.  NVKV_ERR_CUDA if the lookup fails.
+ *    array's device address (cudaGetSymbolAddress) and caches it for that
+ *    device's CUDA context; a new context (after a device reset) gets a new
+ *    lookup on its first call.  Make that first call before any stream
+ *    capture.  NVKV_ERR_CUDA if the lookup fails.
  *  - All calls on a device share the one array, and it keeps the last call's
- *    contents (nothing needs to start at zero).  Calls whose kernels overlap
- *    on the GPU (different streams without ordering) race on it: order them
- *    on one stream or with events. */
+ *    contents (nothing needs to start at zero: every slot the merge reads is
+ *    written by the same call first).  Calls whose kernels overlap on the GPU
+ *    (different streams without ordering) race on it: order them on one
+ *    stream or with events. */
 size_t nvkv_decode_static_scratch_bytes(void);
 nvkv_status nvkv_decode_attn_static(const nvkv_cache *cache, const nvkv_seqs *seqs,
                                     const void *q, int32_t T, int32_t num_q_heads,

@@ -17,6 +17,9 @@ cudaError_t launch_append_k8v4(const nvkv_cache &, const nvkv_seqs &, const void
 cudaError_t launch_decode_simt(const nvkv_cache &, const nvkv_seqs &, const void *, int, int,
                                float, int, float *, float *, cudaStream_t, bool);
 bool decode_tc_supported(const nvkv_cache &, int, int);
+bool decode_qk4_supported(const nvkv_cache &, int, int);
+cudaError_t launch_decode_qk4(const nvkv_cache &, const nvkv_seqs &, const void *, int, int, float,
+                              int, float *, float *, cudaStream_t);
 cudaError_t launch_decode_tc(const nvkv_cache &, const nvkv_seqs &, const void *, int, int, float,
                              int, float *, float *, cudaStream_t);
 bool prefill_tc_supported(const nvkv_cache &);
@@ -167,13 +170,15 @@ nvkv_status check_prefill(const nvkv_cache *cache, const nvkv_seqs *seqs, const 
   return NVKV_OK;
 }
 
-// NVKV_DECODE_KERNEL=simt forces the CUDA-core decode and prefill kernels
-// (used by the tests to cross-check the two kernel families on the same
-// shapes).
-bool force_simt() {
+// NVKV_DECODE_KERNEL=simt forces the CUDA-core decode and prefill kernels;
+// NVKV_DECODE_KERNEL=tc forces the decode kernel that dequantises K for
+// the f16 tensor-core scores (where it takes the shape).  The tests use
+// them to cross-check the kernel families on the same shapes.
+bool force_kernel(const char *name) {
   const char *v = std::getenv("NVKV_DECODE_KERNEL");
-  return v && std::strcmp(v, "simt") == 0;
+  return v && std::strcmp(v, name) == 0;
 }
+bool force_simt() { return force_kernel("simt"); }
 
 }  // namespace
 
@@ -283,6 +288,9 @@ nvkv_status nvkv_decode_attn(const nvkv_cache *cache, const nvkv_seqs *seqs, con
                                       workspace, workspace_bytes, a);
   if (st != NVKV_OK) return st;
   cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
+  if (!force_simt() && !force_kernel("tc") && decode_qk4_supported(*cache, T, num_q_heads))
+    return cuda_status(
+        launch_decode_qk4(*cache, *seqs, q, T, num_q_heads, sm_scale, a.S, a.ws_o, a.ws_lse, st_));
   if (!force_simt() && decode_tc_supported(*cache, T, num_q_heads))
     return cuda_status(
         launch_decode_tc(*cache, *seqs, q, T, num_q_heads, sm_scale, a.S, a.ws_o, a.ws_lse, st_));

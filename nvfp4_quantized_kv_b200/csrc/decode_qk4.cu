@@ -1,0 +1,898 @@
+// decode_qk4.cu -- split-K GQA decode attention over the NVFP4 paged pool,
+// head_dim 256, up to 6 query rows per (sequence, kv-head): the scores on
+// the NVFP4 block-scaled tensor-core MMA, straight from the cached codes.
+//
+// What it computes is the decode half of the path in the "knoopx/ninfer"
+// README, "Capabilities and limits" (batched decode, MTP verify), over the
+// NVFP4 KV cache of the "gzenz/ninfer" README, "Fork changes vs upstream" ->
+// "Context and model": for every query row (t, g) of kv-head h of sequence
+// b, at position kv_len - T + t, the softmax-weighted sum of the dequantised
+// V rows over the visible keys of one split, as a partial result (o,
+// base-2 log-sum-exp) that nvkv_combine merges.  Same contract, split plan
+// and workspace layout as the other decode kernels.
+//
+// The cache format is the tensor core's own NVFP4 operand format: E2M1 codes
+// packed two per byte (low nibble first) with one unsigned E4M3 scale per 16
+// consecutive elements along the contraction.  K's groups run along
+// head_dim, which is the contraction of the scores, so the K codes the TMA
+// copies into shared memory are the A operand of tcgen05.mma
+// kind::mxf4nvf4 as they are, and the K scale bytes are its scale factors:
+// no K dequantisation at all, and 64 head_dim elements per instruction.
+// The query side must be NVFP4 too.  Each query row x = q * sm_scale * log2(e)
+// (fp32) is written as a sum of L = 8 NVFP4 terms, x = sum_l 2^-k_l * c_l,
+// each term quantising the residual the previous terms left (scale = E4M3 of
+// group amax / 6, codes = E2M1 nearest, after a power-of-two prescale 2^k_l
+// that puts the row maximum in [256, 512)); every term shrinks the residual
+// by at least 5.6x (at most one E2M1 half-gap, scale/1, per element), so
+// the dropped remainder is below 0.177^8 = 1e-6 of each group's maximum.
+// The terms are the N side of the MMA (row r, term l -> column r*L + l), and
+// the softmax recombines each row's L columns with their 2^-k_l factors in
+// fp32.  The products of E2M1 codes and E4M3 scales are exact; the MMA
+// accumulates them in fp32.
+//
+// V's groups run along head_dim, not along the tokens the value sum
+// contracts, so the value sum is an f16 MMA (swap-AB: V^T is the M = 128
+// side).  Its scales move to the other operand: with g(d) the group of
+// head_dim row d,
+//     o[r][d] = sum_j p[r][j] * vscale[j][g(d)] * code[j][d],
+// so the N side holds P'[(r, g)][j] = p[r][j] * vscale[j][g] for every row r
+// and every group g of the 128-row half (N = 8 * rows: 48 at 6 rows, which
+// costs the MMA no more than 16), and each O^T row d keeps the column of its
+// own group.  V^T itself is then the bare codes, built with integer
+// operations: the f16 bit pattern (mag << 9) | (sign << 15) is exactly
+// E2M1(code) * 2^-14 (the E2M1 subnormal 0.5 included), so a 32-bit word of
+// 8 codes becomes four f16 pairs with a shift, two masks and a multiply-add
+// each -- no conversion instructions, which run at a fraction of the rate.
+// The pair of a word holds tokens (t, t+4), so P' uses the same permutation
+// of the tokens along K.  P' = f16(f16(p/4) * vscale) stays below the f16
+// maximum (p <= 2^8 with the lazy maximum, vscale <= 448), and the
+// epilogue applies 2^16 / (4 * denominator).  P comes from an fp32 exp2.
+//
+// Per 128-token unit the tensor pipe runs 4 NVFP4 MMAs (scores) and 16 f16
+// MMAs (values), against 16 + 16 f16 MMAs when K is dequantised, and the
+// CUDA cores convert no code.
+//
+// Roles (one persistent CTA per split-plan range, 448 threads):
+//  * warp 12 (TMA): per page two tiled loads, no multicast: the 16 rows of K
+//    codes (128-byte swizzle, into the unit's contiguous K tile) and the 20
+//    rows of K scales, V codes and V scales (no swizzle); 4-stage ring.
+//  * warps 0..3 copy the unit's K scale bytes into the Tensor Memory
+//    scale-factor layout (every lane quarter holds the same 32 rows);
+//    warps 0..7 write the V^T codes into Tensor Memory (one head_dim row a
+//    lane).
+//  * warps 8..11 (softmax, one token a lane): recombine the terms, mask,
+//    running max raised lazily (only when a score exceeds it by more than
+//    2^8, detected by a vote), fp32 exp2, P' to shared memory, the
+//    denominator from the same f16 weights; at a segment start they build
+//    the query terms.
+//  * warp 13: one thread issues all MMAs.
+//  * Every wait is bounded; a timeout sets NVKV_DEVERR_TIMEOUT, turns later
+//    waits into no-ops and lets the kernel drain and free its Tensor Memory.
+#include <cfloat>
+
+#include "nvkv_common.cuh"
+#include "sm100.cuh"
+
+namespace nvkv {
+namespace {
+
+using namespace sm100;
+
+constexpr int kD = 256;
+constexpr int kRowsPerHead = 36;         // 18*D bytes / 128
+constexpr int kHeadBytes = 18 * kD;      // 4608
+constexpr int kUnitPages = 8;
+constexpr int kKRows = 16;               // K-code rows of a page block (one per token)
+constexpr int kAuxRows = 20;             // K scales (2), V codes (16), V scales (2)
+constexpr int kKPageBytes = kKRows * 128;         // 2048
+constexpr int kAuxPageBytes = kAuxRows * 128;     // 2560
+constexpr int kKTileBytes = kUnitPages * kKPageBytes;      // 16384
+constexpr int kStageBytes = kKTileBytes + kUnitPages * kAuxPageBytes;  // 36864
+constexpr int kAuxKs = 0, kAuxVc = 256, kAuxVs = 2304;    // offsets inside a page's aux block
+constexpr int kStages = 4;
+
+constexpr int kRowsCap = 6;              // query rows per pair (T * G) this kernel takes
+constexpr int kTerms = 8;                // NVFP4 terms per query row
+constexpr int kNSMax = kRowsCap * kTerms;   // 48: largest N of the score MMA
+constexpr int kHalfGroups = 8;           // scale groups in a 128-row half of head_dim
+constexpr int kNPMax = kRowsCap * kHalfGroups;  // 48: largest N of the value MMA
+constexpr int kNP = 16;                  // rows of the per-row scratch arrays
+
+constexpr int kDeqWarps = 8;             // warps 0..7
+constexpr int kSmxWarp0 = 8;             // warps 8..11
+constexpr int kSmxWarps = 4;
+constexpr int kProducerWarp = 12;
+constexpr int kMmaWarp = 13;             // issues the score MMAs
+constexpr int kPvWarp = 14;              // issues the value MMAs
+constexpr int kThreads = 15 * 32;
+constexpr int kSegThreads = (kDeqWarps + kSmxWarps) * 32;
+constexpr uint32_t kTmemCols = 512;
+constexpr long long kWaitBudget = 2000000000LL;  // clock cycles (~1 s)
+constexpr float kLazyRescale = 8.0f;             // log2 units
+
+// Tensor Memory columns.
+constexpr uint32_t kColV = 0;      // 2 slots x 128: V^T codes (d-half h at +64h), f16 token pairs
+constexpr uint32_t kColS = 256;    // 2 slots x kNSMax: S^T, fp32, one token per lane
+constexpr uint32_t kColO = 352;    // 2 halves x kNPMax: O^T per (row, group), fp32
+constexpr uint32_t kColSFA = 448;  // 2 slots x 16: K scale factors, column 4*ks + m1
+constexpr uint32_t kColSFB = 480;  // 4 x 4: query-term scale factors, column 4*ks + n1 (n1 < 2)
+static_assert(kColS + 2 * kNSMax <= kColO && kColO + 2 * kNPMax <= kColSFA &&
+                  kColSFB + 16 <= kTmemCols, "tensor memory");
+
+// Shared memory (offsets from a 1024-byte aligned base).
+constexpr int kOffQ = kStages * kStageBytes;        // query terms, kNSMax rows x 128 B, swizzled
+constexpr int kOffP = kOffQ + kNSMax * 128;         // P' tiles [slot][half], MN-major f16
+constexpr int kPHalfBytes = kRowsCap * 2048;        // (row r, group g) x 128 tokens
+constexpr int kPSlotBytes = 2 * kPHalfBytes;
+constexpr int kOffSfb = kOffP + 2 * kPSlotBytes;    // [kNSMax][16] scale bytes of the terms
+constexpr int kOffFac = kOffSfb + kNSMax * 16;      // float [kRowsCap]: 2^-k of each row's terms
+constexpr int kOffRed = kOffFac + kNSMax * 4;       // float [4][kNP]
+constexpr int kOffMask = kOffRed + kSmxWarps * kNP * 4;  // u32 [2][4][4]
+constexpr int kOffM = kOffMask + 2 * kSmxWarps * 4 * 4;  // float [kNP]
+constexpr int kOffAlpha = kOffM + kNP * 4;
+constexpr int kOffNvis = kOffAlpha + kNP * 4;
+constexpr int kOffFlags = kOffNvis + kNP * 4;        // int[4]: abort at [2]
+constexpr int kOffPages = kOffFlags + 16;            // int[stages][8]
+constexpr int kOffBars = kOffPages + kStages * kUnitPages * 4;
+constexpr int kNumBars = 2 * kStages + 13;
+constexpr int kOffTmem = kOffBars + kNumBars * 8;
+constexpr int kSmemBytes = kOffTmem + 16 + 1024;    // + alignment slack
+static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+static_assert(kOffQ % 1024 == 0 && kStageBytes % 1024 == 0 && kOffP % 16 == 0 &&
+                  kOffSfb % 16 == 0 && kOffPages % 16 == 0 && kOffBars % 8 == 0,
+              "alignment");
+
+struct Shared {
+  uint8_t *stages, *qtile, *ptile, *sfb;
+  float *fac, *red, *m_s, *alpha_s;
+  int32_t *nvis_s, *pages;
+  uint32_t *masks;
+  volatile int *flags;
+  // Barriers of the per-slot resources exist once per slot: slot s completes
+  // once per unit with (unit & 1) == s, so a parity wait is never more than
+  // one phase behind.
+  uint64_t *full, *empty, *sfa_ready, *sready, *pready, *vready, *pvdone, *qready, *final_bar,
+      *final_pv;
+  uint32_t *tmem_slot;
+};
+
+__device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *flags,
+                                         int32_t *err) {
+  if (flags[2]) return false;  // aborted: do not wait any more
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (flags[2]) return false;
+    if (clock64() - t0 > kWaitBudget) {
+      flags[2] = 1;
+      report(err, NVKV_DEVERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+
+// Segment of the CTA's range: units [u, seg_end) of pair (b, h).
+struct Seg {
+  int b, h, kv_len;
+  int64_t pair_start, seg_end;
+  bool bad;
+};
+
+__device__ __forceinline__ Seg segment_at(int64_t u, int64_t u1, const int32_t *kv_lens, int B,
+                                          int Hkv, int max_kv_len, int max_pages) {
+  Seg s;
+  int units;
+  locate_pair(kv_lens, B, Hkv, u, s.b, s.h, s.pair_start, units);
+  s.seg_end = min(u1, s.pair_start + units);
+  s.kv_len = kv_lens[s.b];
+  s.bad = s.kv_len > max_kv_len || s.kv_len > max_pages * kPageTokens;
+  if (s.bad) s.kv_len = 0;  // nothing of a bad sequence is read
+  return s;
+}
+
+__device__ __forceinline__ int page_of(const int32_t *pt_row, int tok, int kv_len, int num_pages) {
+  if (tok >= kv_len) return -1;
+  const int p = pt_row[tok / kPageTokens];
+  return (p >= 0 && p < num_pages) ? p : -1;
+}
+
+// 2^k as a float for -126 <= k <= 127 (exact).
+__device__ __forceinline__ float pow2f(int k) { return __int_as_float((k + 127) << 23); }
+// x * 2^k for -252 <= k <= 254 as two exact power-of-two multiplies (the
+// result is exact unless it leaves the float range).
+__device__ __forceinline__ float scale_pow2(float x, int k) {
+  const int k1 = k / 2;
+  return x * pow2f(k1) * pow2f(k - k1);
+}
+
+// Four f16 pairs from a word of 8 E2M1 codes (code i in bits 4i..4i+3):
+// pair t holds codes t (low half) and t+4 (high half), each as the f16 bit
+// pattern (mag << 9) | (sign << 15) = E2M1(code) * 2^-14, exactly.  The
+// shift puts code t at bits 9..12 and code t+4 at bits 25..28; the masks keep
+// the magnitudes and the sign bits, and the multiply-add moves the sign bits
+// 12 and 28 up to 15 and 31.
+template <int t>
+__device__ __forceinline__ uint32_t code_pair(uint32_t w) {
+  const uint32_t a = t < 3 ? (w << (9 - 4 * t)) : (w >> 3);
+  return (a & 0x10001000u) * 8u + (a & 0x0E000E00u);
+}
+
+template <int RM>
+__global__ void __launch_bounds__(kThreads, 1)
+decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
+                  const __grid_constant__ CUtensorMap tmap_aux, int num_pages, int Hkv,
+                  const int32_t *__restrict__ page_table, int max_pages,
+                  const int32_t *__restrict__ kv_lens, int B, int max_kv_len,
+                  const __nv_bfloat16 *__restrict__ q, int T, int Hq, float qscale, int S,
+                  float *__restrict__ ws_o, float *__restrict__ ws_lse, int32_t *err) {
+  // RM: query rows per pair rounded up to an even count (padding rows are
+  // zero); the score MMA has N = RM * kTerms columns.
+  static_assert(RM % 2 == 0 && RM >= 2 && RM <= kRowsCap, "rows");
+  constexpr int NS = RM * kTerms;        // score MMA: (row, term) columns
+  constexpr int NP = RM * kHalfGroups;   // value MMA: (row, group of the half) columns
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
+                                              ~uintptr_t(1023));
+  Shared sh;
+  sh.stages = smem;
+  sh.qtile = smem + kOffQ;
+  sh.ptile = smem + kOffP;
+  sh.sfb = smem + kOffSfb;
+  sh.fac = reinterpret_cast<float *>(smem + kOffFac);
+  sh.red = reinterpret_cast<float *>(smem + kOffRed);
+  sh.masks = reinterpret_cast<uint32_t *>(smem + kOffMask);
+  sh.m_s = reinterpret_cast<float *>(smem + kOffM);
+  sh.alpha_s = reinterpret_cast<float *>(smem + kOffAlpha);
+  sh.nvis_s = reinterpret_cast<int32_t *>(smem + kOffNvis);
+  sh.flags = reinterpret_cast<volatile int *>(smem + kOffFlags);
+  sh.pages = reinterpret_cast<int32_t *>(smem + kOffPages);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBars);
+  sh.full = bars;
+  sh.empty = bars + kStages;
+  sh.sfa_ready = bars + 2 * kStages;  // [2]
+  sh.sready = sh.sfa_ready + 2;       // [2]
+  sh.pready = sh.sfa_ready + 4;       // [2]
+  sh.vready = sh.sfa_ready + 6;       // [2]
+  sh.pvdone = sh.sfa_ready + 8;       // [2]
+  sh.qready = sh.sfa_ready + 10;
+  sh.final_bar = sh.sfa_ready + 11;
+  sh.final_pv = sh.sfa_ready + 12;
+  sh.tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffTmem);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int G = Hq / Hkv;
+  const int R = T * G;
+
+  if (threadIdx.x == 0) {
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&sh.full[i], 1);
+      // the score MMAs' commit, the V-code readers and the V-scale readers
+      mbar_init(&sh.empty[i], 1 + kDeqWarps + kSmxWarps);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&sh.sfa_ready[i], 4);
+      mbar_init(&sh.sready[i], 1);
+      mbar_init(&sh.pready[i], kSmxWarps);
+      mbar_init(&sh.vready[i], kDeqWarps);
+      mbar_init(&sh.pvdone[i], 1);
+    }
+    mbar_init(sh.qready, kSmxWarps);
+    mbar_init(sh.final_bar, 1);
+    mbar_init(sh.final_pv, 1);
+    fence_mbar_init();
+  }
+  if (threadIdx.x < 4) sh.flags[threadIdx.x] = 0;
+  if (warp == kMmaWarp) {
+    tmem_alloc(sh.tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  fence_proxy_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *sh.tmem_slot;
+
+  int64_t U = 0;
+  for (int b = 0; b < B; ++b) U += (int64_t)units_of_len(kv_lens[b]) * Hkv;
+  const int c = blockIdx.x;
+  const int64_t u0 = U > 0 ? range_begin(c, U, S) : 0;
+  const int64_t u1 = U > 0 ? range_begin(c + 1, U, S) : 0;
+
+  if (warp == kProducerWarp) {
+    // ------------------------------------------------------------------ TMA
+    // Lane p < 8 owns page p of a unit; the page ids of unit u+1 are loaded
+    // while unit u's copies are issued.
+    prefetch_tmap(&tmap_k);
+    prefetch_tmap(&tmap_aux);
+    const int p = lane & 7;
+    int64_t u = u0;
+    Seg sg = segment_at(u, u1, kv_lens, B, Hkv, max_kv_len, max_pages);
+    auto page_for = [&](const Seg &g, int64_t uu) -> int {
+      const int tok = (int)(uu - g.pair_start) * kUnitTokens + p * kPageTokens;
+      const int32_t *pt = page_table + (size_t)g.b * max_pages;
+      const int pg = page_of(pt, tok, g.kv_len, num_pages);
+      if (lane < kUnitPages && tok < g.kv_len && pg < 0) report(err, NVKV_DEVERR_PAGE_ID);
+      return pg;
+    };
+    int cur = u < u1 ? page_for(sg, u) : -1;
+    uint32_t uc = 0;
+    for (; u < u1; ++u, ++uc) {
+      const int stage = uc % kStages;
+      int nxt = -1;
+      Seg nsg = sg;
+      if (u + 1 < u1) {
+        if (u + 1 >= sg.seg_end) nsg = segment_at(u + 1, u1, kv_lens, B, Hkv, max_kv_len, max_pages);
+        nxt = page_for(nsg, u + 1);
+      }
+      if (uc >= (uint32_t)kStages) {
+        if (lane == 0) wait_bar(&sh.empty[stage], ((uc / kStages) + 1) & 1, sh.flags, err);
+        __syncwarp();
+      }
+      const bool mine = lane < kUnitPages && cur >= 0;
+      if (lane < kUnitPages) sh.pages[stage * kUnitPages + lane] = cur;
+      const uint32_t bytes = __popc(__ballot_sync(0xffffffffu, mine)) * kHeadBytes;
+      __syncwarp();
+      if (lane == 0) mbar_arrive_expect_tx(&sh.full[stage], bytes);
+      __syncwarp();
+      if (mine) {
+        uint8_t *st = sh.stages + stage * kStageBytes;
+        const int y = (cur * Hkv + sg.h) * kRowsPerHead;
+        tma_load_2d(st + lane * kKPageBytes, &tmap_k, 0, y, &sh.full[stage]);
+        tma_load_2d(st + kKTileBytes + lane * kAuxPageBytes, &tmap_aux, 0, y + kKRows,
+                    &sh.full[stage]);
+      }
+      cur = nxt;
+      sg = nsg;
+    }
+    // Drain: every issued copy must land before the CTA may exit.
+    if (lane == 0) {
+      const uint32_t first = uc > (uint32_t)kStages ? uc - kStages : 0;
+      for (uint32_t k = first; k < uc; ++k)
+        mbar_wait(&sh.full[k % kStages], (k / kStages) & 1, kWaitBudget);
+    }
+    __syncwarp();
+  } else if (warp == kMmaWarp || warp == kPvWarp) {
+    // ------------------------------------------------------------------ MMA
+    // Two issuing threads: issuing a batch of tcgen05.mma blocks the thread
+    // until the batch has nearly executed, so a single thread would leave
+    // the tensor pipe idle while it waits for the next step's inputs.  One
+    // thread issues the scores of each unit as soon as its tiles, scale
+    // factors, query terms and S^T slot are ready; the other issues the
+    // value MMAs of each unit once its V^T codes and P' are ready.  Each
+    // commits its own MMAs; the tensor pipe runs both streams.
+    if (lane == 0) {
+      const uint32_t n_units = (uint32_t)(u1 - u0);
+      int64_t seg_end = segment_at(u0, u1, kv_lens, B, Hkv, max_kv_len, max_pages).seg_end;
+      bool issued = false;
+      if (warp == kMmaWarp) {
+        const uint32_t idesc_qk = idesc_nvf4(128, NS);
+        const uint32_t qb = smem_u32(sh.qtile);
+        const uint32_t kt0 = smem_u32(sh.stages);
+        uint32_t seg_idx = 0;
+        for (uint32_t qk = 0; qk < n_units && !sh.flags[2]; ++qk) {
+          const int64_t uu = u0 + qk;
+          const bool opens = qk == 0 || uu >= seg_end;
+          if (uu >= seg_end) {
+            seg_end = segment_at(uu, u1, kv_lens, B, Hkv, max_kv_len, max_pages).seg_end;
+            ++seg_idx;
+          }
+          if (opens) wait_bar(sh.qready, seg_idx & 1, sh.flags, err);
+          const int stage = qk % kStages;
+          wait_bar(&sh.full[stage], (qk / kStages) & 1, sh.flags, err);
+          wait_bar(&sh.sfa_ready[qk & 1], (qk >> 1) & 1, sh.flags, err);
+          // S^T slot qk&1 was read by the softmax of unit qk-2
+          if (qk > 1) wait_bar(&sh.pready[qk & 1], ((qk >> 1) + 1) & 1, sh.flags, err);
+          tc_fence_after();
+          const uint32_t sslot = tmem + kColS + (qk & 1) * kNSMax;
+          const uint32_t sfa = tmem + kColSFA + (qk & 1) * 16;
+          const uint32_t kt = kt0 + stage * kStageBytes;
+#pragma unroll
+          for (int ks = 0; ks < 4; ++ks)
+            mma_nvf4_ss(sslot, smem_desc_sw128(kt + 32 * ks), smem_desc_sw128(qb + 32 * ks),
+                        idesc_qk, ks > 0, sfa + 4 * ks, tmem + kColSFB + 4 * ks);
+          mma_commit(&sh.sready[qk & 1]);
+          mma_commit(&sh.empty[stage]);  // the K tile has been read
+          issued = true;
+        }
+        if (issued) {
+          mma_commit(sh.final_bar);
+          mbar_wait(sh.final_bar, 0, kWaitBudget);
+        }
+      } else {
+        const uint32_t idesc_pv = idesc_f16_f32(128, NP, false, true);
+        const uint32_t pb = smem_u32(sh.ptile);
+        for (uint32_t pv = 0; pv < n_units && !sh.flags[2]; ++pv) {
+          const int64_t uu = u0 + pv;
+          const bool first = pv == 0 || uu >= seg_end;  // O^T starts from zero
+          if (uu >= seg_end)
+            seg_end = segment_at(uu, u1, kv_lens, B, Hkv, max_kv_len, max_pages).seg_end;
+          wait_bar(&sh.vready[pv & 1], (pv >> 1) & 1, sh.flags, err);
+          wait_bar(&sh.pready[pv & 1], (pv >> 1) & 1, sh.flags, err);
+          tc_fence_after();
+          const uint32_t pslot = pb + (pv & 1) * kPSlotBytes;
+          const uint32_t vslot = tmem + kColV + (pv & 1) * 128;
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint32_t acc = (!first) || ks > 0;
+#pragma unroll
+            for (int hf = 0; hf < 2; ++hf)
+              mma_f16_ts(tmem + kColO + hf * kNPMax, vslot + 64 * hf + ks * 8,
+                         smem_desc(pslot + hf * kPHalfBytes + ks * 256, 128, 2048), idesc_pv,
+                         acc);
+          }
+          mma_commit(&sh.pvdone[pv & 1]);
+          issued = true;
+        }
+        if (issued) {
+          mma_commit(sh.final_pv);
+          mbar_wait(sh.final_pv, 0, kWaitBudget);
+        }
+      }
+    }
+  } else {
+    // -------------------------------------------------------------- workers
+    const bool smx = warp >= kSmxWarp0;
+    const int lq = warp & 3;                   // lane quarter of Tensor Memory
+    const int hv = smx ? 0 : ((warp >> 2) & 1);  // V^T half of a code-writing warp
+    const uint32_t tl = tmem + ((uint32_t)(32 * lq) << 16);
+    const int stid = threadIdx.x - kSmxWarp0 * 32;  // softmax thread 0..127
+    float l_part[RM], facr[RM];
+#pragma unroll
+    for (int i = 0; i < RM; ++i) l_part[i] = facr[i] = 0.f;
+
+    uint32_t uc = 0;
+    uint32_t seg_idx = 0;
+    for (int64_t u = u0; u < u1; ++seg_idx) {
+      const Seg sg = segment_at(u, u1, kv_lens, B, Hkv, max_kv_len, max_pages);
+      if (sg.bad && threadIdx.x == 0) report(err, NVKV_DEVERR_LENGTH);
+      const int64_t seg_start = u;
+      const size_t slot = (size_t)c + (size_t)sg.b * Hkv + sg.h;
+
+      if (smx) {
+        // ---- query terms of this pair (the previous segment's score MMAs
+        // have completed: its last softmax waited for them) ----
+        if (stid < kNP) {
+          sh.nvis_s[stid] = stid < R ? sg.kv_len - T + stid / G + 1 : 0;
+          sh.m_s[stid] = -INFINITY;
+        }
+#pragma unroll
+        for (int i = 0; i < RM; ++i) l_part[i] = 0.f;
+        // Row r of x = q * sm_scale * log2(e): one power-of-two prescale 2^k
+        // puts the row maximum in [256, 512); then term l quantises the
+        // residual y (group scale = E4M3 of its 16-element maximum / 6,
+        // codes = nearest E2M1) and leaves y - term, exactly.  Each term
+        // shrinks every group's residual at least 5.6x, so the scales of the
+        // 8 terms stay inside the E4M3 range (448 down to 2^-9) until the
+        // remainder is below about 2^-15 of the row maximum.  The MMA's
+        // columns r*8 .. r*8+7 summed and times 2^-k give the row's scores.
+        // (Any rounding of the scales and codes would do: only the residual
+        // bookkeeping has to be exact.)
+        for (int r = lq; r < RM; r += kSmxWarps) {
+          float y[8];
+          if (r < R) {
+            const int t = r / G, g = r % G;
+            const uint4 raw = *reinterpret_cast<const uint4 *>(
+                q + ((size_t)(sg.b * T + t) * Hq + sg.h * G + g) * kD + 8 * lane);
+            const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              y[2 * i] = __uint_as_float(w[i] << 16) * qscale;
+              y[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u) * qscale;
+            }
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) y[i] = 0.f;
+          }
+          float a = 0.f;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(y[i]));
+          a = warp_max(a);
+          // A row whose largest element is below the smallest normal float
+          // (2^-126) is taken as zero: its scores would be below 2^-110.
+          const int eb = (int)((__float_as_uint(a) >> 23) & 0xffu);  // biased exponent
+          const int k = 135 - eb;  // a in [2^(eb-127), 2^(eb-126)): a * 2^k in [256, 512)
+          if (eb > 0) {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) y[i] = scale_pow2(y[i], k);
+          } else {
+#pragma unroll
+            for (int i = 0; i < 8; ++i) y[i] = 0.f;
+          }
+#pragma unroll 1
+          for (int l = 0; l < kTerms; ++l) {
+            const int n = r * kTerms + l;
+            float ga = 0.f;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) ga = fmaxf(ga, fabsf(y[i]));
+            ga = fmaxf(ga, __shfl_xor_sync(0xffffffffu, ga, 1));  // 16-element group
+            const uint32_t sb = (uint32_t)__nv_cvt_float_to_fp8(ga * (1.0f / 6.0f), __NV_SATFINITE,
+                                                                __NV_E4M3);
+            const float sv = e4m3_to_float((uint8_t)sb);
+            const float rs = sv > 0.f ? 1.0f / sv : 0.f;
+            uint32_t codes = 0;
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+              // codes of y/s (the hardware's rounding; any choice is exact
+              // bookkeeping below), then the chosen values, exact in f16
+              const uint32_t pair = f32x2_to_e2m1x2(y[2 * i] * rs, y[2 * i + 1] * rs);
+              codes |= pair << (8 * i);
+              const float2 v = f16x2_to_float2(e2m1x2_to_f16x2(pair));
+              y[2 * i] -= v.x * sv;  // the products are exact
+              y[2 * i + 1] -= v.y * sv;
+            }
+            // Row n of the term tile: bytes 4*lane..4*lane+3, 128-byte swizzle.
+            *reinterpret_cast<uint32_t *>(sh.qtile + n * 128 + (((lane >> 2) ^ (n & 7)) << 4) +
+                                          (lane & 3) * 4) = codes;
+            if ((lane & 1) == 0) sh.sfb[n * 16 + (lane >> 1)] = (uint8_t)sb;
+          }
+          if (lane == 0) sh.fac[r] = eb > 0 ? scale_pow2(1.f, -k) : 0.f;
+        }
+        fence_proxy_async_smem();
+        named_barrier(1, kSmxWarps * 32);
+#pragma unroll
+        for (int r = 0; r < RM; ++r) facr[r] = sh.fac[r];
+        // Scale factors of the terms into Tensor Memory (each lane quarter
+        // holds all rows): column 4*ks + n1, lane l -> row 32*n1 + l (every
+        // K step's block starts on a multiple of 4 columns).
+        {
+          uint32_t w[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) w[i] = 0u;
+#pragma unroll
+          for (int n1 = 0; n1 < 2; ++n1) {
+            const uint4 v = *reinterpret_cast<const uint4 *>(sh.sfb + (32 * n1 + lane) * 16);
+            w[0 * 4 + n1] = v.x;
+            w[1 * 4 + n1] = v.y;
+            w[2 * 4 + n1] = v.z;
+            w[3 * 4 + n1] = v.w;
+          }
+          tmem_st16(tl + kColSFB, w);
+          tmem_wait_st();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sh.qready);
+      }
+
+      for (; u < sg.seg_end; ++u, ++uc) {
+        const bool first = (u == seg_start);
+        const int stage = uc % kStages;
+        const uint8_t *stg = sh.stages + stage * kStageBytes;
+        const uint8_t *aux = stg + kKTileBytes;
+        const int tok0 = (int)(u - sg.pair_start) * kUnitTokens;
+        if (!smx) {
+          wait_bar(&sh.full[stage], (uc / kStages) & 1, sh.flags, err);
+          if (warp < 4) {
+            // ---- K scale factors into slot uc&1 (read by the score MMAs of
+            // unit uc-2 before) ----
+            if (uc > 1) {
+              wait_bar(&sh.sready[uc & 1], ((uc >> 1) + 1) & 1, sh.flags, err);
+              tc_fence_after();
+            }
+            uint32_t w[16];
+#pragma unroll
+            for (int m1 = 0; m1 < 4; ++m1) {
+              const int j = 32 * m1 + lane;  // token of the unit
+              const uint4 v = *reinterpret_cast<const uint4 *>(aux + (j >> 4) * kAuxPageBytes +
+                                                               kAuxKs + (j & 15) * 16);
+              w[0 * 4 + m1] = v.x;
+              w[1 * 4 + m1] = v.y;
+              w[2 * 4 + m1] = v.z;
+              w[3 * 4 + m1] = v.w;
+            }
+            tmem_st16(tl + kColSFA + (uc & 1) * 16, w);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.sfa_ready[uc & 1]);
+          }
+          // ---- V^T codes into slot uc&1 (read by the value MMAs of uc-2):
+          // head_dim row d = 128*hv + 32*lq + lane, all 8 pages.
+          // Every code gives a finite value, so the slots of absent tokens
+          // need no clearing: their weights P' are zero. ----
+          if (uc > 1) {
+            wait_bar(&sh.pvdone[uc & 1], ((uc >> 1) + 1) & 1, sh.flags, err);
+            tc_fence_after();
+          }
+          {
+            const int d = 128 * hv + 32 * lq + lane;
+            const uint32_t vcol = kColV + (uc & 1) * 128 + 64 * hv;
+#pragma unroll
+            for (int p = 0; p < kUnitPages; ++p) {
+              const uint2 cw =
+                  *reinterpret_cast<const uint2 *>(aux + p * kAuxPageBytes + kAuxVc + d * 8);
+              const uint32_t o8[8] = {code_pair<0>(cw.x), code_pair<1>(cw.x), code_pair<2>(cw.x),
+                                      code_pair<3>(cw.x), code_pair<0>(cw.y), code_pair<1>(cw.y),
+                                      code_pair<2>(cw.y), code_pair<3>(cw.y)};
+              tmem_st8(tl + vcol + 8 * p, o8);
+            }
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) {
+              mbar_arrive(&sh.vready[uc & 1]);
+              mbar_arrive(&sh.empty[stage]);  // this warp's reads of the stage are done
+            }
+          }
+        } else {
+          // ---- softmax on S^T slot uc&1: thread = token tok0 + 32*lq + lane ----
+          const int pos = tok0 + 32 * lq + lane;
+          // The token's V scales (one per group of 16 head_dim elements) as
+          // f16 pairs of groups (2k, 2k+1), read as soon as the stage has
+          // landed, before the scores are ready.  A token without data (past
+          // kv_len, or an absent page) gets zero scales, so whatever its
+          // bytes hold cannot reach the sum.
+          wait_bar(&sh.full[stage], (uc / kStages) & 1, sh.flags, err);
+          const int pg = (32 * lq + lane) >> 4, i = lane & 15;
+          uint32_t sc2[kHalfGroups];
+          {
+            const bool tok_ok = pos < sg.kv_len && sh.pages[stage * kUnitPages + pg] >= 0;
+            const uint8_t *vs = aux + pg * kAuxPageBytes + kAuxVs + i;
+#pragma unroll
+            for (int k2 = 0; k2 < kHalfGroups; ++k2) {
+              const uint32_t two =
+                  (uint32_t)vs[(2 * k2) * 16] | ((uint32_t)vs[(2 * k2 + 1) * 16] << 8);
+              sc2[k2] = tok_ok ? e4m3x2_to_f16x2(two) : 0u;
+            }
+          }
+          wait_bar(&sh.sready[uc & 1], (uc >> 1) & 1, sh.flags, err);
+          tc_fence_after();
+          const bool vis_all = tok0 + kUnitTokens <= sg.kv_len - T + 1;
+          const uint32_t sslot = tl + kColS + (uc & 1) * kNSMax;
+          uint32_t *my_mask = sh.masks + ((uc & 1) * kSmxWarps + lq) * 4;
+          // Scores of the rows: the sum of each row's 8 term columns (packed
+          // fp32 adds) times the row's 2^-k; invisible keys and padding rows
+          // -inf.
+          auto load_scores = [&](float (&x)[RM]) {
+            uint32_t rr[NS];
+#pragma unroll
+            for (int c32 = 0; c32 < NS / 32; ++c32) tmem_ld32(sslot + 32 * c32, rr + 32 * c32);
+            if (NS % 32) tmem_ld16(sslot + NS - 16, *reinterpret_cast<uint32_t(*)[16]>(rr + NS - 16));
+            tmem_wait_ld();
+#pragma unroll
+            for (int r = 0; r < RM; ++r) {
+              const uint32_t *c8 = rr + r * kTerms;
+              const float2 a0 = add_f32x2(make_float2(__uint_as_float(c8[0]), __uint_as_float(c8[1])),
+                                          make_float2(__uint_as_float(c8[2]), __uint_as_float(c8[3])));
+              const float2 a1 = add_f32x2(make_float2(__uint_as_float(c8[4]), __uint_as_float(c8[5])),
+                                          make_float2(__uint_as_float(c8[6]), __uint_as_float(c8[7])));
+              const float2 a2 = add_f32x2(a0, a1);
+              const float sc = (a2.x + a2.y) * facr[r];
+              const int nv = vis_all ? (r < R ? 0x7fffffff : 0) : sh.nvis_s[r];
+              x[r] = pos < nv ? sc : -INFINITY;
+            }
+          };
+          float x[RM], m[RM];
+          load_scores(x);
+          // A running max of -inf (no key seen yet) is taken as -FLT_MAX, so
+          // an invisible key gives weight 0 and a visible one forces the slow
+          // path, never -inf - -inf.
+#pragma unroll
+          for (int r = 0; r < RM; ++r) m[r] = fmaxf(sh.m_s[r], -FLT_MAX);
+          // Weights of the value MMA: f16(p/4) in both halves of a pair, p =
+          // 2^(score - running max) in fp32 (2^-inf = 0).
+          uint32_t pq2[RM];
+          bool up = false;
+          auto weights = [&]() {
+#pragma unroll
+            for (int r = 0; r < RM; ++r) {
+              const float dd = x[r] - m[r];
+              up |= dd > kLazyRescale;
+              pq2[r] = ex2_quarter_f16x2(dd);
+            }
+          };
+          weights();
+          const uint32_t wup = __ballot_sync(0xffffffffu, up);
+          if (lane == 0) my_mask[0] = wup;
+          named_barrier(1, kSmxWarps * 32);
+          uint32_t any = 0;
+#pragma unroll
+          for (int w = 0; w < kSmxWarps; ++w) any |= sh.masks[((uc & 1) * kSmxWarps + w) * 4];
+          if (any) {
+            // Slow path (the first unit of a segment and rare max raises):
+            // exact row maxima, new running max, rescale of everything
+            // accumulated against the old max, weights recomputed.
+#pragma unroll
+            for (int r = 0; r < RM; ++r) {
+              const float wm = warp_max(x[r]);
+              if (lane == 0) sh.red[lq * kNP + r] = wm;
+            }
+            named_barrier(1, kSmxWarps * 32);
+            if (stid < kNP) {
+              const int n = stid;
+              float alpha = 1.f;
+              if (n < R) {
+                float tmax = -INFINITY;
+#pragma unroll
+                for (int w = 0; w < kSmxWarps; ++w) tmax = fmaxf(tmax, sh.red[w * kNP + n]);
+                const float m_old = sh.m_s[n];
+                if (tmax > -INFINITY && (m_old == -INFINITY || tmax > m_old + kLazyRescale)) {
+                  alpha = exp2f(m_old - tmax);  // 0 when the old max was -inf
+                  sh.m_s[n] = tmax;
+                }
+              }
+              sh.alpha_s[n] = alpha;
+            }
+            named_barrier(1, kSmxWarps * 32);
+#pragma unroll
+            for (int n = 0; n < RM; ++n) l_part[n] *= sh.alpha_s[n];
+            if (!first) {
+              // O^T rows d = 32*lq + lane and d + 128, accumulated up to the
+              // previous unit, scale by alpha once its value MMAs finished.
+              wait_bar(&sh.pvdone[(uc - 1) & 1], ((uc - 1) >> 1) & 1, sh.flags, err);
+              tc_fence_after();
+#pragma unroll
+              for (int half = 0; half < 2; ++half) {
+#pragma unroll
+                for (int r = 0; r < RM; ++r) {  // the 8 group columns of row r
+                  uint32_t r8[8];
+                  const uint32_t col = tl + kColO + half * kNPMax + r * kHalfGroups;
+                  tmem_ld8(col, r8);
+                  tmem_wait_ld();
+                  const float al = sh.alpha_s[r];
+#pragma unroll
+                  for (int j = 0; j < 8; ++j) r8[j] = __float_as_uint(__uint_as_float(r8[j]) * al);
+                  tmem_st8(col, r8);
+                }
+              }
+              tmem_wait_st();
+            }
+#pragma unroll
+            for (int r = 0; r < RM; ++r) m[r] = fmaxf(sh.m_s[r], -FLT_MAX);
+            weights();
+          }
+          // P' into slot uc&1 (read by the value MMAs of unit uc-2 before):
+          // for each half of head_dim and each row r, the 8 values
+          // f16(p_r/4) * vscale[g] of the half's groups g, as the MN-major B
+          // operand: element (n = 8r + g, k) at (n/8)*2048 + (k/8)*128 +
+          // (k%8)*16 + (n%8)*2.  Token slot i of page pg sits at K position
+          // k = 16*pg + 8*(i/8) + 2*(i%4) + (i/4)%2, the order of the V^T
+          // code pairs.  A token without data (past kv_len, or an absent
+          // page) gets zero scales, so whatever its bytes hold cannot reach
+          // the sum.
+          if (uc > 1) {
+            wait_bar(&sh.pvdone[uc & 1], ((uc >> 1) + 1) & 1, sh.flags, err);
+            tc_fence_after();
+          }
+          {
+            const int kk = 16 * pg + 8 * (i >> 3) + 2 * (i & 3) + ((i >> 2) & 1);
+            uint8_t *pt = sh.ptile + (uc & 1) * kPSlotBytes + (kk >> 3) * 128 + (kk & 7) * 16;
+#pragma unroll
+            for (int half = 0; half < 2; ++half)
+#pragma unroll
+              for (int r = 0; r < RM; ++r)
+                *reinterpret_cast<uint4 *>(pt + half * kPHalfBytes + r * 2048) = make_uint4(
+                    hmul2_u32(pq2[r], sc2[4 * half + 0]), hmul2_u32(pq2[r], sc2[4 * half + 1]),
+                    hmul2_u32(pq2[r], sc2[4 * half + 2]), hmul2_u32(pq2[r], sc2[4 * half + 3]));
+          }
+          // the denominator sums the same f16(p/4) the value MMAs start from
+#pragma unroll
+          for (int r = 0; r < RM; ++r) l_part[r] += f16x2_to_float2(pq2[r]).x;
+          fence_proxy_async_smem();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            mbar_arrive(&sh.pready[uc & 1]);
+            mbar_arrive(&sh.empty[stage]);  // the V scales have been read
+          }
+        }
+      }
+
+      // ---- end of segment: O^T / l -> workspace, lse ----
+      if (uc > 0) {
+        wait_bar(&sh.pvdone[(uc - 1) & 1], ((uc - 1) >> 1) & 1, sh.flags, err);  // last PV
+        tc_fence_after();
+      }
+      if (smx) {
+#pragma unroll
+        for (int n = 0; n < RM; ++n) {
+          const float ls = warp_sum(l_part[n]);
+          if (lane == 0) sh.red[lq * kNP + n] = ls;
+        }
+      }
+      named_barrier(2, kSegThreads);
+      if (smx && stid < RM) {
+        float l = 0.f;
+#pragma unroll
+        for (int w = 0; w < kSmxWarps; ++w) l += sh.red[w * kNP + stid];
+        sh.alpha_s[stid] = l;
+      }
+      named_barrier(2, kSegThreads);
+      if (!smx) {
+        // Row d keeps the column of its own group; the sums carry the 2^-14
+        // of the codes and the 1/4 of the weights, and l the same 1/4:
+        // o = O * 2^14 / l, lse = m + log2(4 l).
+        const int d = 128 * hv + 32 * lq + lane;
+        const int gl = (32 * lq + lane) >> 4;  // group within the half
+#pragma unroll
+        for (int n = 0; n < RM; ++n) {
+          uint32_t o8[8];
+          tmem_ld8(tl + kColO + hv * kNPMax + n * kHalfGroups, o8);
+          tmem_wait_ld();
+          float v = 0.f;
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v = j == gl ? __uint_as_float(o8[j]) : v;
+          if (n < R) {
+            const float lv = sh.alpha_s[n];
+            ws_o[(slot * R + n) * kD + d] = lv > 0.f ? v * 16384.f / lv : 0.f;
+            if (d == 0) ws_lse[slot * R + n] = lv > 0.f ? sh.m_s[n] + 2.f + log2f(lv) : -INFINITY;
+          }
+        }
+      }
+      tc_fence_before();
+      named_barrier(2, kSegThreads);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
+}
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  if (!fn) {
+    void *p = nullptr;
+    cudaDriverEntryPointQueryResult qr;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &qr) ==
+            cudaSuccess &&
+        qr == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  }
+  return fn;
+}
+
+// The pool as a 2-D byte tensor of 128-byte rows; a box of `rows` rows
+// starting at row (page * Hkv + h) * 36 + r0 is part of one page's kv-head
+// block (head_dim 256).
+bool make_map(const nvkv_cache &c, int rows, CUtensorMapSwizzle swz, CUtensorMap *map) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t total = (cuuint64_t)c.num_pages * c.num_kv_heads * kRowsPerHead;
+  const cuuint64_t dims[2] = {128, total};
+  const cuuint64_t strides[1] = {128};
+  const cuuint32_t box[2] = {128, (cuuint32_t)rows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, c.pool, dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, swz, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace
+
+// True when this kernel takes the shape: head_dim 256 and at most 6 query
+// rows (T * Hq/Hkv) per (sequence, kv-head).
+bool decode_qk4_supported(const nvkv_cache &c, int T, int Hq) {
+  const int R = T * (Hq / c.num_kv_heads);
+  return c.head_dim == kD && R >= 1 && R <= kRowsCap && encode_fn() != nullptr;
+}
+
+cudaError_t launch_decode_qk4(const nvkv_cache &c, const nvkv_seqs &s, const void *q, int T,
+                              int Hq, float sm_scale, int S, float *ws_o, float *ws_lse,
+                              cudaStream_t stream) {
+  CUtensorMap map_k, map_aux;
+  if (!make_map(c, kKRows, CU_TENSOR_MAP_SWIZZLE_128B, &map_k) ||
+      !make_map(c, kAuxRows, CU_TENSOR_MAP_SWIZZLE_NONE, &map_aux))
+    return cudaErrorNotSupported;
+  const float qscale = sm_scale * 1.4426950408889634f;
+  const int R = T * (Hq / c.num_kv_heads);
+  auto kernel = R <= 2 ? decode_qk4_kernel<2> : R <= 4 ? decode_qk4_kernel<4>
+                                                         : decode_qk4_kernel<6>;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       kSmemBytes);
+  if (e != cudaSuccess) return e;
+  kernel<<<S, kThreads, kSmemBytes, stream>>>(
+      map_k, map_aux, c.num_pages, c.num_kv_heads, s.page_table, s.max_pages_per_seq, s.kv_lens,
+      s.batch, s.max_kv_len, static_cast<const __nv_bfloat16 *>(q), T, Hq, qscale, S, ws_o,
+      ws_lse, s.err_word);
+  return cudaGetLastError();
+}
+
+}  // namespace nvkv

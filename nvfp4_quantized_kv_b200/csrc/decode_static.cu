@@ -2,16 +2,22 @@
 // (split-K partials + combine) whose split-K scratch lives in a fixed,
 // library-owned device array instead of a caller-provided workspace.
 //
-// Who needs it: callers that cannot allocate device memory at the point
-// where they run attention -- code inside a CUDA Graph capture region (an
-// allocation there may synchronise and break the capture), runtimes whose
-// device memory is owned by another pool or allocator, and real-time paths
-// that must not take allocator locks.  They pass only inputs and outputs.
+// Who needs it: callers that cannot call cudaMalloc (or any allocator) at
+// the point where they run attention -- runtimes whose device memory belongs
+// to another pool or allocator they may not draw from, plugins hosted by an
+// application that owns all device memory, and real-time paths that must not
+// take allocator locks or risk an allocation failure.  They pass only inputs
+// and outputs.
 //
 // The scratch is one file-scope __device__ array of kStaticScratchBytes.
-// Host code cannot use the array's name as a device address, so the address
-// is looked up with cudaGetSymbolAddress once per device, on the first call
-// made with that device current, and cached.
+// Host code cannot use the array's name as a device address (it names a
+// host-side stand-in), so the address is looked up with cudaGetSymbolAddress
+// with the device current: once per device and CUDA context, on the first
+// call made in that context, and cached.  The cache is keyed by the
+// context's unique id, so a context torn down and recreated (a device reset)
+// gets a fresh lookup instead of a stale address.
+#include <cuda.h>
+
 #include <mutex>
 
 #include "nvkv_common.cuh"
@@ -23,23 +29,64 @@ constexpr int kMaxDevices = 64;
 
 __device__ __align__(256) unsigned char g_decode_scratch[kStaticScratchBytes];
 
-std::mutex g_mutex;
-void *g_scratch_addr[kMaxDevices] = {};
+typedef CUresult (*CtxGetCurrentFn)(CUcontext *);
+typedef CUresult (*CtxGetIdFn)(CUcontext, unsigned long long *);
 
-// Device address of the scratch array on the current device, or NULL.
+struct ScratchSlot {
+  void *addr = nullptr;
+  unsigned long long ctx_id = 0;
+  bool keyed = false;  // ctx_id is valid
+};
+
+std::mutex g_mutex;
+ScratchSlot g_slot[kMaxDevices];
+
+template <class Fn>
+Fn driver_fn(const char *name) {
+  void *p = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint(name, &p, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  return reinterpret_cast<Fn>(p);
+}
+
+// Unique id of the current CUDA context (false when there is none yet or the
+// driver cannot tell).
+bool current_ctx_id(unsigned long long *id) {
+  static const CtxGetCurrentFn get_current = driver_fn<CtxGetCurrentFn>("cuCtxGetCurrent");
+  static const CtxGetIdFn get_id = driver_fn<CtxGetIdFn>("cuCtxGetId");
+  if (!get_current || !get_id) return false;
+  CUcontext ctx = nullptr;
+  if (get_current(&ctx) != CUDA_SUCCESS || !ctx) return false;
+  return get_id(ctx, id) == CUDA_SUCCESS;
+}
+
+// Device address of the scratch array in the current device's context, or
+// NULL when the lookup fails.
 void *scratch_on_current_device() {
   int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  std::lock_guard<std::mutex> lock(g_mutex);
-  if (!g_scratch_addr[dev]) {
-    void *p = nullptr;
-    if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) {
-      cudaGetLastError();  // leave no error behind for the caller's next call
-      return nullptr;
-    }
-    g_scratch_addr[dev] = p;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return nullptr;
   }
-  return g_scratch_addr[dev];
+  unsigned long long id = 0;
+  const bool have_id = current_ctx_id(&id);
+  std::lock_guard<std::mutex> lock(g_mutex);
+  ScratchSlot &s = g_slot[dev];
+  if (s.addr && s.keyed && have_id && s.ctx_id == id) return s.addr;
+  void *p = nullptr;
+  if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess || !p) {
+    cudaGetLastError();  // leave no error behind for the caller's next call
+    s = ScratchSlot();
+    return nullptr;
+  }
+  // The lookup made the device's context current if it was not yet.
+  s.addr = p;
+  s.keyed = current_ctx_id(&s.ctx_id);
+  return p;
 }
 
 }  // namespace
@@ -53,6 +100,9 @@ nvkv_status nvkv_decode_attn_static(const nvkv_cache *cache, const nvkv_seqs *se
                                     float sm_scale, int32_t num_splits, void *out,
                                     nvkv_stream_t stream) {
   if (!cache || !seqs) return NVKV_ERR_INVALID_ARG;
+  // out is only written by the merge, after the partials kernel: reject a bad
+  // one before anything is launched.
+  if (!out || (reinterpret_cast<uintptr_t>(out) & 15u)) return NVKV_ERR_INVALID_ARG;
   const size_t need = nvkv_decode_workspace_bytes(seqs->batch, T, num_q_heads,
                                                   cache->num_kv_heads, cache->head_dim,
                                                   num_splits);

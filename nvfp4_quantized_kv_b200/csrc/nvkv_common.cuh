@@ -143,6 +143,16 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
   return out;
 }
 
+// Two floats -> one byte of E2M1 codes (a in the low nibble), rounded to
+// nearest with ties to even and saturated at 6 by the hardware conversion.
+__device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float a, float b) {
+  uint32_t out;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %2, %1;\n\tcvt.u32.u8 %0, t;\n\t}"
+      : "=r"(out)
+      : "f"(a), "f"(b));
+  return out;
+}
+
 // Four E2M1 code pairs (one 32-bit word, byte k = elements 2k, 2k+1) ->
 // four f16x2.  The bytes are split by register unpacking, not converted.
 __device__ __forceinline__ void e2m1x8_to_f16x2x4(uint32_t w, uint32_t (&o)[4]) {
@@ -189,6 +199,29 @@ __device__ __forceinline__ uint32_t ex2_f16x2(float a, float b) {
   asm("cvt.rn.f16x2.f32 %0, %2, %1;" : "=r"(h) : "f"(a), "f"(b));
   asm("ex2.approx.f16x2 %0, %1;" : "=r"(r) : "r"(h));
   return r;
+}
+
+// (2^a, 2^b) as an f16 pair (a in the low half): each exponential in fp32
+// (ex2.approx, relative error about 2^-22), then one rounding to f16.
+// 2^-inf = +0.
+__device__ __forceinline__ uint32_t ex2_f32_to_f16x2(float a, float b) {
+  float ea, eb;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(ea) : "f"(a));
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(eb) : "f"(b));
+  uint32_t h;
+  asm("cvt.rn.f16x2.f32 %0, %2, %1;" : "=r"(h) : "f"(ea), "f"(eb));
+  return h;
+}
+
+// (q, q) as an f16 pair with q = 2^a / 4: the exponential in fp32
+// (ex2.approx, relative error about 2^-22), one rounding to f16.  2^-inf = +0.
+__device__ __forceinline__ uint32_t ex2_quarter_f16x2(float a) {
+  float e;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(a));
+  e *= 0.25f;
+  uint32_t h;
+  asm("cvt.rn.f16x2.f32 %0, %1, %1;" : "=r"(h) : "f"(e));
+  return h;
 }
 
 // Warp reductions.

@@ -78,6 +78,8 @@ def lib():
             L.oracle_dequant.argtypes = [i32, i32]
             L.oracle_qdq_row.restype = None
             L.oracle_qdq_row.argtypes = [vp, i32, vp]
+            L.oracle_qdq_rows.restype = None
+            L.oracle_qdq_rows.argtypes = [vp, ctypes.c_long, i32, vp]
             L.oracle_page_bytes.restype = ctypes.c_size_t
             L.oracle_page_bytes.argtypes = [i32, i32]
             L.oracle_append.restype = None
@@ -182,10 +184,53 @@ def qdq_rows(x_bits) -> np.ndarray:
     D = x.shape[-1]
     flat = np.ascontiguousarray(x.reshape(-1, D))
     out = np.zeros(flat.shape, np.float64)
+    n = flat.shape[0]
     L = lib()
-    for i in range(flat.shape[0]):
-        L.oracle_qdq_row(flat[i].ctypes.data, D, out[i].ctypes.data)
+
+    def run(lo, hi):  # ctypes releases the GIL: blocks of rows run in parallel
+        L.oracle_qdq_rows(flat[lo:hi].ctypes.data, ctypes.c_long(hi - lo), D, out[lo:hi].ctypes.data)
+
+    nthreads = min(os.cpu_count() or 1, max(1, n // 4096))
+    if nthreads <= 1:
+        run(0, n)
+    else:
+        bounds = [n * i // nthreads for i in range(nthreads + 1)]
+        ts = [threading.Thread(target=run, args=(bounds[i], bounds[i + 1]))
+              for i in range(nthreads)]
+        for t in ts:
+            t.start()
+        for t in ts:
+            t.join()
     return out.reshape(x.shape)
+
+
+def attention_dense(k_hat: np.ndarray, v_hat: np.ndarray, q_bits, n_visible, sm_scale: float):
+    """Exact softmax attention of several query rows of one kv-head over
+    already dequantised keys and values (float64 [n][D], e.g. from
+    qdq_rows), straight from the definition with numpy's float64 matrix
+    product as the dot-product step: row i sees keys 0 .. n_visible[i]-1,
+    s = sm_scale * q.k, p = exp(s - max s) / sum, out = sum p v.  Used where
+    many rows share one long cache (the per-row oracle re-quantises every key
+    for every row).  Returns (out [m][D], lse [m] natural log)."""
+    qb = _u16(q_bits).reshape(-1, k_hat.shape[1])
+    q = (qb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)  # bf16 -> f64, exact
+    nvis = np.asarray(n_visible, np.int64).reshape(-1)
+    m = q.shape[0]
+    out = np.zeros((m, k_hat.shape[1]), np.float64)
+    lse = np.full(m, -np.inf)
+    n = int(nvis.max()) if m else 0
+    if n <= 0:
+        return out, lse
+    s = (q @ k_hat[:n].T) * float(sm_scale)          # [m][n]
+    s[np.arange(n)[None, :] >= nvis[:, None]] = -np.inf
+    top = s.max(axis=1)
+    ok = np.isfinite(top)
+    p = np.zeros_like(s)
+    p[ok] = np.exp(s[ok] - top[ok, None])
+    denom = p.sum(axis=1)
+    out[ok] = (p[ok] @ v_hat[:n]) / denom[ok, None]
+    lse[ok] = top[ok] + np.log(denom[ok])
+    return out, lse
 
 
 # --------------------------------------------------------------------------

@@ -192,6 +192,11 @@ void oracle_qdq_row(const uint16_t *x, int D, double *out) {
     }
 }
 
+/* oracle_qdq_row over n consecutive rows of D elements. */
+void oracle_qdq_rows(const uint16_t *x, long n, int D, double *out) {
+    for (long r = 0; r < n; ++r) oracle_qdq_row(x + (size_t)r * D, D, out + (size_t)r * D);
+}
+
 /* ------------------------------------------------------------------------ */
 /* Page layout                                                               */
 /* ------------------------------------------------------------------------ */

@@ -34,6 +34,38 @@ def oracle_outputs(wl: Workload, rows, nthreads=None, k8=False):
     return out
 
 
+def oracle_outputs_dense(wl: Workload, rows):
+    """As oracle_outputs, for many rows over long caches: the keys and values
+    of each (sequence, kv-head) are quantised and dequantised once by the
+    oracle (qdq_rows) and the rows are computed by oracle.attention_dense
+    (pinned against the per-row oracle in test_oracle_dense_pins.py)."""
+    q = wl.queries()
+    G = wl.group
+    out = np.zeros((len(rows), wl.head_dim), np.float64)
+    by = {}
+    for i, (b, t, hq) in enumerate(rows):
+        by.setdefault((b, hq // G), []).append((i, t, hq))
+    for b in sorted({b for b, _ in by}):
+        k, v = wl.kv_rows(b, 0, int(wl.kv_lens[b]))
+        for h in sorted(h for bb, h in by if bb == b):
+            items = by[(b, h)]
+            k_hat = oracle.qdq_rows(np.ascontiguousarray(k[:, h]))
+            v_hat = oracle.qdq_rows(np.ascontiguousarray(v[:, h]))
+            qs = np.stack([q[b * wl.T + t, hq] for _, t, hq in items])
+            nvis = [wl.query_position(b, t) + 1 for _, t, _ in items]
+            o, _ = oracle.attention_dense(k_hat, v_hat, qs, nvis, wl.sm_scale)
+            for (i, _, _), row in zip(items, o):
+                out[i] = row
+            del k_hat, v_hat
+    return out
+
+
+def prefill_sample_queries(n: int):
+    """The deterministic sample of a prefill chunk's queries: the first 64,
+    the last 64 and every 31st."""
+    return sorted(set(range(min(64, n))) | set(range(max(0, n - 64), n)) | set(range(0, n, 31)))
+
+
 def gpu_rows(out: torch.Tensor, wl: Workload, rows) -> np.ndarray:
     o = out.float().cpu().numpy()
     return np.stack([o[b * wl.T + t, hq] for b, t, hq in rows]).astype(np.float64)

@@ -12,7 +12,8 @@ import nvfp4_quantized_kv_b200 as nv
 from nvfp4_quantized_kv_b200 import workload as W
 from nvfp4_quantized_kv_b200.harness import DeviceWorkload
 
-from parity_util import all_rows, assert_close, gpu_rows, oracle_outputs, sample_rows
+from parity_util import (all_rows, assert_close, gpu_rows, oracle_outputs, oracle_outputs_dense,
+                         sample_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -75,10 +76,30 @@ def test_ragged_batch_config():
 
 @pytest.mark.parametrize("T", [1, 6])
 def test_long_context_config_sampled(T):
+    """3 x {330k, 420k, 470k}: every head of the last query of each
+    sequence, and for T=6 every head of the first query too."""
     wl = W.long_context(T=T)
     dw = run_step(wl)
-    rows = [(0, T - 1, 0), (1, 0, 13), (2, T - 1, 23), (2, 0, 6)]
-    assert_close(gpu_rows(dw.out, wl, rows), oracle_outputs(wl, rows), wl.name)
+    ts = sorted({0, T - 1})
+    rows = [(b, t, hq) for b in range(wl.batch) for t in ts for hq in range(wl.num_q_heads)]
+    assert_close(gpu_rows(dw.out, wl, rows), oracle_outputs_dense(wl, rows), wl.name)
+
+
+@pytest.mark.parametrize("T", [1, 6])
+@pytest.mark.parametrize("num_splits", [0, 12, 1502])
+def test_rows_ending_on_page_unit_and_split_boundaries(T, num_splits):
+    """Visible ranges that end exactly on a page, a 128-token unit and a
+    split boundary.  Every pair has 500 or 501 units; 12 splits put
+    boundaries at pair ends, 1502 (= units of all pairs / 4) at every fourth
+    unit, so the last row of sequence 0 ends where a split ends and rows of
+    sequences 1 and 2 end on the unit boundary at 64000 keys.  All rows."""
+    ctx = {1: [63999, 64002, 64000], 6: [63994, 63997, 63995]}[T]
+    wl = W.small(f"bounds_T{T}", 3, 24, 4, 256, T, ctx, seed=41)
+    dw = run_step(wl, num_splits)
+    ends = {(b, t): wl.query_position(b, t) + 1 for b in range(3) for t in range(T)}
+    assert 64000 in ends.values()
+    rows = all_rows(wl)
+    assert_close(gpu_rows(dw.out, wl, rows), oracle_outputs_dense(wl, rows), wl.name)
 
 
 def test_split_count_does_not_change_the_result():

@@ -12,7 +12,8 @@ import torch
 from nvfp4_quantized_kv_b200 import workload as W
 from nvfp4_quantized_kv_b200.harness import DeviceWorkload
 
-from parity_util import ATOL, RTOL, all_rows, assert_close, gpu_rows, oracle_outputs, sample_rows
+from parity_util import (ATOL, RTOL, all_rows, assert_close, gpu_rows, oracle_outputs,
+                         oracle_outputs_dense, prefill_sample_queries, sample_rows)
 
 pytestmark = pytest.mark.gpu
 
@@ -63,12 +64,12 @@ def test_prefill_kernels_agree(case, monkeypatch):
 
 
 def test_chunked_prefill_config_sampled():
-    """65536 cached tokens + a 2048-token chunk, 24/4 heads, head_dim 256."""
+    """65536 cached tokens + a 2048-token chunk, 24/4 heads, head_dim 256:
+    the first 64, the last 64 and every 31st chunk query, all heads."""
     wl = W.chunked_prefill()
     dw = run(wl)
-    rows = [(0, 0, 0), (0, 0, 23), (0, 2047, 0), (0, 2047, 17), (0, 1024, 5), (0, 21, 6),
-            (0, 22, 11), (0, 1500, 12)]
-    assert_close(gpu_rows(dw.out, wl, rows), oracle_outputs(wl, rows), wl.name)
+    rows = [(0, t, hq) for t in prefill_sample_queries(wl.T) for hq in range(wl.num_q_heads)]
+    assert_close(gpu_rows(dw.out, wl, rows), oracle_outputs_dense(wl, rows), wl.name)
 
 
 def test_prefill_tail_matches_decode_verify():
