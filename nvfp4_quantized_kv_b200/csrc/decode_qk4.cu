@@ -32,40 +32,39 @@
 //
 // V's groups run along head_dim, not along the tokens the value sum
 // contracts, so the value sum is an f16 MMA (swap-AB: V^T is the M = 128
-// side).  Its scales move to the other operand: with g(d) the group of
-// head_dim row d,
-//     o[r][d] = sum_j p[r][j] * vscale[j][g(d)] * code[j][d],
-// so the N side holds P'[(r, g)][j] = p[r][j] * vscale[j][g] for every row r
-// and every group g of the 128-row half (N = 8 * rows: 48 at 6 rows, which
-// costs the MMA no more than 16), and each O^T row d keeps the column of its
-// own group.  V^T itself is then the bare codes, built with integer
-// operations: the f16 bit pattern (mag << 9) | (sign << 15) is exactly
-// E2M1(code) * 2^-14 (the E2M1 subnormal 0.5 included), so a 32-bit word of
-// 8 codes becomes four f16 pairs with a shift, two masks and a multiply-add
-// each -- no conversion instructions, which run at a fraction of the rate.
-// The pair of a word holds tokens (t, t+4), so P' uses the same permutation
-// of the tokens along K.  P' = f16(f16(p/4) * vscale) stays below the f16
-// maximum (p <= 2^8 with the lazy maximum, vscale <= 448), and the
-// epilogue applies 2^16 / (4 * denominator).  P comes from an fp32 exp2.
+// side, the query rows the N = 16 side).  V^T goes into Tensor Memory as
+// exact f16 values: E2M1 * E4M3 has at most 6 significant bits and lies in
+// [2^-10, 2688], so v * 2^-14 is an f16 number (subnormal at the bottom)
+// and needs no rounding.  A 32-bit word of 8 codes becomes four f16 pairs
+// with integer operations: the bit pattern (mag << 9) | (sign << 15) is
+// exactly E2M1(code) * 2^-14 (the E2M1 subnormal 0.5 included), built with a
+// shift, two masks and a multiply-add -- no conversion instructions, which
+// run at a fraction of the rate -- and one f16 multiply by the pair's scales
+// applies the scales.  A warp covers 32 head_dim rows, i.e. two scale
+// groups, so it converts the 2 x 128 scale bytes of a unit once (4
+// conversions a lane) into a table in shared memory that its lanes read.
+// The pair of a word holds tokens (t, t+4), so P uses the same permutation
+// of the tokens along K.  P = f16(2^(score - running max)) from an fp32
+// exp2, at most 2^8 with the lazy maximum, and the epilogue applies
+// 2^14 / denominator, the denominator summing the same f16 weights.
 //
 // Per 128-token unit the tensor pipe runs 4 NVFP4 MMAs (scores) and 16 f16
-// MMAs (values), against 16 + 16 f16 MMAs when K is dequantised, and the
-// CUDA cores convert no code.
+// MMAs (values), against 16 + 16 f16 MMAs when K is dequantised.
 //
-// Roles (one persistent CTA per split-plan range, 448 threads):
+// Roles (one persistent CTA per split-plan range, 480 threads):
 //  * warp 12 (TMA): per page two tiled loads, no multicast: the 16 rows of K
 //    codes (128-byte swizzle, into the unit's contiguous K tile) and the 20
 //    rows of K scales, V codes and V scales (no swizzle); 4-stage ring.
-//  * warps 0..3 copy the unit's K scale bytes into the Tensor Memory
-//    scale-factor layout (every lane quarter holds the same 32 rows);
-//    warps 0..7 write the V^T codes into Tensor Memory (one head_dim row a
+//  * warps 0..3 copy the K scale bytes of the next unit into the Tensor
+//    Memory scale-factor layout (every lane quarter holds the same 32 rows);
+//    warps 0..7 write the scaled V^T into Tensor Memory (one head_dim row a
 //    lane).
 //  * warps 8..11 (softmax, one token a lane): recombine the terms, mask,
 //    running max raised lazily (only when a score exceeds it by more than
-//    2^8, detected by a vote), fp32 exp2, P' to shared memory, the
-//    denominator from the same f16 weights; at a segment start they build
-//    the query terms.
-//  * warp 13: one thread issues all MMAs.
+//    2^8, detected by a vote), fp32 exp2, P to a 4-slot ring in shared
+//    memory, the denominator from the same f16 weights; at a segment start
+//    they build the query terms.
+//  * warp 13 issues the score MMAs, warp 14 the value MMAs (one thread each).
 //  * Every wait is bounded; a timeout sets NVKV_DEVERR_TIMEOUT, turns later
 //    waits into no-ops and lets the kernel drain and free its Tensor Memory.
 #include <cfloat>
@@ -94,9 +93,8 @@ constexpr int kStages = 4;
 constexpr int kRowsCap = 6;              // query rows per pair (T * G) this kernel takes
 constexpr int kTerms = 8;                // NVFP4 terms per query row
 constexpr int kNSMax = kRowsCap * kTerms;   // 48: largest N of the score MMA
-constexpr int kHalfGroups = 8;           // scale groups in a 128-row half of head_dim
-constexpr int kNPMax = kRowsCap * kHalfGroups;  // 48: largest N of the value MMA
-constexpr int kNP = 16;                  // rows of the per-row scratch arrays
+constexpr int kNP = 16;                  // N of the value MMA: the query rows, padded
+constexpr int kPSlots = 4;               // P ring depth
 
 constexpr int kDeqWarps = 8;             // warps 0..7
 constexpr int kSmxWarp0 = 8;             // warps 8..11
@@ -111,48 +109,55 @@ constexpr long long kWaitBudget = 2000000000LL;  // clock cycles (~1 s)
 constexpr float kLazyRescale = 8.0f;             // log2 units
 
 // Tensor Memory columns.
-constexpr uint32_t kColV = 0;      // 2 slots x 128: V^T codes (d-half h at +64h), f16 token pairs
+constexpr uint32_t kColV = 0;      // 2 slots x 128: V^T (d-half h at +64h), f16 token pairs
 constexpr uint32_t kColS = 256;    // 2 slots x kNSMax: S^T, fp32, one token per lane
-constexpr uint32_t kColO = 352;    // 2 halves x kNPMax: O^T per (row, group), fp32
-constexpr uint32_t kColSFA = 448;  // 2 slots x 16: K scale factors, column 4*ks + m1
-constexpr uint32_t kColSFB = 480;  // 4 x 4: query-term scale factors, column 4*ks + n1 (n1 < 2)
-static_assert(kColS + 2 * kNSMax <= kColO && kColO + 2 * kNPMax <= kColSFA &&
-                  kColSFB + 16 <= kTmemCols, "tensor memory");
+constexpr uint32_t kColO = 352;    // 2 halves x kNP: O^T, fp32, column = query row
+constexpr uint32_t kColSFA = 384;  // 2 slots x 16: K scale factors, column 4*ks + m1
+constexpr uint32_t kColSFB = 416;  // 4 x 4: query-term scale factors, column 4*ks + n1 (n1 < 2)
+static_assert(kColS + 2 * kNSMax <= kColO && kColO + 2 * kNP <= kColSFA &&
+                  kColSFB + 16 <= kTmemCols && kColSFA % 4 == 0 && kColSFB % 4 == 0,
+              "tensor memory");
 
 // Shared memory (offsets from a 1024-byte aligned base).
 constexpr int kOffQ = kStages * kStageBytes;        // query terms, kNSMax rows x 128 B, swizzled
-constexpr int kOffP = kOffQ + kNSMax * 128;         // P' tiles [slot][half], MN-major f16
-constexpr int kPHalfBytes = kRowsCap * 2048;        // (row r, group g) x 128 tokens
-constexpr int kPSlotBytes = 2 * kPHalfBytes;
-constexpr int kOffSfb = kOffP + 2 * kPSlotBytes;    // [kNSMax][16] scale bytes of the terms
+constexpr int kOffP = kOffQ + kNSMax * 128;         // P tiles [slot], MN-major f16
+constexpr int kPSlotBytes = 2 * 2048;               // rows 0..7, rows 8..15 (zero) x 128 tokens
+constexpr int kOffVsc = kOffP + kPSlots * kPSlotBytes;  // V scale pairs [warp][page][group][8]
+constexpr int kVscWarpBytes = kUnitPages * 2 * 8 * 4;   // 512
+constexpr int kOffSfb = kOffVsc + kDeqWarps * kVscWarpBytes;  // [kNSMax][16] term scale bytes
 constexpr int kOffFac = kOffSfb + kNSMax * 16;      // float [kRowsCap]: 2^-k of each row's terms
-constexpr int kOffRed = kOffFac + kNSMax * 4;       // float [4][kNP]
-constexpr int kOffMask = kOffRed + kSmxWarps * kNP * 4;  // u32 [2][4][4]
-constexpr int kOffM = kOffMask + 2 * kSmxWarps * 4 * 4;  // float [kNP]
+constexpr int kOffRed = kOffFac + kNSMax * 4;       // float [quarter][kNP]
+constexpr int kOffMask = kOffRed + 4 * kNP * 4;     // u32 [parity][quarter]
+constexpr int kOffM = kOffMask + 2 * 4 * 4;         // float [kNP]
 constexpr int kOffAlpha = kOffM + kNP * 4;
 constexpr int kOffNvis = kOffAlpha + kNP * 4;
-constexpr int kOffFlags = kOffNvis + kNP * 4;        // int[4]: abort at [2]
-constexpr int kOffPages = kOffFlags + 16;            // int[stages][8]
+constexpr int kOffFlags = kOffNvis + kNP * 4;       // int[4]: abort at [2]
+constexpr int kOffPages = kOffFlags + 16;           // int[stages][8]
 constexpr int kOffBars = kOffPages + kStages * kUnitPages * 4;
-constexpr int kNumBars = 2 * kStages + 13;
+constexpr int kNumBars = 2 * kStages + 2 * 4 + 3 * kPSlots + 3;
 constexpr int kOffTmem = kOffBars + kNumBars * 8;
 constexpr int kSmemBytes = kOffTmem + 16 + 1024;    // + alignment slack
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
-static_assert(kOffQ % 1024 == 0 && kStageBytes % 1024 == 0 && kOffP % 16 == 0 &&
-                  kOffSfb % 16 == 0 && kOffPages % 16 == 0 && kOffBars % 8 == 0,
+static_assert(kOffQ % 1024 == 0 && kStageBytes % 1024 == 0 && kOffP % 128 == 0 &&
+                  kOffVsc % 16 == 0 && kOffSfb % 16 == 0 && kOffPages % 16 == 0 &&
+                  kOffBars % 8 == 0,
               "alignment");
 
 struct Shared {
   uint8_t *stages, *qtile, *ptile, *sfb;
+  uint32_t *vsc;
   float *fac, *red, *m_s, *alpha_s;
   int32_t *nvis_s, *pages;
   uint32_t *masks;
   volatile int *flags;
-  // Barriers of the per-slot resources exist once per slot: slot s completes
-  // once per unit with (unit & 1) == s, so a parity wait is never more than
-  // one phase behind.
-  uint64_t *full, *empty, *sfa_ready, *sready, *pready, *vready, *pvdone, *qready, *final_bar,
-      *final_pv;
+  // A barrier of a ring slot completes once per unit that uses the slot, so
+  // a parity wait is never more than one phase behind.
+  uint64_t *full, *empty;        // [kStages]
+  uint64_t *sfa_ready, *sready;  // [2]: scale factors of K written; S^T written
+  uint64_t *sfree;               // [2]: S^T read by the softmax
+  uint64_t *vready, *pvdone;     // [slot][half]: V^T written; value MMAs done
+  uint64_t *pready, *pfree;      // [kPSlots]: P written; P read by the value MMAs
+  uint64_t *qready, *final_bar, *final_pv;
   uint32_t *tmem_slot;
 };
 
@@ -218,6 +223,14 @@ __device__ __forceinline__ uint32_t code_pair(uint32_t w) {
   return (a & 0x10001000u) * 8u + (a & 0x0E000E00u);
 }
 
+// f16 pair product, round to nearest, subnormals kept (the V^T values at the
+// bottom of the range are f16 subnormals, and exact).
+__device__ __forceinline__ uint32_t mul_f16x2(uint32_t a, uint32_t b) {
+  uint32_t d;
+  asm("mul.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+  return d;
+}
+
 template <int RM>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
@@ -229,8 +242,7 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
   // RM: query rows per pair rounded up to an even count (padding rows are
   // zero); the score MMA has N = RM * kTerms columns.
   static_assert(RM % 2 == 0 && RM >= 2 && RM <= kRowsCap, "rows");
-  constexpr int NS = RM * kTerms;        // score MMA: (row, term) columns
-  constexpr int NP = RM * kHalfGroups;   // value MMA: (row, group of the half) columns
+  constexpr int NS = RM * kTerms;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -238,6 +250,7 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
   sh.stages = smem;
   sh.qtile = smem + kOffQ;
   sh.ptile = smem + kOffP;
+  sh.vsc = reinterpret_cast<uint32_t *>(smem + kOffVsc);
   sh.sfb = smem + kOffSfb;
   sh.fac = reinterpret_cast<float *>(smem + kOffFac);
   sh.red = reinterpret_cast<float *>(smem + kOffRed);
@@ -250,14 +263,16 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBars);
   sh.full = bars;
   sh.empty = bars + kStages;
-  sh.sfa_ready = bars + 2 * kStages;  // [2]
-  sh.sready = sh.sfa_ready + 2;       // [2]
-  sh.pready = sh.sfa_ready + 4;       // [2]
-  sh.vready = sh.sfa_ready + 6;       // [2]
-  sh.pvdone = sh.sfa_ready + 8;       // [2]
-  sh.qready = sh.sfa_ready + 10;
-  sh.final_bar = sh.sfa_ready + 11;
-  sh.final_pv = sh.sfa_ready + 12;
+  sh.sfa_ready = bars + 2 * kStages;
+  sh.sready = sh.sfa_ready + 2;
+  sh.sfree = sh.sfa_ready + 4;
+  sh.vready = sh.sfa_ready + 6;   // [slot][half]
+  sh.pvdone = sh.sfa_ready + 10;  // [slot][half]
+  sh.pready = sh.sfa_ready + 14;
+  sh.pfree = sh.pready + kPSlots;
+  sh.qready = sh.pfree + kPSlots;
+  sh.final_bar = sh.qready + 1;
+  sh.final_pv = sh.qready + 2;
   sh.tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffTmem);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -267,15 +282,20 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&sh.full[i], 1);
-      // the score MMAs' commit, the V-code readers and the V-scale readers
-      mbar_init(&sh.empty[i], 1 + kDeqWarps + kSmxWarps);
+      mbar_init(&sh.empty[i], 1 + kDeqWarps);  // the score MMAs' commit, the V^T writers
     }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&sh.sfa_ready[i], 4);
       mbar_init(&sh.sready[i], 1);
+      mbar_init(&sh.sfree[i], kSmxWarps);
+      for (int h = 0; h < 2; ++h) {
+        mbar_init(&sh.vready[2 * i + h], kDeqWarps / 2);
+        mbar_init(&sh.pvdone[2 * i + h], 1);
+      }
+    }
+    for (int i = 0; i < kPSlots; ++i) {
       mbar_init(&sh.pready[i], kSmxWarps);
-      mbar_init(&sh.vready[i], kDeqWarps);
-      mbar_init(&sh.pvdone[i], 1);
+      mbar_init(&sh.pfree[i], 1);
     }
     mbar_init(sh.qready, kSmxWarps);
     mbar_init(sh.final_bar, 1);
@@ -283,6 +303,9 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
     fence_mbar_init();
   }
   if (threadIdx.x < 4) sh.flags[threadIdx.x] = 0;
+  // The P tiles start as zeros: rows R..15 are never written.
+  for (int i = threadIdx.x; i < kPSlots * kPSlotBytes / 16; i += kThreads)
+    reinterpret_cast<uint4 *>(sh.ptile)[i] = make_uint4(0u, 0u, 0u, 0u);
   if (warp == kMmaWarp) {
     tmem_alloc(sh.tmem_slot, kTmemCols);
     tmem_relinquish();
@@ -298,6 +321,7 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
   const int c = blockIdx.x;
   const int64_t u0 = U > 0 ? range_begin(c, U, S) : 0;
   const int64_t u1 = U > 0 ? range_begin(c + 1, U, S) : 0;
+  const uint32_t n_units = (uint32_t)(u1 - u0);
 
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ TMA
@@ -359,10 +383,9 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
     // the tensor pipe idle while it waits for the next step's inputs.  One
     // thread issues the scores of each unit as soon as its tiles, scale
     // factors, query terms and S^T slot are ready; the other issues the
-    // value MMAs of each unit once its V^T codes and P' are ready.  Each
-    // commits its own MMAs; the tensor pipe runs both streams.
+    // value MMAs of each unit once its V^T and P are ready.  Each commits
+    // its own MMAs; the tensor pipe runs both streams.
     if (lane == 0) {
-      const uint32_t n_units = (uint32_t)(u1 - u0);
       int64_t seg_end = segment_at(u0, u1, kv_lens, B, Hkv, max_kv_len, max_pages).seg_end;
       bool issued = false;
       if (warp == kMmaWarp) {
@@ -382,7 +405,7 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
           wait_bar(&sh.full[stage], (qk / kStages) & 1, sh.flags, err);
           wait_bar(&sh.sfa_ready[qk & 1], (qk >> 1) & 1, sh.flags, err);
           // S^T slot qk&1 was read by the softmax of unit qk-2
-          if (qk > 1) wait_bar(&sh.pready[qk & 1], ((qk >> 1) + 1) & 1, sh.flags, err);
+          if (qk > 1) wait_bar(&sh.sfree[qk & 1], ((qk >> 1) + 1) & 1, sh.flags, err);
           tc_fence_after();
           const uint32_t sslot = tmem + kColS + (qk & 1) * kNSMax;
           const uint32_t sfa = tmem + kColSFA + (qk & 1) * 16;
@@ -400,28 +423,30 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
           mbar_wait(sh.final_bar, 0, kWaitBudget);
         }
       } else {
-        const uint32_t idesc_pv = idesc_f16_f32(128, NP, false, true);
+        const uint32_t idesc_pv = idesc_f16_f32(128, kNP, false, true);
         const uint32_t pb = smem_u32(sh.ptile);
         for (uint32_t pv = 0; pv < n_units && !sh.flags[2]; ++pv) {
           const int64_t uu = u0 + pv;
           const bool first = pv == 0 || uu >= seg_end;  // O^T starts from zero
           if (uu >= seg_end)
             seg_end = segment_at(uu, u1, kv_lens, B, Hkv, max_kv_len, max_pages).seg_end;
-          wait_bar(&sh.vready[pv & 1], (pv >> 1) & 1, sh.flags, err);
-          wait_bar(&sh.pready[pv & 1], (pv >> 1) & 1, sh.flags, err);
-          tc_fence_after();
-          const uint32_t pslot = pb + (pv & 1) * kPSlotBytes;
+          const int ps = pv % kPSlots;
+          wait_bar(&sh.pready[ps], (pv / kPSlots) & 1, sh.flags, err);
+          const uint32_t pslot = pb + ps * kPSlotBytes;
           const uint32_t vslot = tmem + kColV + (pv & 1) * 128;
+          // One head_dim half at a time: each half's V^T rows are released
+          // as soon as its MMAs complete.
 #pragma unroll
-          for (int ks = 0; ks < 8; ++ks) {
-            const uint32_t acc = (!first) || ks > 0;
+          for (int hf = 0; hf < 2; ++hf) {
+            wait_bar(&sh.vready[(pv & 1) * 2 + hf], (pv >> 1) & 1, sh.flags, err);
+            tc_fence_after();
 #pragma unroll
-            for (int hf = 0; hf < 2; ++hf)
-              mma_f16_ts(tmem + kColO + hf * kNPMax, vslot + 64 * hf + ks * 8,
-                         smem_desc(pslot + hf * kPHalfBytes + ks * 256, 128, 2048), idesc_pv,
-                         acc);
+            for (int ks = 0; ks < 8; ++ks)
+              mma_f16_ts(tmem + kColO + hf * kNP, vslot + 64 * hf + ks * 8,
+                         smem_desc(pslot + ks * 256, 128, 2048), idesc_pv, (!first) || ks > 0);
+            mma_commit(&sh.pvdone[(pv & 1) * 2 + hf]);
           }
-          mma_commit(&sh.pvdone[pv & 1]);
+          mma_commit(&sh.pfree[ps]);
           issued = true;
         }
         if (issued) {
@@ -433,13 +458,44 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
   } else {
     // -------------------------------------------------------------- workers
     const bool smx = warp >= kSmxWarp0;
-    const int lq = warp & 3;                   // lane quarter of Tensor Memory
-    const int hv = smx ? 0 : ((warp >> 2) & 1);  // V^T half of a code-writing warp
+    const int lq = warp & 3;                     // lane quarter of Tensor Memory
+    const int hv = smx ? 0 : ((warp >> 2) & 1);  // V^T half of a V^T-writing warp
     const uint32_t tl = tmem + ((uint32_t)(32 * lq) << 16);
     const int stid = threadIdx.x - kSmxWarp0 * 32;  // softmax thread 0..127
-    float l_part[RM], facr[RM];
+    float l_part[RM], facr[RM], mr[RM];
 #pragma unroll
-    for (int i = 0; i < RM; ++i) l_part[i] = facr[i] = 0.f;
+    for (int i = 0; i < RM; ++i) l_part[i] = facr[i] = 0.f, mr[i] = -FLT_MAX;
+
+    // K scale factors of unit un (its stage) into slot un&1, which the
+    // score MMAs of unit un-2 read before (warps 0..3: every lane quarter
+    // holds the same rows).  Column 4*ks + m1, lane l: the 4 scale bytes of
+    // token 32*m1 + l for head_dim elements 64*ks .. 64*ks+63.
+    auto write_sfa = [&](uint32_t un) {
+      const int st = un % kStages;
+      const uint8_t *ax = sh.stages + st * kStageBytes + kKTileBytes;
+      wait_bar(&sh.full[st], (un / kStages) & 1, sh.flags, err);
+      if (un > 1) {
+        wait_bar(&sh.sready[un & 1], ((un >> 1) + 1) & 1, sh.flags, err);
+        tc_fence_after();
+      }
+      uint32_t w[16];
+#pragma unroll
+      for (int m1 = 0; m1 < 4; ++m1) {
+        const int j = 32 * m1 + lane;  // token of the unit
+        const uint4 v = *reinterpret_cast<const uint4 *>(ax + (j >> 4) * kAuxPageBytes + kAuxKs +
+                                                         (j & 15) * 16);
+        w[0 * 4 + m1] = v.x;
+        w[1 * 4 + m1] = v.y;
+        w[2 * 4 + m1] = v.z;
+        w[3 * 4 + m1] = v.w;
+      }
+      tmem_st16(tl + kColSFA + (un & 1) * 16, w);
+      tmem_wait_st();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&sh.sfa_ready[un & 1]);
+    };
+    if (!smx && warp < 4 && n_units > 0) write_sfa(0);
 
     uint32_t uc = 0;
     uint32_t seg_idx = 0;
@@ -454,10 +510,10 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
         // have completed: its last softmax waited for them) ----
         if (stid < kNP) {
           sh.nvis_s[stid] = stid < R ? sg.kv_len - T + stid / G + 1 : 0;
-          sh.m_s[stid] = -INFINITY;
+          sh.m_s[stid] = -FLT_MAX;
         }
 #pragma unroll
-        for (int i = 0; i < RM; ++i) l_part[i] = 0.f;
+        for (int i = 0; i < RM; ++i) l_part[i] = 0.f, mr[i] = -FLT_MAX;
         // Row r of x = q * sm_scale * log2(e): one power-of-two prescale 2^k
         // puts the row maximum in [256, 512); then term l quantises the
         // residual y (group scale = E4M3 of its 16-element maximum / 6,
@@ -468,7 +524,7 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
         // columns r*8 .. r*8+7 summed and times 2^-k give the row's scores.
         // (Any rounding of the scales and codes would do: only the residual
         // bookkeeping has to be exact.)
-        for (int r = lq; r < RM; r += kSmxWarps) {
+        for (int r = warp - kSmxWarp0; r < RM; r += kSmxWarps) {
           float y[8];
           if (r < R) {
             const int t = r / G, g = r % G;
@@ -531,7 +587,7 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
         fence_proxy_async_smem();
         named_barrier(1, kSmxWarps * 32);
 #pragma unroll
-        for (int r = 0; r < RM; ++r) facr[r] = sh.fac[r];
+        for (int i = 0; i < RM; ++i) facr[i] = sh.fac[i];
         // Scale factors of the terms into Tensor Memory (each lane quarter
         // holds all rows): column 4*ks + n1, lane l -> row 32*n1 + l (every
         // K step's block starts on a multiple of 4 columns).
@@ -549,274 +605,252 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
           }
           tmem_st16(tl + kColSFB, w);
           tmem_wait_st();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(sh.qready);
         }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(sh.qready);
       }
 
       for (; u < sg.seg_end; ++u, ++uc) {
         const bool first = (u == seg_start);
         const int stage = uc % kStages;
-        const uint8_t *stg = sh.stages + stage * kStageBytes;
-        const uint8_t *aux = stg + kKTileBytes;
+        const uint8_t *aux = sh.stages + stage * kStageBytes + kKTileBytes;
         const int tok0 = (int)(u - sg.pair_start) * kUnitTokens;
         if (!smx) {
+          // Warps 0..3 write the K scale factors one unit ahead, so the
+          // scores of unit uc+1 need not wait for this unit's V^T.
+          if (warp < 4 && uc + 1 < n_units) write_sfa(uc + 1);
           wait_bar(&sh.full[stage], (uc / kStages) & 1, sh.flags, err);
-          if (warp < 4) {
-            // ---- K scale factors into slot uc&1 (read by the score MMAs of
-            // unit uc-2 before) ----
-            if (uc > 1) {
-              wait_bar(&sh.sready[uc & 1], ((uc >> 1) + 1) & 1, sh.flags, err);
-              tc_fence_after();
+          // ---- scale pairs of this warp's two groups (head_dim rows
+          // d0 .. d0+31, d0 = 128*hv + 32*lq), in the token pairs of the
+          // V^T words: lane (gsel, page pp, half h8) converts the pairs
+          // (8*h8 + t, 8*h8 + t + 4), t < 4.  Tokens without data (past
+          // kv_len, or an absent page) get scale 0: their bytes may hold
+          // anything, NaN patterns included. ----
+          uint32_t *vsc = sh.vsc + (warp * kVscWarpBytes) / 4;
+          {
+            const int gsel = lane >> 4, pp = (lane & 15) >> 1, h8 = lane & 1;
+            const int g = 8 * hv + 2 * lq + gsel;
+            const uint2 sw = *reinterpret_cast<const uint2 *>(aux + pp * kAuxPageBytes + kAuxVs +
+                                                              g * 16 + 8 * h8);
+            int nval = sg.kv_len - (tok0 + 16 * pp + 8 * h8);
+            if (sh.pages[stage * kUnitPages + pp] < 0) nval = 0;
+            uint32_t w0 = sw.x, w1 = sw.y;
+            if (nval < 8) {
+              w0 = nval >= 4 ? w0 : nval <= 0 ? 0u : w0 & ((1u << (8 * nval)) - 1u);
+              w1 = nval <= 4 ? 0u : w1 & ((1u << (8 * (nval - 4))) - 1u);
             }
-            uint32_t w[16];
-#pragma unroll
-            for (int m1 = 0; m1 < 4; ++m1) {
-              const int j = 32 * m1 + lane;  // token of the unit
-              const uint4 v = *reinterpret_cast<const uint4 *>(aux + (j >> 4) * kAuxPageBytes +
-                                                               kAuxKs + (j & 15) * 16);
-              w[0 * 4 + m1] = v.x;
-              w[1 * 4 + m1] = v.y;
-              w[2 * 4 + m1] = v.z;
-              w[3 * 4 + m1] = v.w;
-            }
-            tmem_st16(tl + kColSFA + (uc & 1) * 16, w);
-            tmem_wait_st();
-            tc_fence_before();
+            const uint4 t4 = make_uint4(e4m3x2_to_f16x2(__byte_perm(w0, w1, 0x40)),
+                                        e4m3x2_to_f16x2(__byte_perm(w0, w1, 0x51)),
+                                        e4m3x2_to_f16x2(__byte_perm(w0, w1, 0x62)),
+                                        e4m3x2_to_f16x2(__byte_perm(w0, w1, 0x73)));
+            __syncwarp();  // the previous unit's table has been read
+            *reinterpret_cast<uint4 *>(vsc + pp * 16 + gsel * 8 + 4 * h8) = t4;
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.sfa_ready[uc & 1]);
           }
-          // ---- V^T codes into slot uc&1 (read by the value MMAs of uc-2):
-          // head_dim row d = 128*hv + 32*lq + lane, all 8 pages.
-          // Every code gives a finite value, so the slots of absent tokens
-          // need no clearing: their weights P' are zero. ----
+          // ---- V^T into slot uc&1, this warp's half (read by the value
+          // MMAs of that half of unit uc-2): head_dim row
+          // d = 128*hv + 32*lq + lane, all 8 pages. ----
           if (uc > 1) {
-            wait_bar(&sh.pvdone[uc & 1], ((uc >> 1) + 1) & 1, sh.flags, err);
+            wait_bar(&sh.pvdone[(uc & 1) * 2 + hv], ((uc >> 1) + 1) & 1, sh.flags, err);
             tc_fence_after();
           }
           {
             const int d = 128 * hv + 32 * lq + lane;
             const uint32_t vcol = kColV + (uc & 1) * 128 + 64 * hv;
+            const uint32_t *vg = vsc + (lane >> 4) * 8;
 #pragma unroll
             for (int p = 0; p < kUnitPages; ++p) {
               const uint2 cw =
                   *reinterpret_cast<const uint2 *>(aux + p * kAuxPageBytes + kAuxVc + d * 8);
-              const uint32_t o8[8] = {code_pair<0>(cw.x), code_pair<1>(cw.x), code_pair<2>(cw.x),
-                                      code_pair<3>(cw.x), code_pair<0>(cw.y), code_pair<1>(cw.y),
-                                      code_pair<2>(cw.y), code_pair<3>(cw.y)};
+              const uint4 s0 = *reinterpret_cast<const uint4 *>(vg + p * 16);
+              const uint4 s1 = *reinterpret_cast<const uint4 *>(vg + p * 16 + 4);
+              const uint32_t o8[8] = {
+                  mul_f16x2(code_pair<0>(cw.x), s0.x), mul_f16x2(code_pair<1>(cw.x), s0.y),
+                  mul_f16x2(code_pair<2>(cw.x), s0.z), mul_f16x2(code_pair<3>(cw.x), s0.w),
+                  mul_f16x2(code_pair<0>(cw.y), s1.x), mul_f16x2(code_pair<1>(cw.y), s1.y),
+                  mul_f16x2(code_pair<2>(cw.y), s1.z), mul_f16x2(code_pair<3>(cw.y), s1.w)};
               tmem_st8(tl + vcol + 8 * p, o8);
             }
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-              mbar_arrive(&sh.vready[uc & 1]);
+              mbar_arrive(&sh.vready[(uc & 1) * 2 + hv]);
               mbar_arrive(&sh.empty[stage]);  // this warp's reads of the stage are done
             }
           }
         } else {
-          // ---- softmax on S^T slot uc&1: thread = token tok0 + 32*lq + lane ----
+          // ---- softmax on S^T slot uc&1: thread = token tok0 + 32*lq + lane
           const int pos = tok0 + 32 * lq + lane;
-          // The token's V scales (one per group of 16 head_dim elements) as
-          // f16 pairs of groups (2k, 2k+1), read as soon as the stage has
-          // landed, before the scores are ready.  A token without data (past
-          // kv_len, or an absent page) gets zero scales, so whatever its
-          // bytes hold cannot reach the sum.
-          wait_bar(&sh.full[stage], (uc / kStages) & 1, sh.flags, err);
-          const int pg = (32 * lq + lane) >> 4, i = lane & 15;
-          uint32_t sc2[kHalfGroups];
-          {
-            const bool tok_ok = pos < sg.kv_len && sh.pages[stage * kUnitPages + pg] >= 0;
-            const uint8_t *vs = aux + pg * kAuxPageBytes + kAuxVs + i;
-#pragma unroll
-            for (int k2 = 0; k2 < kHalfGroups; ++k2) {
-              const uint32_t two =
-                  (uint32_t)vs[(2 * k2) * 16] | ((uint32_t)vs[(2 * k2 + 1) * 16] << 8);
-              sc2[k2] = tok_ok ? e4m3x2_to_f16x2(two) : 0u;
-            }
-          }
           wait_bar(&sh.sready[uc & 1], (uc >> 1) & 1, sh.flags, err);
           tc_fence_after();
-          const bool vis_all = tok0 + kUnitTokens <= sg.kv_len - T + 1;
-          const uint32_t sslot = tl + kColS + (uc & 1) * kNSMax;
-          uint32_t *my_mask = sh.masks + ((uc & 1) * kSmxWarps + lq) * 4;
-          // Scores of the rows: the sum of each row's 8 term columns (packed
-          // fp32 adds) times the row's 2^-k; invisible keys and padding rows
-          // -inf.
-          auto load_scores = [&](float (&x)[RM]) {
+          // Scores: the sum of each row's 8 term columns (packed fp32 adds)
+          // times the row's 2^-k; invisible keys and padding rows -inf.
+          float x[RM];
+          {
             uint32_t rr[NS];
+            const uint32_t scol = tl + kColS + (uc & 1) * kNSMax;
 #pragma unroll
-            for (int c32 = 0; c32 < NS / 32; ++c32) tmem_ld32(sslot + 32 * c32, rr + 32 * c32);
-            if (NS % 32) tmem_ld16(sslot + NS - 16, *reinterpret_cast<uint32_t(*)[16]>(rr + NS - 16));
+            for (int i = 0; i < NS / 16; ++i)
+              tmem_ld16(scol + 16 * i, *reinterpret_cast<uint32_t(*)[16]>(rr + 16 * i));
             tmem_wait_ld();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sh.sfree[uc & 1]);  // S^T slot read
+            const bool vis_all = tok0 + kUnitTokens <= sg.kv_len - T + 1;
 #pragma unroll
-            for (int r = 0; r < RM; ++r) {
-              const uint32_t *c8 = rr + r * kTerms;
+            for (int j = 0; j < RM; ++j) {
+              const uint32_t *c8 = rr + j * kTerms;
               const float2 a0 = add_f32x2(make_float2(__uint_as_float(c8[0]), __uint_as_float(c8[1])),
                                           make_float2(__uint_as_float(c8[2]), __uint_as_float(c8[3])));
               const float2 a1 = add_f32x2(make_float2(__uint_as_float(c8[4]), __uint_as_float(c8[5])),
                                           make_float2(__uint_as_float(c8[6]), __uint_as_float(c8[7])));
               const float2 a2 = add_f32x2(a0, a1);
-              const float sc = (a2.x + a2.y) * facr[r];
-              const int nv = vis_all ? (r < R ? 0x7fffffff : 0) : sh.nvis_s[r];
-              x[r] = pos < nv ? sc : -INFINITY;
+              const float sc = (a2.x + a2.y) * facr[j];
+              const int nv = vis_all ? (j < R ? 0x7fffffff : 0) : sh.nvis_s[j];
+              x[j] = pos < nv ? sc : -INFINITY;
             }
-          };
-          float x[RM], m[RM];
-          load_scores(x);
-          // A running max of -inf (no key seen yet) is taken as -FLT_MAX, so
-          // an invisible key gives weight 0 and a visible one forces the slow
-          // path, never -inf - -inf.
-#pragma unroll
-          for (int r = 0; r < RM; ++r) m[r] = fmaxf(sh.m_s[r], -FLT_MAX);
-          // Weights of the value MMA: f16(p/4) in both halves of a pair, p =
-          // 2^(score - running max) in fp32 (2^-inf = 0).
-          uint32_t pq2[RM];
+          }
+          // Weights: p = 2^(score - running max) in fp32 (2^-inf = 0), as
+          // f16 pairs of rows (2i, 2i+1).  The running max starts at -FLT_MAX
+          // (no key seen yet), so a visible key always forces the slow path.
+          uint32_t pw[RM / 2];
           bool up = false;
           auto weights = [&]() {
 #pragma unroll
-            for (int r = 0; r < RM; ++r) {
-              const float dd = x[r] - m[r];
-              up |= dd > kLazyRescale;
-              pq2[r] = ex2_quarter_f16x2(dd);
+            for (int j = 0; j < RM; j += 2) {
+              const float d0 = x[j] - mr[j], d1 = x[j + 1] - mr[j + 1];
+              up |= (d0 > kLazyRescale) | (d1 > kLazyRescale);
+              pw[j / 2] = ex2_f32_to_f16x2(d0, d1);
             }
           };
           weights();
+          uint32_t *masks = sh.masks + (uc & 1) * 4;
           const uint32_t wup = __ballot_sync(0xffffffffu, up);
-          if (lane == 0) my_mask[0] = wup;
+          if (lane == 0) masks[lq] = wup;
           named_barrier(1, kSmxWarps * 32);
-          uint32_t any = 0;
-#pragma unroll
-          for (int w = 0; w < kSmxWarps; ++w) any |= sh.masks[((uc & 1) * kSmxWarps + w) * 4];
+          const uint32_t any = masks[0] | masks[1] | masks[2] | masks[3];
           if (any) {
             // Slow path (the first unit of a segment and rare max raises):
             // exact row maxima, new running max, rescale of everything
             // accumulated against the old max, weights recomputed.
 #pragma unroll
-            for (int r = 0; r < RM; ++r) {
-              const float wm = warp_max(x[r]);
-              if (lane == 0) sh.red[lq * kNP + r] = wm;
+            for (int j = 0; j < RM; ++j) {
+              const float wm = warp_max(x[j]);
+              if (lane == 0) sh.red[lq * kNP + j] = wm;
             }
             named_barrier(1, kSmxWarps * 32);
-            if (stid < kNP) {
-              const int n = stid;
+            if (stid < RM) {
               float alpha = 1.f;
-              if (n < R) {
+              if (stid < R) {
                 float tmax = -INFINITY;
 #pragma unroll
-                for (int w = 0; w < kSmxWarps; ++w) tmax = fmaxf(tmax, sh.red[w * kNP + n]);
-                const float m_old = sh.m_s[n];
-                if (tmax > -INFINITY && (m_old == -INFINITY || tmax > m_old + kLazyRescale)) {
-                  alpha = exp2f(m_old - tmax);  // 0 when the old max was -inf
-                  sh.m_s[n] = tmax;
+                for (int w = 0; w < 4; ++w) tmax = fmaxf(tmax, sh.red[w * kNP + stid]);
+                const float m_old = sh.m_s[stid];
+                if (tmax > m_old + kLazyRescale) {
+                  alpha = exp2f(m_old - tmax);  // 0 when nothing was seen before
+                  sh.m_s[stid] = tmax;
                 }
               }
-              sh.alpha_s[n] = alpha;
+              sh.alpha_s[stid] = alpha;
             }
             named_barrier(1, kSmxWarps * 32);
+            float al[RM];
 #pragma unroll
-            for (int n = 0; n < RM; ++n) l_part[n] *= sh.alpha_s[n];
+            for (int j = 0; j < RM; ++j) {
+              al[j] = sh.alpha_s[j];
+              l_part[j] *= al[j];
+              mr[j] = sh.m_s[j];
+            }
             if (!first) {
               // O^T rows d = 32*lq + lane and d + 128, accumulated up to the
               // previous unit, scale by alpha once its value MMAs finished.
-              wait_bar(&sh.pvdone[(uc - 1) & 1], ((uc - 1) >> 1) & 1, sh.flags, err);
+              wait_bar(&sh.pvdone[((uc - 1) & 1) * 2], ((uc - 1) >> 1) & 1, sh.flags, err);
+              wait_bar(&sh.pvdone[((uc - 1) & 1) * 2 + 1], ((uc - 1) >> 1) & 1, sh.flags, err);
               tc_fence_after();
 #pragma unroll
               for (int half = 0; half < 2; ++half) {
+                uint32_t r8[8];
+                const uint32_t col = tl + kColO + half * kNP;
+                tmem_ld8(col, r8);
+                tmem_wait_ld();
 #pragma unroll
-                for (int r = 0; r < RM; ++r) {  // the 8 group columns of row r
-                  uint32_t r8[8];
-                  const uint32_t col = tl + kColO + half * kNPMax + r * kHalfGroups;
-                  tmem_ld8(col, r8);
-                  tmem_wait_ld();
-                  const float al = sh.alpha_s[r];
-#pragma unroll
-                  for (int j = 0; j < 8; ++j) r8[j] = __float_as_uint(__uint_as_float(r8[j]) * al);
-                  tmem_st8(col, r8);
-                }
+                for (int j = 0; j < RM; ++j) r8[j] = __float_as_uint(__uint_as_float(r8[j]) * al[j]);
+                tmem_st8(col, r8);
               }
               tmem_wait_st();
             }
-#pragma unroll
-            for (int r = 0; r < RM; ++r) m[r] = fmaxf(sh.m_s[r], -FLT_MAX);
             weights();
           }
-          // P' into slot uc&1 (read by the value MMAs of unit uc-2 before):
-          // for each half of head_dim and each row r, the 8 values
-          // f16(p_r/4) * vscale[g] of the half's groups g, as the MN-major B
-          // operand: element (n = 8r + g, k) at (n/8)*2048 + (k/8)*128 +
-          // (k%8)*16 + (n%8)*2.  Token slot i of page pg sits at K position
+          // P into ring slot uc%4 (read by the value MMAs of unit uc-4
+          // before): rows 0..7 of token slot i of page pg at K position
           // k = 16*pg + 8*(i/8) + 2*(i%4) + (i/4)%2, the order of the V^T
-          // code pairs.  A token without data (past kv_len, or an absent
-          // page) gets zero scales, so whatever its bytes hold cannot reach
-          // the sum.
-          if (uc > 1) {
-            wait_bar(&sh.pvdone[uc & 1], ((uc >> 1) + 1) & 1, sh.flags, err);
+          // token pairs; the MN-major B operand puts element (n, k) at
+          // (n/8)*2048 + (k/8)*128 + (k%8)*16 + (n%8)*2.
+          const int ps = uc % kPSlots;
+          if (uc >= (uint32_t)kPSlots) {
+            wait_bar(&sh.pfree[ps], ((uc / kPSlots) + 1) & 1, sh.flags, err);
             tc_fence_after();
           }
           {
+            const int j = 32 * lq + lane, pg = j >> 4, i = j & 15;
             const int kk = 16 * pg + 8 * (i >> 3) + 2 * (i & 3) + ((i >> 2) & 1);
-            uint8_t *pt = sh.ptile + (uc & 1) * kPSlotBytes + (kk >> 3) * 128 + (kk & 7) * 16;
+            uint32_t w4[4] = {0u, 0u, 0u, 0u};
 #pragma unroll
-            for (int half = 0; half < 2; ++half)
-#pragma unroll
-              for (int r = 0; r < RM; ++r)
-                *reinterpret_cast<uint4 *>(pt + half * kPHalfBytes + r * 2048) = make_uint4(
-                    hmul2_u32(pq2[r], sc2[4 * half + 0]), hmul2_u32(pq2[r], sc2[4 * half + 1]),
-                    hmul2_u32(pq2[r], sc2[4 * half + 2]), hmul2_u32(pq2[r], sc2[4 * half + 3]));
+            for (int k2 = 0; k2 < RM / 2; ++k2) w4[k2] = pw[k2];
+            *reinterpret_cast<uint4 *>(sh.ptile + ps * kPSlotBytes + (kk >> 3) * 128 +
+                                       (kk & 7) * 16) = make_uint4(w4[0], w4[1], w4[2], w4[3]);
           }
-          // the denominator sums the same f16(p/4) the value MMAs start from
+          // the denominator sums the same f16 weights the value MMAs use
 #pragma unroll
-          for (int r = 0; r < RM; ++r) l_part[r] += f16x2_to_float2(pq2[r]).x;
+          for (int k2 = 0; k2 < RM / 2; ++k2) {
+            const float2 f = f16x2_to_float2(pw[k2]);
+            l_part[2 * k2] += f.x;
+            l_part[2 * k2 + 1] += f.y;
+          }
           fence_proxy_async_smem();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) {
-            mbar_arrive(&sh.pready[uc & 1]);
-            mbar_arrive(&sh.empty[stage]);  // the V scales have been read
-          }
+          if (lane == 0) mbar_arrive(&sh.pready[ps]);
         }
       }
 
       // ---- end of segment: O^T / l -> workspace, lse ----
       if (uc > 0) {
-        wait_bar(&sh.pvdone[(uc - 1) & 1], ((uc - 1) >> 1) & 1, sh.flags, err);  // last PV
+        // the last unit's value MMAs, both halves
+        wait_bar(&sh.pvdone[((uc - 1) & 1) * 2], ((uc - 1) >> 1) & 1, sh.flags, err);
+        wait_bar(&sh.pvdone[((uc - 1) & 1) * 2 + 1], ((uc - 1) >> 1) & 1, sh.flags, err);
         tc_fence_after();
       }
       if (smx) {
 #pragma unroll
-        for (int n = 0; n < RM; ++n) {
-          const float ls = warp_sum(l_part[n]);
-          if (lane == 0) sh.red[lq * kNP + n] = ls;
+        for (int j = 0; j < RM; ++j) {
+          const float ls = warp_sum(l_part[j]);
+          if (lane == 0) sh.red[lq * kNP + j] = ls;
         }
       }
       named_barrier(2, kSegThreads);
       if (smx && stid < RM) {
         float l = 0.f;
 #pragma unroll
-        for (int w = 0; w < kSmxWarps; ++w) l += sh.red[w * kNP + stid];
+        for (int w = 0; w < 4; ++w) l += sh.red[w * kNP + stid];
         sh.alpha_s[stid] = l;
       }
       named_barrier(2, kSegThreads);
       if (!smx) {
-        // Row d keeps the column of its own group; the sums carry the 2^-14
-        // of the codes and the 1/4 of the weights, and l the same 1/4:
-        // o = O * 2^14 / l, lse = m + log2(4 l).
+        // The sums carry the 2^-14 of V^T: o = O * 2^14 / l, lse = m + log2(l).
         const int d = 128 * hv + 32 * lq + lane;
-        const int gl = (32 * lq + lane) >> 4;  // group within the half
+        uint32_t o8[8];
+        tmem_ld8(tl + kColO + hv * kNP, o8);
+        tmem_wait_ld();
 #pragma unroll
         for (int n = 0; n < RM; ++n) {
-          uint32_t o8[8];
-          tmem_ld8(tl + kColO + hv * kNPMax + n * kHalfGroups, o8);
-          tmem_wait_ld();
-          float v = 0.f;
-#pragma unroll
-          for (int j = 0; j < 8; ++j) v = j == gl ? __uint_as_float(o8[j]) : v;
           if (n < R) {
             const float lv = sh.alpha_s[n];
+            const float v = __uint_as_float(o8[n]);
             ws_o[(slot * R + n) * kD + d] = lv > 0.f ? v * 16384.f / lv : 0.f;
-            if (d == 0) ws_lse[slot * R + n] = lv > 0.f ? sh.m_s[n] + 2.f + log2f(lv) : -INFINITY;
+            if (d == 0) ws_lse[slot * R + n] = lv > 0.f ? sh.m_s[n] + log2f(lv) : -INFINITY;
           }
         }
       }
