@@ -51,15 +51,18 @@
 // Per 128-token unit the tensor pipe runs 4 NVFP4 MMAs (scores) and 16 f16
 // MMAs (values), against 16 + 16 f16 MMAs when K is dequantised.
 //
-// Roles (one persistent CTA per split-plan range, 480 threads):
+// Roles (one persistent CTA per split-plan range, 512 threads):
 //  * warp 12 (TMA): per page two tiled loads, no multicast: the 16 rows of K
-//    codes (128-byte swizzle, into the unit's contiguous K tile) and the 20
-//    rows of K scales, V codes and V scales (no swizzle); 4-stage ring.
-//  * warps 0..3 copy the K scale bytes of the next unit into the Tensor
-//    Memory scale-factor layout (every lane quarter holds the same 32 rows);
-//    warps 0..7 write the scaled V^T into Tensor Memory (one head_dim row a
-//    lane).
-//  * warps 8..11 (softmax, one token a lane): recombine the terms, mask,
+//    codes (128-byte swizzle, into the unit's contiguous K tile) and the 18
+//    rows of V codes and V scales (no swizzle); 5-stage ring.  Warp 15 loads
+//    the 2 rows of K scale bytes of each page into a separate 8-slot ring,
+//    so the scale factors written one unit ahead hold no stage of the big
+//    ring and the big ring keeps 5 units of loads in flight.
+//  * warps 0..7 write the scaled V^T into Tensor Memory (one head_dim row
+//    a lane).
+//  * warps 8..11 (softmax, one token a lane): copy the K scale bytes of the
+//    next unit into the Tensor Memory scale-factor layout (every lane
+//    quarter holds the same 32 rows), recombine the terms, mask,
 //    running max raised lazily (only when a score exceeds it by more than
 //    2^8, detected by a vote), fp32 exp2, P to a 4-slot ring in shared
 //    memory, the denominator from the same f16 weights; at a segment start
@@ -79,16 +82,19 @@ using namespace sm100;
 
 constexpr int kD = 256;
 constexpr int kRowsPerHead = 36;         // 18*D bytes / 128
-constexpr int kHeadBytes = 18 * kD;      // 4608
 constexpr int kUnitPages = 8;
 constexpr int kKRows = 16;               // K-code rows of a page block (one per token)
-constexpr int kAuxRows = 20;             // K scales (2), V codes (16), V scales (2)
+constexpr int kKsRows = 2;               // K scales: 16 tokens x 16 groups
+constexpr int kVRows = 18;               // V codes (16), V scales (2)
 constexpr int kKPageBytes = kKRows * 128;         // 2048
-constexpr int kAuxPageBytes = kAuxRows * 128;     // 2560
+constexpr int kVPageBytes = kVRows * 128;         // 2304
+constexpr int kKsPageBytes = kKsRows * 128;       // 256
 constexpr int kKTileBytes = kUnitPages * kKPageBytes;      // 16384
-constexpr int kStageBytes = kKTileBytes + kUnitPages * kAuxPageBytes;  // 36864
-constexpr int kAuxKs = 0, kAuxVc = 256, kAuxVs = 2304;    // offsets inside a page's aux block
-constexpr int kStages = 4;
+constexpr int kStageBytes = kKTileBytes + kUnitPages * kVPageBytes;  // 34816
+constexpr int kVc = 0, kVs = 2048;       // V codes, V scales inside a page's V block
+constexpr int kStages = 5;
+constexpr int kKsSlots = 8;              // ring of the units' K scale bytes
+constexpr int kKsSlotBytes = kUnitPages * kKsPageBytes;    // 2048
 
 constexpr int kRowsCap = 6;              // query rows per pair (T * G) this kernel takes
 constexpr int kTerms = 8;                // NVFP4 terms per query row
@@ -99,10 +105,11 @@ constexpr int kPSlots = 4;               // P ring depth
 constexpr int kDeqWarps = 8;             // warps 0..7
 constexpr int kSmxWarp0 = 8;             // warps 8..11
 constexpr int kSmxWarps = 4;
-constexpr int kProducerWarp = 12;
+constexpr int kProducerWarp = 12;        // K codes and V
 constexpr int kMmaWarp = 13;             // issues the score MMAs
 constexpr int kPvWarp = 14;              // issues the value MMAs
-constexpr int kThreads = 15 * 32;
+constexpr int kKsProducerWarp = 15;      // K scales
+constexpr int kThreads = 16 * 32;
 constexpr int kSegThreads = (kDeqWarps + kSmxWarps) * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr long long kWaitBudget = 2000000000LL;  // clock cycles (~1 s)
@@ -119,7 +126,8 @@ static_assert(kColS + 2 * kNSMax <= kColO && kColO + 2 * kNP <= kColSFA &&
               "tensor memory");
 
 // Shared memory (offsets from a 1024-byte aligned base).
-constexpr int kOffQ = kStages * kStageBytes;        // query terms, kNSMax rows x 128 B, swizzled
+constexpr int kOffKs = kStages * kStageBytes;       // K scale ring [slot][page][token][16]
+constexpr int kOffQ = kOffKs + kKsSlots * kKsSlotBytes;  // query terms, kNSMax rows x 128 B, swizzled
 constexpr int kOffP = kOffQ + kNSMax * 128;         // P tiles [slot], MN-major f16
 constexpr int kPSlotBytes = 2 * 2048;               // rows 0..7, rows 8..15 (zero) x 128 tokens
 constexpr int kOffVsc = kOffP + kPSlots * kPSlotBytes;  // V scale pairs [warp][page][group][8]
@@ -134,25 +142,29 @@ constexpr int kOffNvis = kOffAlpha + kNP * 4;
 constexpr int kOffFlags = kOffNvis + kNP * 4;       // int[4]: abort at [2]
 constexpr int kOffPages = kOffFlags + 16;           // int[stages][8]
 constexpr int kOffBars = kOffPages + kStages * kUnitPages * 4;
-constexpr int kNumBars = 2 * kStages + 2 * 4 + 3 * kPSlots + 3;
+constexpr int kNumBars = 2 * kStages + 2 * kKsSlots + 2 * 4 + 3 * kPSlots + 3;
 constexpr int kOffTmem = kOffBars + kNumBars * 8;
 constexpr int kSmemBytes = kOffTmem + 16 + 1024;    // + alignment slack
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
 static_assert(kOffQ % 1024 == 0 && kStageBytes % 1024 == 0 && kOffP % 128 == 0 &&
+                  kOffKs % 128 == 0 &&
                   kOffVsc % 16 == 0 && kOffSfb % 16 == 0 && kOffPages % 16 == 0 &&
                   kOffBars % 8 == 0,
               "alignment");
 
 struct Shared {
-  uint8_t *stages, *qtile, *ptile, *sfb;
+  uint8_t *stages, *ks, *qtile, *ptile, *sfb;
   uint32_t *vsc;
   float *fac, *red, *m_s, *alpha_s;
   int32_t *nvis_s, *pages;
   uint32_t *masks;
   volatile int *flags;
-  // A barrier of a ring slot completes once per unit that uses the slot, so
-  // a parity wait is never more than one phase behind.
+  // A barrier of a ring slot completes once per unit that uses the slot.  A
+  // parity wait for unit u on it is only valid once the unit before u on
+  // the same slot has been seen complete (else the parity aliases); every
+  // wait below states or follows from that.
   uint64_t *full, *empty;        // [kStages]
+  uint64_t *ks_full, *ks_empty;  // [kKsSlots]
   uint64_t *sfa_ready, *sready;  // [2]: scale factors of K written; S^T written
   uint64_t *sfree;               // [2]: S^T read by the softmax
   uint64_t *vready, *pvdone;     // [slot][half]: V^T written; value MMAs done
@@ -234,7 +246,8 @@ __device__ __forceinline__ uint32_t mul_f16x2(uint32_t a, uint32_t b) {
 template <int RM>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
-                  const __grid_constant__ CUtensorMap tmap_aux, int num_pages, int Hkv,
+                  const __grid_constant__ CUtensorMap tmap_ks,
+                  const __grid_constant__ CUtensorMap tmap_v, int num_pages, int Hkv,
                   const int32_t *__restrict__ page_table, int max_pages,
                   const int32_t *__restrict__ kv_lens, int B, int max_kv_len,
                   const __nv_bfloat16 *__restrict__ q, int T, int Hq, float qscale, int S,
@@ -248,6 +261,7 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
                                               ~uintptr_t(1023));
   Shared sh;
   sh.stages = smem;
+  sh.ks = smem + kOffKs;
   sh.qtile = smem + kOffQ;
   sh.ptile = smem + kOffP;
   sh.vsc = reinterpret_cast<uint32_t *>(smem + kOffVsc);
@@ -263,7 +277,9 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBars);
   sh.full = bars;
   sh.empty = bars + kStages;
-  sh.sfa_ready = bars + 2 * kStages;
+  sh.ks_full = bars + 2 * kStages;
+  sh.ks_empty = sh.ks_full + kKsSlots;
+  sh.sfa_ready = sh.ks_empty + kKsSlots;
   sh.sready = sh.sfa_ready + 2;
   sh.sfree = sh.sfa_ready + 4;
   sh.vready = sh.sfa_ready + 6;   // [slot][half]
@@ -284,8 +300,12 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
       mbar_init(&sh.full[i], 1);
       mbar_init(&sh.empty[i], 1 + kDeqWarps);  // the score MMAs' commit, the V^T writers
     }
+    for (int i = 0; i < kKsSlots; ++i) {
+      mbar_init(&sh.ks_full[i], 1);
+      mbar_init(&sh.ks_empty[i], kSmxWarps);  // the scale-factor writers
+    }
     for (int i = 0; i < 2; ++i) {
-      mbar_init(&sh.sfa_ready[i], 4);
+      mbar_init(&sh.sfa_ready[i], kSmxWarps);
       mbar_init(&sh.sready[i], 1);
       mbar_init(&sh.sfree[i], kSmxWarps);
       for (int h = 0; h < 2; ++h) {
@@ -323,12 +343,23 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
   const int64_t u1 = U > 0 ? range_begin(c + 1, U, S) : 0;
   const uint32_t n_units = (uint32_t)(u1 - u0);
 
-  if (warp == kProducerWarp) {
+  if (warp == kProducerWarp || warp == kKsProducerWarp) {
     // ------------------------------------------------------------------ TMA
     // Lane p < 8 owns page p of a unit; the page ids of unit u+1 are loaded
-    // while unit u's copies are issued.
-    prefetch_tmap(&tmap_k);
-    prefetch_tmap(&tmap_aux);
+    // while unit u's copies are issued.  One warp fills the stage ring (K
+    // codes into the unit's contiguous K tile, V codes and scales), the
+    // other the deeper ring of K scale bytes, which the scale-factor
+    // writers read one unit ahead of the rest.
+    const bool big = warp == kProducerWarp;
+    const int ring = big ? kStages : kKsSlots;
+    uint64_t *fullb = big ? sh.full : sh.ks_full;
+    uint64_t *emptyb = big ? sh.empty : sh.ks_empty;
+    if (big) {
+      prefetch_tmap(&tmap_k);
+      prefetch_tmap(&tmap_v);
+    } else {
+      prefetch_tmap(&tmap_ks);
+    }
     const int p = lane & 7;
     int64_t u = u0;
     Seg sg = segment_at(u, u1, kv_lens, B, Hkv, max_kv_len, max_pages);
@@ -336,44 +367,50 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
       const int tok = (int)(uu - g.pair_start) * kUnitTokens + p * kPageTokens;
       const int32_t *pt = page_table + (size_t)g.b * max_pages;
       const int pg = page_of(pt, tok, g.kv_len, num_pages);
-      if (lane < kUnitPages && tok < g.kv_len && pg < 0) report(err, NVKV_DEVERR_PAGE_ID);
+      if (big && lane < kUnitPages && tok < g.kv_len && pg < 0) report(err, NVKV_DEVERR_PAGE_ID);
       return pg;
     };
     int cur = u < u1 ? page_for(sg, u) : -1;
     uint32_t uc = 0;
     for (; u < u1; ++u, ++uc) {
-      const int stage = uc % kStages;
+      const int slot = uc % ring;
       int nxt = -1;
       Seg nsg = sg;
       if (u + 1 < u1) {
         if (u + 1 >= sg.seg_end) nsg = segment_at(u + 1, u1, kv_lens, B, Hkv, max_kv_len, max_pages);
         nxt = page_for(nsg, u + 1);
       }
-      if (uc >= (uint32_t)kStages) {
-        if (lane == 0) wait_bar(&sh.empty[stage], ((uc / kStages) + 1) & 1, sh.flags, err);
+      if (uc >= (uint32_t)ring) {
+        if (lane == 0) wait_bar(&emptyb[slot], ((uc / ring) + 1) & 1, sh.flags, err);
         __syncwarp();
       }
       const bool mine = lane < kUnitPages && cur >= 0;
-      if (lane < kUnitPages) sh.pages[stage * kUnitPages + lane] = cur;
-      const uint32_t bytes = __popc(__ballot_sync(0xffffffffu, mine)) * kHeadBytes;
+      if (big && lane < kUnitPages) sh.pages[slot * kUnitPages + lane] = cur;
+      const uint32_t bytes = __popc(__ballot_sync(0xffffffffu, mine)) *
+                             (big ? kKPageBytes + kVPageBytes : kKsPageBytes);
       __syncwarp();
-      if (lane == 0) mbar_arrive_expect_tx(&sh.full[stage], bytes);
+      if (lane == 0) mbar_arrive_expect_tx(&fullb[slot], bytes);
       __syncwarp();
       if (mine) {
-        uint8_t *st = sh.stages + stage * kStageBytes;
         const int y = (cur * Hkv + sg.h) * kRowsPerHead;
-        tma_load_2d(st + lane * kKPageBytes, &tmap_k, 0, y, &sh.full[stage]);
-        tma_load_2d(st + kKTileBytes + lane * kAuxPageBytes, &tmap_aux, 0, y + kKRows,
-                    &sh.full[stage]);
+        if (big) {
+          uint8_t *st = sh.stages + slot * kStageBytes;
+          tma_load_2d(st + lane * kKPageBytes, &tmap_k, 0, y, &fullb[slot]);
+          tma_load_2d(st + kKTileBytes + lane * kVPageBytes, &tmap_v, 0, y + kKRows + kKsRows,
+                      &fullb[slot]);
+        } else {
+          tma_load_2d(sh.ks + slot * kKsSlotBytes + lane * kKsPageBytes, &tmap_ks, 0, y + kKRows,
+                      &fullb[slot]);
+        }
       }
       cur = nxt;
       sg = nsg;
     }
     // Drain: every issued copy must land before the CTA may exit.
     if (lane == 0) {
-      const uint32_t first = uc > (uint32_t)kStages ? uc - kStages : 0;
+      const uint32_t first = uc > (uint32_t)ring ? uc - ring : 0;
       for (uint32_t k = first; k < uc; ++k)
-        mbar_wait(&sh.full[k % kStages], (k / kStages) & 1, kWaitBudget);
+        mbar_wait(&fullb[k % ring], (k / ring) & 1, kWaitBudget);
     }
     __syncwarp();
   } else if (warp == kMmaWarp || warp == kPvWarp) {
@@ -466,14 +503,15 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
 #pragma unroll
     for (int i = 0; i < RM; ++i) l_part[i] = facr[i] = 0.f, mr[i] = -FLT_MAX;
 
-    // K scale factors of unit un (its stage) into slot un&1, which the
-    // score MMAs of unit un-2 read before (warps 0..3: every lane quarter
-    // holds the same rows).  Column 4*ks + m1, lane l: the 4 scale bytes of
-    // token 32*m1 + l for head_dim elements 64*ks .. 64*ks+63.
+    // K scale factors of unit un (from the K-scale ring) into slot un&1,
+    // which the score MMAs of unit un-2 read before (the softmax warps, one
+    // unit ahead of their own; every lane quarter holds the same rows).
+    // Column 4*ks + m1, lane l: the 4 scale bytes of token 32*m1 + l for
+    // head_dim elements 64*ks .. 64*ks+63.
     auto write_sfa = [&](uint32_t un) {
-      const int st = un % kStages;
-      const uint8_t *ax = sh.stages + st * kStageBytes + kKTileBytes;
-      wait_bar(&sh.full[st], (un / kStages) & 1, sh.flags, err);
+      const int ksl = un % kKsSlots;
+      const uint8_t *kb = sh.ks + ksl * kKsSlotBytes;
+      wait_bar(&sh.ks_full[ksl], (un / kKsSlots) & 1, sh.flags, err);
       if (un > 1) {
         wait_bar(&sh.sready[un & 1], ((un >> 1) + 1) & 1, sh.flags, err);
         tc_fence_after();
@@ -481,9 +519,7 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
       uint32_t w[16];
 #pragma unroll
       for (int m1 = 0; m1 < 4; ++m1) {
-        const int j = 32 * m1 + lane;  // token of the unit
-        const uint4 v = *reinterpret_cast<const uint4 *>(ax + (j >> 4) * kAuxPageBytes + kAuxKs +
-                                                         (j & 15) * 16);
+        const uint4 v = *reinterpret_cast<const uint4 *>(kb + (32 * m1 + lane) * 16);
         w[0 * 4 + m1] = v.x;
         w[1 * 4 + m1] = v.y;
         w[2 * 4 + m1] = v.z;
@@ -493,9 +529,12 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&sh.sfa_ready[un & 1]);
+      if (lane == 0) {
+        mbar_arrive(&sh.sfa_ready[un & 1]);
+        mbar_arrive(&sh.ks_empty[ksl]);
+      }
     };
-    if (!smx && warp < 4 && n_units > 0) write_sfa(0);
+    if (smx && n_units > 0) write_sfa(0);
 
     uint32_t uc = 0;
     uint32_t seg_idx = 0;
@@ -614,12 +653,9 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
       for (; u < sg.seg_end; ++u, ++uc) {
         const bool first = (u == seg_start);
         const int stage = uc % kStages;
-        const uint8_t *aux = sh.stages + stage * kStageBytes + kKTileBytes;
+        const uint8_t *vb = sh.stages + stage * kStageBytes + kKTileBytes;
         const int tok0 = (int)(u - sg.pair_start) * kUnitTokens;
         if (!smx) {
-          // Warps 0..3 write the K scale factors one unit ahead, so the
-          // scores of unit uc+1 need not wait for this unit's V^T.
-          if (warp < 4 && uc + 1 < n_units) write_sfa(uc + 1);
           wait_bar(&sh.full[stage], (uc / kStages) & 1, sh.flags, err);
           // ---- scale pairs of this warp's two groups (head_dim rows
           // d0 .. d0+31, d0 = 128*hv + 32*lq), in the token pairs of the
@@ -631,7 +667,7 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
           {
             const int gsel = lane >> 4, pp = (lane & 15) >> 1, h8 = lane & 1;
             const int g = 8 * hv + 2 * lq + gsel;
-            const uint2 sw = *reinterpret_cast<const uint2 *>(aux + pp * kAuxPageBytes + kAuxVs +
+            const uint2 sw = *reinterpret_cast<const uint2 *>(vb + pp * kVPageBytes + kVs +
                                                               g * 16 + 8 * h8);
             int nval = sg.kv_len - (tok0 + 16 * pp + 8 * h8);
             if (sh.pages[stage * kUnitPages + pp] < 0) nval = 0;
@@ -662,7 +698,7 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
 #pragma unroll
             for (int p = 0; p < kUnitPages; ++p) {
               const uint2 cw =
-                  *reinterpret_cast<const uint2 *>(aux + p * kAuxPageBytes + kAuxVc + d * 8);
+                  *reinterpret_cast<const uint2 *>(vb + p * kVPageBytes + kVc + d * 8);
               const uint4 s0 = *reinterpret_cast<const uint4 *>(vg + p * 16);
               const uint4 s1 = *reinterpret_cast<const uint4 *>(vg + p * 16 + 4);
               const uint32_t o8[8] = {
@@ -681,7 +717,10 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
           }
         } else {
-          // ---- softmax on S^T slot uc&1: thread = token tok0 + 32*lq + lane
+          // ---- softmax on S^T slot uc&1: thread = token tok0 + 32*lq + lane.
+          // First the K scale factors of the next unit, while the scores of
+          // this one are computed.
+          if (uc + 1 < n_units) write_sfa(uc + 1);
           const int pos = tok0 + 32 * lq + lane;
           wait_bar(&sh.sready[uc & 1], (uc >> 1) & 1, sh.flags, err);
           tc_fence_after();
@@ -765,9 +804,11 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
             if (!first) {
               // O^T rows d = 32*lq + lane and d + 128, accumulated up to the
-              // previous unit, scale by alpha once its value MMAs finished.
-              wait_bar(&sh.pvdone[((uc - 1) & 1) * 2], ((uc - 1) >> 1) & 1, sh.flags, err);
-              wait_bar(&sh.pvdone[((uc - 1) & 1) * 2 + 1], ((uc - 1) >> 1) & 1, sh.flags, err);
+              // previous unit, scale by alpha once its value MMAs finished
+              // (P slot release of unit uc-1: committed after both halves;
+              // the wait of unit uc-5 on that slot is behind, so the parity
+              // cannot alias).
+              wait_bar(&sh.pfree[(uc - 1) % kPSlots], ((uc - 1) / kPSlots) & 1, sh.flags, err);
               tc_fence_after();
 #pragma unroll
               for (int half = 0; half < 2; ++half) {
@@ -818,9 +859,9 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
 
       // ---- end of segment: O^T / l -> workspace, lse ----
       if (uc > 0) {
-        // the last unit's value MMAs, both halves
-        wait_bar(&sh.pvdone[((uc - 1) & 1) * 2], ((uc - 1) >> 1) & 1, sh.flags, err);
-        wait_bar(&sh.pvdone[((uc - 1) & 1) * 2 + 1], ((uc - 1) >> 1) & 1, sh.flags, err);
+        // the last unit's value MMAs, both halves (every worker has seen
+        // the value MMAs of unit uc-5 complete)
+        wait_bar(&sh.pfree[(uc - 1) % kPSlots], ((uc - 1) / kPSlots) & 1, sh.flags, err);
         tc_fence_after();
       }
       if (smx) {
@@ -911,9 +952,10 @@ bool decode_qk4_supported(const nvkv_cache &c, int T, int Hq) {
 cudaError_t launch_decode_qk4(const nvkv_cache &c, const nvkv_seqs &s, const void *q, int T,
                               int Hq, float sm_scale, int S, float *ws_o, float *ws_lse,
                               cudaStream_t stream) {
-  CUtensorMap map_k, map_aux;
+  CUtensorMap map_k, map_ks, map_v;
   if (!make_map(c, kKRows, CU_TENSOR_MAP_SWIZZLE_128B, &map_k) ||
-      !make_map(c, kAuxRows, CU_TENSOR_MAP_SWIZZLE_NONE, &map_aux))
+      !make_map(c, kKsRows, CU_TENSOR_MAP_SWIZZLE_NONE, &map_ks) ||
+      !make_map(c, kVRows, CU_TENSOR_MAP_SWIZZLE_NONE, &map_v))
     return cudaErrorNotSupported;
   const float qscale = sm_scale * 1.4426950408889634f;
   const int R = T * (Hq / c.num_kv_heads);
@@ -923,7 +965,7 @@ cudaError_t launch_decode_qk4(const nvkv_cache &c, const nvkv_seqs &s, const voi
                                        kSmemBytes);
   if (e != cudaSuccess) return e;
   kernel<<<S, kThreads, kSmemBytes, stream>>>(
-      map_k, map_aux, c.num_pages, c.num_kv_heads, s.page_table, s.max_pages_per_seq, s.kv_lens,
+      map_k, map_ks, map_v, c.num_pages, c.num_kv_heads, s.page_table, s.max_pages_per_seq, s.kv_lens,
       s.batch, s.max_kv_len, static_cast<const __nv_bfloat16 *>(q), T, Hq, qscale, S, ws_o,
       ws_lse, s.err_word);
   return cudaGetLastError();
