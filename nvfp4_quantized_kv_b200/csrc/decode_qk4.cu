@@ -101,6 +101,7 @@ constexpr int kTerms = 8;                // NVFP4 terms per query row
 constexpr int kNSMax = kRowsCap * kTerms;   // 48: largest N of the score MMA
 constexpr int kNP = 16;                  // N of the value MMA: the query rows, padded
 constexpr int kPSlots = 4;               // P ring depth
+constexpr int kVSlots = 3;               // V^T ring depth (Tensor Memory)
 
 constexpr int kDeqWarps = 8;             // warps 0..7
 constexpr int kSmxWarp0 = 8;             // warps 8..11
@@ -115,13 +116,14 @@ constexpr uint32_t kTmemCols = 512;
 constexpr long long kWaitBudget = 2000000000LL;  // clock cycles (~1 s)
 constexpr float kLazyRescale = 8.0f;             // log2 units
 
-// Tensor Memory columns.
-constexpr uint32_t kColV = 0;      // 2 slots x 128: V^T (d-half h at +64h), f16 token pairs
-constexpr uint32_t kColS = 256;    // 2 slots x kNSMax: S^T, fp32, one token per lane
-constexpr uint32_t kColO = 352;    // 2 halves x kNP: O^T, fp32, column = query row
-constexpr uint32_t kColSFA = 384;  // 2 slots x 16: K scale factors, column 4*ks + m1
-constexpr uint32_t kColSFB = 416;  // 4 x 4: query-term scale factors, column 4*ks + n1 (n1 < 2)
-static_assert(kColS + 2 * kNSMax <= kColO && kColO + 2 * kNP <= kColSFA &&
+// Tensor Memory columns (all 512).
+constexpr uint32_t kColV = 0;      // kVSlots x 128: V^T (d-half h at +64h), f16 token pairs
+constexpr uint32_t kColS = 384;    // kNSMax: S^T, fp32, one token per lane
+constexpr uint32_t kColO = 432;    // 2 halves x kNP: O^T, fp32, column = query row
+constexpr uint32_t kColSFA = 464;  // 2 slots x 16: K scale factors, column 4*ks + m1
+constexpr uint32_t kColSFB = 496;  // 4 x 4: query-term scale factors, column 4*ks + n1 (n1 < 2)
+static_assert(kColV + kVSlots * 128 <= kColS && kColS + kNSMax <= kColO &&
+                  kColO + 2 * kNP <= kColSFA &&
                   kColSFB + 16 <= kTmemCols && kColSFA % 4 == 0 && kColSFB % 4 == 0,
               "tensor memory");
 
@@ -142,7 +144,7 @@ constexpr int kOffNvis = kOffAlpha + kNP * 4;
 constexpr int kOffFlags = kOffNvis + kNP * 4;       // int[4]: abort at [2]
 constexpr int kOffPages = kOffFlags + 16;           // int[stages][8]
 constexpr int kOffBars = kOffPages + kStages * kUnitPages * 4;
-constexpr int kNumBars = 2 * kStages + 2 * kKsSlots + 2 * 4 + 3 * kPSlots + 3;
+constexpr int kNumBars = 2 * kStages + 2 * kKsSlots + 4 + 4 * kVSlots + 2 * kPSlots + 3;
 constexpr int kOffTmem = kOffBars + kNumBars * 8;
 constexpr int kSmemBytes = kOffTmem + 16 + 1024;    // + alignment slack
 static_assert(kSmemBytes <= 227 * 1024, "shared memory");
@@ -165,9 +167,9 @@ struct Shared {
   // wait below states or follows from that.
   uint64_t *full, *empty;        // [kStages]
   uint64_t *ks_full, *ks_empty;  // [kKsSlots]
-  uint64_t *sfa_ready, *sready;  // [2]: scale factors of K written; S^T written
-  uint64_t *sfree;               // [2]: S^T read by the softmax
-  uint64_t *vready, *pvdone;     // [slot][half]: V^T written; value MMAs done
+  uint64_t *sfa_ready;           // [2]: scale factors of K written
+  uint64_t *sready, *sfree;      // S^T written; S^T read by the softmax
+  uint64_t *vready, *pvdone;     // [kVSlots][half]: V^T written; value MMAs done
   uint64_t *pready, *pfree;      // [kPSlots]: P written; P read by the value MMAs
   uint64_t *qready, *final_bar, *final_pv;
   uint32_t *tmem_slot;
@@ -281,10 +283,10 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
   sh.ks_empty = sh.ks_full + kKsSlots;
   sh.sfa_ready = sh.ks_empty + kKsSlots;
   sh.sready = sh.sfa_ready + 2;
-  sh.sfree = sh.sfa_ready + 4;
-  sh.vready = sh.sfa_ready + 6;   // [slot][half]
-  sh.pvdone = sh.sfa_ready + 10;  // [slot][half]
-  sh.pready = sh.sfa_ready + 14;
+  sh.sfree = sh.sfa_ready + 3;
+  sh.vready = sh.sfa_ready + 4;
+  sh.pvdone = sh.vready + 2 * kVSlots;
+  sh.pready = sh.pvdone + 2 * kVSlots;
   sh.pfree = sh.pready + kPSlots;
   sh.qready = sh.pfree + kPSlots;
   sh.final_bar = sh.qready + 1;
@@ -304,14 +306,12 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
       mbar_init(&sh.ks_full[i], 1);
       mbar_init(&sh.ks_empty[i], kSmxWarps);  // the scale-factor writers
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&sh.sfa_ready[i], kSmxWarps);
-      mbar_init(&sh.sready[i], 1);
-      mbar_init(&sh.sfree[i], kSmxWarps);
-      for (int h = 0; h < 2; ++h) {
-        mbar_init(&sh.vready[2 * i + h], kDeqWarps / 2);
-        mbar_init(&sh.pvdone[2 * i + h], 1);
-      }
+    for (int i = 0; i < 2; ++i) mbar_init(&sh.sfa_ready[i], kSmxWarps);
+    mbar_init(sh.sready, 1);
+    mbar_init(sh.sfree, kSmxWarps);
+    for (int i = 0; i < 2 * kVSlots; ++i) {
+      mbar_init(&sh.vready[i], kDeqWarps / 2);
+      mbar_init(&sh.pvdone[i], 1);
     }
     for (int i = 0; i < kPSlots; ++i) {
       mbar_init(&sh.pready[i], kSmxWarps);
@@ -441,17 +441,17 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
           const int stage = qk % kStages;
           wait_bar(&sh.full[stage], (qk / kStages) & 1, sh.flags, err);
           wait_bar(&sh.sfa_ready[qk & 1], (qk >> 1) & 1, sh.flags, err);
-          // S^T slot qk&1 was read by the softmax of unit qk-2
-          if (qk > 1) wait_bar(&sh.sfree[qk & 1], ((qk >> 1) + 1) & 1, sh.flags, err);
+          // S^T was read by the softmax of unit qk-1
+          if (qk > 0) wait_bar(sh.sfree, (qk - 1) & 1, sh.flags, err);
           tc_fence_after();
-          const uint32_t sslot = tmem + kColS + (qk & 1) * kNSMax;
+          const uint32_t sslot = tmem + kColS;
           const uint32_t sfa = tmem + kColSFA + (qk & 1) * 16;
           const uint32_t kt = kt0 + stage * kStageBytes;
 #pragma unroll
           for (int ks = 0; ks < 4; ++ks)
             mma_nvf4_ss(sslot, smem_desc_sw128(kt + 32 * ks), smem_desc_sw128(qb + 32 * ks),
                         idesc_qk, ks > 0, sfa + 4 * ks, tmem + kColSFB + 4 * ks);
-          mma_commit(&sh.sready[qk & 1]);
+          mma_commit(sh.sready);
           mma_commit(&sh.empty[stage]);  // the K tile has been read
           issued = true;
         }
@@ -470,18 +470,19 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
           const int ps = pv % kPSlots;
           wait_bar(&sh.pready[ps], (pv / kPSlots) & 1, sh.flags, err);
           const uint32_t pslot = pb + ps * kPSlotBytes;
-          const uint32_t vslot = tmem + kColV + (pv & 1) * 128;
+          const int vs = pv % kVSlots;
+          const uint32_t vslot = tmem + kColV + vs * 128;
           // One head_dim half at a time: each half's V^T rows are released
           // as soon as its MMAs complete.
 #pragma unroll
           for (int hf = 0; hf < 2; ++hf) {
-            wait_bar(&sh.vready[(pv & 1) * 2 + hf], (pv >> 1) & 1, sh.flags, err);
+            wait_bar(&sh.vready[vs * 2 + hf], (pv / kVSlots) & 1, sh.flags, err);
             tc_fence_after();
 #pragma unroll
             for (int ks = 0; ks < 8; ++ks)
               mma_f16_ts(tmem + kColO + hf * kNP, vslot + 64 * hf + ks * 8,
                          smem_desc(pslot + ks * 256, 128, 2048), idesc_pv, (!first) || ks > 0);
-            mma_commit(&sh.pvdone[(pv & 1) * 2 + hf]);
+            mma_commit(&sh.pvdone[vs * 2 + hf]);
           }
           mma_commit(&sh.pfree[ps]);
           issued = true;
@@ -504,18 +505,16 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
     for (int i = 0; i < RM; ++i) l_part[i] = facr[i] = 0.f, mr[i] = -FLT_MAX;
 
     // K scale factors of unit un (from the K-scale ring) into slot un&1,
-    // which the score MMAs of unit un-2 read before (the softmax warps, one
-    // unit ahead of their own; every lane quarter holds the same rows).
+    // which the score MMAs of unit un-2 read before: the softmax warps write
+    // them at the start of unit un-1, after their wait for the scores of
+    // unit un-2.  Every lane quarter holds the same rows.
     // Column 4*ks + m1, lane l: the 4 scale bytes of token 32*m1 + l for
     // head_dim elements 64*ks .. 64*ks+63.
     auto write_sfa = [&](uint32_t un) {
       const int ksl = un % kKsSlots;
       const uint8_t *kb = sh.ks + ksl * kKsSlotBytes;
       wait_bar(&sh.ks_full[ksl], (un / kKsSlots) & 1, sh.flags, err);
-      if (un > 1) {
-        wait_bar(&sh.sready[un & 1], ((un >> 1) + 1) & 1, sh.flags, err);
-        tc_fence_after();
-      }
+      tc_fence_after();
       uint32_t w[16];
 #pragma unroll
       for (int m1 = 0; m1 < 4; ++m1) {
@@ -684,16 +683,17 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
             *reinterpret_cast<uint4 *>(vsc + pp * 16 + gsel * 8 + 4 * h8) = t4;
             __syncwarp();
           }
-          // ---- V^T into slot uc&1, this warp's half (read by the value
-          // MMAs of that half of unit uc-2): head_dim row
+          // ---- V^T into slot uc%3, this warp's half (read by the value
+          // MMAs of that half of unit uc-3): head_dim row
           // d = 128*hv + 32*lq + lane, all 8 pages. ----
-          if (uc > 1) {
-            wait_bar(&sh.pvdone[(uc & 1) * 2 + hv], ((uc >> 1) + 1) & 1, sh.flags, err);
+          const int vs = uc % kVSlots;
+          if (uc >= (uint32_t)kVSlots) {
+            wait_bar(&sh.pvdone[vs * 2 + hv], ((uc / kVSlots) + 1) & 1, sh.flags, err);
             tc_fence_after();
           }
           {
             const int d = 128 * hv + 32 * lq + lane;
-            const uint32_t vcol = kColV + (uc & 1) * 128 + 64 * hv;
+            const uint32_t vcol = kColV + vs * 128 + 64 * hv;
             const uint32_t *vg = vsc + (lane >> 4) * 8;
 #pragma unroll
             for (int p = 0; p < kUnitPages; ++p) {
@@ -712,31 +712,31 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-              mbar_arrive(&sh.vready[(uc & 1) * 2 + hv]);
+              mbar_arrive(&sh.vready[vs * 2 + hv]);
               mbar_arrive(&sh.empty[stage]);  // this warp's reads of the stage are done
             }
           }
         } else {
-          // ---- softmax on S^T slot uc&1: thread = token tok0 + 32*lq + lane.
+          // ---- softmax on S^T: thread = token tok0 + 32*lq + lane.
           // First the K scale factors of the next unit, while the scores of
           // this one are computed.
           if (uc + 1 < n_units) write_sfa(uc + 1);
           const int pos = tok0 + 32 * lq + lane;
-          wait_bar(&sh.sready[uc & 1], (uc >> 1) & 1, sh.flags, err);
+          wait_bar(sh.sready, uc & 1, sh.flags, err);
           tc_fence_after();
           // Scores: the sum of each row's 8 term columns (packed fp32 adds)
           // times the row's 2^-k; invisible keys and padding rows -inf.
           float x[RM];
           {
             uint32_t rr[NS];
-            const uint32_t scol = tl + kColS + (uc & 1) * kNSMax;
+            const uint32_t scol = tl + kColS;
 #pragma unroll
             for (int i = 0; i < NS / 16; ++i)
               tmem_ld16(scol + 16 * i, *reinterpret_cast<uint32_t(*)[16]>(rr + 16 * i));
             tmem_wait_ld();
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sh.sfree[uc & 1]);  // S^T slot read
+            if (lane == 0) mbar_arrive(sh.sfree);  // S^T read
             const bool vis_all = tok0 + kUnitTokens <= sg.kv_len - T + 1;
 #pragma unroll
             for (int j = 0; j < RM; ++j) {
