@@ -56,23 +56,27 @@ DATASHEET_HBM_GBS = 8000.0
 DATASHEET_BF16_TFLOPS = 2250.0  # dense
 
 # DRAM traffic of one decode-attention launch, from one ncu capture of the
-# kernel source with this SHA-256 (profiles/decode_tc_long_ctx_3x60k_T1_full.md:
+# kernel source with this SHA-256 (profiles/decode_qk4_long_ctx_3x60k_T1.md:
 # 3 x 60000 cached tokens, T=1, 24/4 heads, d 256).  Traffic grows with the
-# KV bytes attended, so it is scaled by them to the benchmarked workload; once
-# the kernel source changes the figure no longer applies and is reported null.
+# KV bytes attended, so it is scaled by them to the benchmarked workload; it
+# applies only to that kernel, and once its source changes the figure no
+# longer applies and is reported null.
 DECODE_CAPTURE = {
-    "source": "nvfp4_quantized_kv_b200/csrc/decode_tc.cu",
-    "sha256": "854b03576476adc3f282c87bc6e05aba24cbfa0a10be5865340f81de9378f374",
-    "dram_bytes_read": 207602944,
-    "dram_bytes_write": 4987136,
+    "kernel": "decode_qk4",
+    "source": "nvfp4_quantized_kv_b200/csrc/decode_qk4.cu",
+    "sha256": "902d501081dd4c3a0763e90bdc0f6130c35acfbf9aa28bac0d9b03d8158469a2",
+    "dram_bytes_read": 207611904,
+    "dram_bytes_write": 3841792,
     "kv_bytes": 207363456,
 }
 
 
-def decode_traffic(kv_bytes):
+def decode_traffic(kv_bytes, kernel):
     """Per-launch DRAM bytes of the decode kernel scaled from the capture, or
-    None when the kernel source is not the captured one."""
+    None when another kernel ran or its source is not the captured one."""
     import hashlib
+    if kernel != DECODE_CAPTURE["kernel"] or not DECODE_CAPTURE["sha256"]:
+        return None
     try:
         with open(os.path.join(ROOT, DECODE_CAPTURE["source"]), "rb") as f:
             digest = hashlib.sha256(f.read()).hexdigest()
@@ -182,6 +186,48 @@ def oracle_sample(wl, rows_max=6, ctx_cap=None, kv=None):
     return kv_bytes / dt / 1e9, dt, min(threads, len(jobs)), desc
 
 
+# What each decode kernel computes in (the bench line's dtype).
+KERNEL_DTYPE = {
+    "decode_qk4": "nvfp4 K codes x nvfp4 q terms (block-scaled MMA), f16 P x exact f16 V MMA, "
+                  "fp32 accumulate and softmax",
+    "decode_tc": "f16 MMA on exactly dequantised K/V (q rounded to f16), f16 weights, "
+                 "fp32 accumulate",
+    "decode_simt": "fp32 on CUDA cores",
+}
+
+
+def prefill_oracle_sample(pw):
+    """Time the float64 oracle on the prefill chunk's row sample: the first
+    64, the last 64 and every 31st query, all heads, each over its causal
+    keys (keys and values quantised once per kv-head, rows from the dense
+    definition).  Returns (TFLOP/s on the sample, seconds, sampled rows,
+    extrapolated seconds for the whole chunk, description)."""
+    import oracle
+    n = pw.T
+    sample = sorted(set(range(min(64, n))) | set(range(max(0, n - 64), n)) | set(range(0, n, 31)))
+    q = pw.queries()
+    G = pw.group
+    kv_len = int(pw.kv_lens[0])
+    k, v = pw.kv_rows(0, 0, kv_len)
+    oracle.lib()
+    t0 = time.perf_counter()
+    flops = 0.0
+    for h in range(pw.num_kv_heads):
+        k_hat = oracle.qdq_rows(np.ascontiguousarray(k[:, h]))
+        v_hat = oracle.qdq_rows(np.ascontiguousarray(v[:, h]))
+        qs = np.stack([q[i, h * G + g] for i in sample for g in range(G)])
+        nvis = [pw.query_position(0, i) + 1 for i in sample for _ in range(G)]
+        oracle.attention_dense(k_hat, v_hat, qs, nvis, pw.sm_scale)
+        flops += 4.0 * pw.head_dim * sum(nvis)
+    dt = time.perf_counter() - t0
+    full = 4.0 * pw.head_dim * pw.num_q_heads * sum(pw.query_position(0, i) + 1 for i in range(n))
+    desc = (f"{len(sample)} of {n} chunk queries (first 64, last 64, every 31st) x "
+            f"{pw.num_q_heads} heads over their causal keys; float64 oracle (dequantised once "
+            f"per kv-head, numpy float64 products); measured on the sample, whole chunk "
+            f"extrapolated by FLOP")
+    return flops / dt / 1e12, dt, len(sample) * pw.num_q_heads, full / (flops / dt), desc
+
+
 def run_reference(args):
     from nvfp4_quantized_kv_b200 import workload as W
     if int(os.environ.get("RANK", "0")) != 0:
@@ -238,6 +284,8 @@ def main():
                     help="skip the K8V4-cache decode line (3 x 60k context)")
     ap.add_argument("--no-verify", action="store_true",
                     help="skip the T=6 MTP-verify line (measured on the T=1 pool)")
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the batch-2, ragged, 3 x 470,001 and T=16 sub-lines")
     ap.add_argument("--ctx", type=str, default=None,
                     help="comma-separated cached lengths replacing 330000,420000,470000 "
                          "(smaller cases for profiling)")
@@ -333,6 +381,7 @@ def main():
     tokens_per_s = world * wl.batch * wl.T / (ms * 1e-3)
     peak, peak_kind = hbm_peak()
     decode_gbs = kv_bytes / (t_decode * 1e-3) / 1e9
+    kernel = nv.nvkv_decode_kernel_name(dw.cache, wl.T, wl.num_q_heads)
 
     # ---- end to end through the public API with host buffers ----
     pin = lambda a: torch.from_numpy(np.ascontiguousarray(a)).pin_memory()
@@ -415,18 +464,89 @@ def main():
         ms6, _, d6, _ = timed_steps(dw6, K6)
         kv6 = wl6.kv_bytes_per_step()
         verify = {"workload": wl6.name, "T": 6, "steps": K6, "ms_per_step": ms6,
+                  "kernel": nv.nvkv_decode_kernel_name(dw6.cache, 6, wl6.num_q_heads),
                   "value": world * kv6 / (ms6 * 1e-3) / 1e9, "unit": "GB/s",
                   "decode_attn_ms": d6, "decode_attn_gbs": kv6 / (d6 * 1e-3) / 1e9,
                   "tokens_per_s": world * wl6.batch * wl6.T / (ms6 * 1e-3),
                   "device_errors": dw6.err_bits()}
         del dw6
 
+    # ---- the other decode workloads: batch-2 MTP verify (pools rotated so
+    # that a step never finds its KV in L2), the 64-sequence ragged batch,
+    # 3 x 470,001 tokens (the metric string's "3x~470k"), and a T=16 verify
+    # window on the long pool ----
+    def config_line(name, make, copies=1, cache_from=None, K_sub=100):
+        try:
+            dws = []
+            for _ in range(copies):
+                w = make()
+                d = DeviceWorkload(w, dev, fill=None, num_splits=args.num_splits,
+                                   cache_from=cache_from)
+                if cache_from is None:
+                    d.fill_context()
+                d.load_step_inputs()
+                dws.append(d)
+            w = dws[0].wl
+            for i in range(3 * copies):
+                dws[i % copies].step(stream)
+            Sw = dws[0].num_splits or nv.nvkv_default_num_splits()
+            ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(K_sub)]
+            torch.cuda.synchronize(dev)
+            for i in range(K_sub):
+                d, e = dws[i % copies], ev[i]
+                e[0].record(stream)
+                d.append(stream)
+                e[1].record(stream)
+                nv.nvkv_decode_attn(d.cache, d.seqs, d.q, w.T, w.num_q_heads, w.sm_scale, Sw,
+                                    d.workspace, stream)
+                e[2].record(stream)
+                nv.nvkv_combine(d.seqs, d.workspace, w.T, w.num_q_heads, w.num_kv_heads,
+                                w.head_dim, Sw, d.out, stream)
+                e[3].record(stream)
+            torch.cuda.synchronize(dev)
+            kvb = w.kv_bytes_per_step()
+            t_dec = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+            t_step = statistics.mean(e[0].elapsed_time(e[3]) for e in ev)
+            line = {"workload": w.name, "kernel": nv.nvkv_decode_kernel_name(
+                        dws[0].cache, w.T, w.num_q_heads), "T": w.T, "batch": w.batch,
+                    "kv_bytes_per_step": kvb, "steps": K_sub, "step_ms": t_step,
+                    "step_gbs": kvb / (t_step * 1e-3) / 1e9, "decode_attn_ms": t_dec,
+                    "decode_attn_gbs": kvb / (t_dec * 1e-3) / 1e9,
+                    "frac": kvb / (t_dec * 1e-3) / 1e9 / peak,
+                    "tokens_per_s": w.batch * w.T / (t_step * 1e-3),
+                    "l2": (f"{copies} pool copies rotated ({copies * kvb / 1e6:.0f} MB, L2 "
+                           f"{l2_bytes / 1e6:.0f} MB)" if copies > 1 else
+                           f"KV {kvb / 1e6:.0f} MB per step, L2 {l2_bytes / 1e6:.0f} MB"),
+                    "device_errors": max(d.err_bits() for d in dws)}
+            del dws
+            torch.cuda.empty_cache()
+            return line
+        except Exception as exc:  # a failure here must not cost the headline line
+            return {"workload": name, "error": repr(exc)[:300]}
+
+    configs = None
+    if not args.no_configs:
+        configs = {}
+        if args.T == 1:
+            configs["verify_T16"] = config_line(
+                "verify_T16", lambda: W.long_context(T=16, ctx=ctx), cache_from=dw, K_sub=50)
+        b2 = W.batch2_verify()
+        n_copies = max(1, -(-2 * l2_bytes // b2.kv_bytes_per_step()) + 1)
+        configs["batch2_T4"] = config_line("batch2_T4", W.batch2_verify, copies=n_copies)
+        configs["ragged64"] = config_line("ragged64", W.ragged_batch)
+
     # ---- chunked prefill (65536 cached + 2048 new tokens), tensor-core kernel ----
     prefill = None
     rope = None
-    if not args.no_prefill:
+    if not args.no_configs:
         del dw
         torch.cuda.empty_cache()
+        configs["long_3x470001"] = config_line(
+            "long_3x470001", lambda: W.long_context(T=1, ctx=(470000, 470000, 470000)), K_sub=50)
+    else:
+        del dw
+        torch.cuda.empty_cache()
+    if not args.no_prefill:
         pw = W.chunked_prefill()
         pdw = DeviceWorkload(pw, dev, fill=None)
         pdw.fill_context()
@@ -500,6 +620,15 @@ def main():
         v, dt, threads, desc = oracle_sample(wl)
         cpu = {"value": v, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": desc,
                "seconds": dt}
+        if prefill is not None and "error" not in prefill:
+            try:
+                tf, pdt, nrows, full_s, pdesc = prefill_oracle_sample(W.chunked_prefill())
+                prefill["cpu_baseline"] = {
+                    "value": tf, "unit": "TFLOP/s", "cores": os.cpu_count(), "kind": "oracle",
+                    "sample": pdesc, "rows": nrows, "seconds": pdt,
+                    "extrapolated_chunk_seconds": full_s}
+            except Exception as exc:
+                prefill["cpu_baseline"] = {"error": repr(exc)[:300]}
 
     # ---- decode step captured in a CUDA Graph and replayed (the serving mode
     # of the pages' engine), on its own 3 x 60k context, last so that nothing
@@ -584,7 +713,8 @@ def main():
         line = {
             "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": K,
             "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
-            "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "scaling": "weak", "vs_baseline": None, "dtype": KERNEL_DTYPE.get(kernel, kernel),
+            "data": "synthetic",
             "config": {"workload": wl.name, "batch": wl.batch, "context": list(wl.ctx),
                        "T": wl.T, "q_heads": wl.num_q_heads, "kv_heads": wl.num_kv_heads,
                        "head_dim": wl.head_dim, "page_tokens": 16, "num_splits": S,
@@ -596,14 +726,15 @@ def main():
             "decode_tokens_per_s": tokens_per_s,
             "kernel_ms": {"append": t_append, "decode_attn": t_decode, "combine": t_combine},
             "roofline": {"bound": "hbm", "achieved": decode_gbs, "peak": peak, "unit": "GB/s",
-                         "frac": decode_gbs / peak, "traffic": decode_traffic(kv_bytes),
-                         "kernel": "decode_attn", "peak_kind": peak_kind},
+                         "frac": decode_gbs / peak, "traffic": decode_traffic(kv_bytes, kernel),
+                         "kernel": kernel, "peak_kind": peak_kind},
             "e2e": {"value": world * kv_bytes / (e2e_ms * 1e-3) / 1e9, "unit": "GB/s",
                     "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms},
             "gpu_launches": 3 * K,
             "clocks": clk,
             "device_errors": err,
             "verify_T6": verify,
+            "configs": configs,
             "spill": spill,
             "prefill": prefill,
             "rope_append": rope,

@@ -141,11 +141,40 @@ nvkv_status nvkv_split_plan(const int32_t *kv_lens_host, int32_t batch, int32_t 
  *   T: 1 .. 16 queries per sequence; Hq a multiple of Hkv with T*Hq/Hkv <= 128.
  *   sm_scale: scores are sm_scale * q.k (typically 1/sqrt(D)).
  *   workspace: device, >= nvkv_decode_workspace_bytes(...), 16-B aligned.
- * The scores, softmax and value sums run in fp32 on dequantised values;
- * nvkv_combine must follow with the same T, heads and num_splits. */
+ * nvkv_combine must follow with the same T, heads and num_splits.
+ *
+ * Arithmetic (which kernel runs: nvkv_decode_kernel_name).  Every kernel
+ * uses the cached values exactly (E2M1 x E4M3 is exact in f16 and fp32),
+ * base-2 scores x = q.k * sm_scale * log2(e), an fp32 running maximum, an
+ * fp32 denominator that sums the same weights the value sum uses, fp32
+ * accumulation of the value sums, and an fp32 partial result per split:
+ *   decode_qk4 (D = 256, T*Hq/Hkv <= 6): the scores on the NVFP4
+ *     block-scaled tensor-core MMA straight from the cached K codes and
+ *     scales; q * sm_scale * log2(e) (fp32) enters as 8 stacked NVFP4
+ *     terms after a power-of-two prescale of each row, leaving a remainder
+ *     below about 1e-6 of each 16-element group's maximum, for any finite
+ *     q; the products are exact and accumulate in fp32.  Weights
+ *     p = 2^(x - m) from an fp32 exp2, rounded to f16 (relative error
+ *     <= 2^-11; below 2^-14 f16 subnormals, absolute error <= 2^-25); the
+ *     value sum is an f16 x f16 MMA with fp32 accumulation.
+ *   decode_tc (D = 256, T*Hq/Hkv <= 48): q * sm_scale * log2(e) (fp32) as
+ *     two f16 terms hi + lo (about 22 significant bits; |q * sm_scale| must
+ *     stay below about 45000, the f16 range, and elements below 2^-14 keep
+ *     an absolute precision of 2^-25), K dequantised to f16, scores on the
+ *     f16 MMA over both terms with fp32 accumulation; weights and value
+ *     sum as for decode_qk4.
+ *   decode_simt (every other shape, and NVKV_DECODE_KERNEL=simt): scores,
+ *     weights and value sums in fp32 on CUDA cores. */
 nvkv_status nvkv_decode_attn(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *q,
                              int32_t T, int32_t num_q_heads, float sm_scale, int32_t num_splits,
                              void *workspace, size_t workspace_bytes, nvkv_stream_t stream);
+
+/* Name of the decode kernel nvkv_decode_attn launches for this cache and
+ * step shape: "decode_qk4", "decode_tc" or "decode_simt" ("none" on invalid
+ * arguments).  A static string; launches nothing.  The environment variable
+ * NVKV_DECODE_KERNEL ("simt", or "tc" to skip decode_qk4) is read on every
+ * call, as nvkv_decode_attn does. */
+const char *nvkv_decode_kernel_name(const nvkv_cache *cache, int32_t T, int32_t num_q_heads);
 
 /* Decode / MTP-verify attention, second half: merges the per-split partial
  * results (log-sum-exp weighting) into out, device bf16 [batch*T][Hq][D].

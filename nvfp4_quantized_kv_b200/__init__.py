@@ -73,6 +73,7 @@ def library():
             "nvkv_split_plan": (ctypes.c_int, [vp, i32, i32, i32, vp, vp]),
             "nvkv_append": (ctypes.c_int, [cp, sp, vp, vp, vp, i32, i32, vp]),
             "nvkv_decode_attn": (ctypes.c_int, [cp, sp, vp, i32, i32, f32, i32, vp, sz, vp]),
+            "nvkv_decode_kernel_name": (ctypes.c_char_p, [cp, i32, i32]),
             "nvkv_combine": (ctypes.c_int, [sp, vp, i32, i32, i32, i32, i32, vp, vp]),
             "nvkv_prefill_attn": (ctypes.c_int, [cp, sp, vp, vp, i32, i32, i32, f32, vp, vp]),
             "nvkv_decode_static_scratch_bytes": (sz, []),
@@ -253,6 +254,14 @@ def nvkv_decode_attn(cache: Cache, seqs: Seqs, q: torch.Tensor, T: int, num_q_he
         ctypes.byref(cache._c), ctypes.byref(seqs._c), _dev(q, torch.bfloat16, "q"), int(T),
         int(num_q_heads), float(sm_scale), int(num_splits), _dev(workspace, torch.uint8, "workspace"),
         workspace.numel(), _stream(stream)), "nvkv_decode_attn")
+
+
+def nvkv_decode_kernel_name(cache: Cache, T: int, num_q_heads: int) -> str:
+    """The decode kernel nvkv_decode_attn launches for this cache and step
+    shape: "decode_qk4", "decode_tc" or "decode_simt"."""
+    _fmt(cache, "nvfp4", "nvkv_decode_kernel_name")
+    return library().nvkv_decode_kernel_name(ctypes.byref(cache._c), int(T),
+                                             int(num_q_heads)).decode()
 
 
 def nvkv_combine(seqs: Seqs, workspace: torch.Tensor, T: int, num_q_heads: int,

@@ -280,6 +280,16 @@ nvkv_status nvkv_append_rope(const nvkv_cache *cache, const nvkv_seqs *seqs, con
                                    reinterpret_cast<cudaStream_t>(stream)));
 }
 
+const char *nvkv_decode_kernel_name(const nvkv_cache *cache, int32_t T, int32_t num_q_heads) {
+  if (!cache || cache->num_kv_heads <= 0 || T <= 0 || num_q_heads <= 0 ||
+      num_q_heads % cache->num_kv_heads != 0)
+    return "none";
+  if (!force_simt() && !force_kernel("tc") && decode_qk4_supported(*cache, T, num_q_heads))
+    return "decode_qk4";
+  if (!force_simt() && decode_tc_supported(*cache, T, num_q_heads)) return "decode_tc";
+  return "decode_simt";
+}
+
 nvkv_status nvkv_decode_attn(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *q,
                              int32_t T, int32_t num_q_heads, float sm_scale, int32_t num_splits,
                              void *workspace, size_t workspace_bytes, nvkv_stream_t stream) {

@@ -15,13 +15,16 @@
 //    producer warp copies each page's 4608-byte kv-head block (36 rows of
 //    128 B) into a 4-stage shared-memory ring with one 2-D tiled load per
 //    page (128-byte swizzle: the dequantising reads are bank-conflict free).
-//    No multicast.
+//    No multicast.  (3 stages at N = 48, where the two Q tiles need room.)
 //  * Swap-AB: the dequantised K tile (128 tokens x 256 d, f16) and V^T tile
 //    (2 x 128 d x 128 tokens) are the A operands, written straight from
 //    registers into Tensor Memory; the G*T query rows (Q, then P) are the
-//    small N side of the MMA, in shared memory.  S^T and O^T accumulate in
-//    Tensor Memory in fp32; each softmax thread keeps per-row partial sums
-//    of the same f16 P the value sums use, reduced once per segment.
+//    small N side of the MMA, in shared memory; q enters as two f16 terms
+//    (hi, and the fp32 remainder lo), both multiplied by the same K tile
+//    into the same S^T.  S^T and O^T accumulate in Tensor Memory in fp32;
+//    the weights p = 2^(x - m) come from an fp32 exp2 rounded to f16, and
+//    each softmax thread keeps per-row partial sums of the same f16 P the
+//    value sums use, reduced once per segment.
 //    Dequantisation is exact in f16 (E2M1 x E4M3 has at most 6 significant
 //    bits).
 //  * 16 dequantising warps (4 per SM sub-partition): each converts a quarter
@@ -49,7 +52,6 @@ constexpr int kHeadBytes = 18 * kD;   // 4608
 constexpr int kPagePitch = 5120;      // staged page pitch (1024-aligned)
 constexpr int kUnitPages = 8;
 constexpr int kStageBytes = kUnitPages * kPagePitch;
-constexpr int kStages = 4;
 constexpr int kWorkerWarps = 16;      // dequantising warps 0..15
 constexpr int kSoftmaxWarps = 4;      // softmax warps 16..19
 constexpr int kSoftmaxWarp0 = 16;
@@ -71,6 +73,8 @@ constexpr uint32_t kColK = 0;      // K half of phase A (and B when N > 32)
 
 template <int N>
 struct Cfg {
+  // Stage ring depth: 3 at N = 48, where the two f16 Q tiles take the room.
+  static constexpr int kStages = N > 32 ? 3 : 4;
   static constexpr bool kSplitK = N <= 32;
   static constexpr uint32_t kColKB = kSplitK ? 64 : 0;       // K half of phase B
   static constexpr uint32_t kColV = kSplitK ? 128 : 64;      // 2 slots x 128: V^T
@@ -81,7 +85,8 @@ struct Cfg {
   static constexpr int kQBytes = N * kD * 2;        // Q tile, K-major, no swizzle
   static constexpr int kPBytes = N * 128 * 2;       // one P^T tile, MN-major, no swizzle
   static constexpr int kOffQ = kStages * kStageBytes;
-  static constexpr int kOffP = kOffQ + kQBytes;                 // 2 P^T tiles
+  static constexpr int kOffQlo = kOffQ + kQBytes;               // low f16 term of the Q tile
+  static constexpr int kOffP = kOffQlo + kQBytes;               // 2 P^T tiles
   static constexpr int kOffRed = kOffP + 2 * kPBytes;           // float [4][N]
   static constexpr int kOffMask = kOffRed + kSoftmaxWarps * N * 4;  // u32 [2][4][4]
   static constexpr int kOffM = kOffMask + 2 * kSoftmaxWarps * 4 * 4;
@@ -99,7 +104,7 @@ struct Cfg {
 };
 
 struct Shared {
-  uint8_t *stages, *qtile, *ptile;
+  uint8_t *stages, *qtile, *qtile_lo, *ptile;
   float *red, *m_s, *alpha_s;
   int32_t *nvis_s, *pages;
   uint32_t *masks;
@@ -165,12 +170,14 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
                  const __nv_bfloat16 *__restrict__ q, int T, int Hq, float qscale, int S,
                  float *__restrict__ ws_o, float *__restrict__ ws_lse, int32_t *err) {
   using C = Cfg<N>;
+  constexpr int kStages = C::kStages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
   Shared sh;
   sh.stages = smem;
   sh.qtile = smem + C::kOffQ;
+  sh.qtile_lo = smem + C::kOffQlo;
   sh.ptile = smem + C::kOffP;
   sh.red = reinterpret_cast<float *>(smem + C::kOffRed);
   sh.masks = reinterpret_cast<uint32_t *>(smem + C::kOffMask);
@@ -295,6 +302,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
       const uint32_t idesc_qk = idesc_f16_f32(128, N, false, false);
       const uint32_t idesc_pv = idesc_f16_f32(128, N, false, true);
       const uint32_t qb = smem_u32(sh.qtile), pb = smem_u32(sh.ptile);
+      const uint32_t qlb = smem_u32(sh.qtile_lo);
       const uint32_t n_units = (uint32_t)(u1 - u0);
       uint32_t qk = 0, pv = 0;
       int qk_phase = 0;
@@ -332,10 +340,16 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
           if (u == seg_start) first_bits |= 1u << (qk & 31);
           else first_bits &= ~(1u << (qk & 31));
           const uint32_t sslot = tmem + C::kColS + (qk & 1) * N;
+          // the high f16 terms of q, then the low ones, into the same S^T
 #pragma unroll
           for (int ks = 0; ks < 8; ++ks) {
             const uint64_t bd = smem_desc(qb + ks * 2 * (N * 16), N * 16, 128);
             mma_f16_ts(sslot, tmem + kColK + ks * 8, bd, idesc_qk, ks > 0);
+          }
+#pragma unroll
+          for (int ks = 0; ks < 8; ++ks) {
+            const uint64_t bd = smem_desc(qlb + ks * 2 * (N * 16), N * 16, 128);
+            mma_f16_ts(sslot, tmem + kColK + ks * 8, bd, idesc_qk, 1u);
           }
           mma_commit(sh.kdone_a);
           qk_phase = 1;
@@ -346,6 +360,11 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
 #pragma unroll
           for (int ks = 8; ks < 16; ++ks) {
             const uint64_t bd = smem_desc(qb + ks * 2 * (N * 16), N * 16, 128);
+            mma_f16_ts(sslot, tmem + C::kColKB + (ks - 8) * 8, bd, idesc_qk, 1u);
+          }
+#pragma unroll
+          for (int ks = 8; ks < 16; ++ks) {
+            const uint64_t bd = smem_desc(qlb + ks * 2 * (N * 16), N * 16, 128);
             mma_f16_ts(sslot, tmem + C::kColKB + (ks - 8) * 8, bd, idesc_qk, 1u);
           }
           mma_commit(&sh.sready[qk & 1]);
@@ -385,29 +404,39 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
       const int64_t seg_start = u;
       const size_t slot = (size_t)c + (size_t)sg.b * Hkv + sg.h;
 
-      // Q tile of this pair: rows n < R are (t, g) = (n / G, n % G), pre-scaled
-      // to base-2 scores, f16, K-major core-matrix layout; rows >= R are zero.
-      // (The previous segment's QK MMAs completed: every worker waited for
-      // its last PV, which follows them.)
+      // Q tiles of this pair: rows n < R are (t, g) = (n / G, n % G), pre-scaled
+      // to base-2 scores (fp32) and written as two f16 terms, hi = f16(x) and
+      // lo = f16(x - hi) (the difference is exact in fp32), which carry
+      // about 22 significant bits between them; K-major core-matrix layout;
+      // rows >= R are zero.  The score MMAs run over both tiles into the
+      // same S^T.  (The previous segment's QK MMAs completed: every worker
+      // waited for its last PV, which follows them.)
       for (int ci = smx ? N * (kD / 8) : tid; ci < N * (kD / 8); ci += kWorkerWarps * 32) {
         const int n = ci / (kD / 8), k8 = ci % (kD / 8);
-        uint4 v = make_uint4(0, 0, 0, 0);
+        uint4 v = make_uint4(0, 0, 0, 0), vl = make_uint4(0, 0, 0, 0);
         if (n < R) {
           const int t = n / G, g = n % G;
           const uint4 raw = *reinterpret_cast<const uint4 *>(
               q + ((size_t)(sg.b * T + t) * Hq + sg.h * G + g) * kD + k8 * 8);
           const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
-          uint32_t o[4];
+          uint32_t o[4], ol[4];
 #pragma unroll
           for (int i = 0; i < 4; ++i) {
-            const float lo = __uint_as_float(w[i] << 16) * qscale;
-            const float hi = __uint_as_float(w[i] & 0xffff0000u) * qscale;
-            __half2 hh = __floats2half2_rn(lo, hi);
-            o[i] = *reinterpret_cast<uint32_t *>(&hh);
+            // element 2i in the low half, 2i+1 in the high half
+            const float x0 = __uint_as_float(w[i] << 16) * qscale;
+            const float x1 = __uint_as_float(w[i] & 0xffff0000u) * qscale;
+            const __half2 hh = __floats2half2_rn(x0, x1);
+            const float2 hf = __half22float2(hh);
+            const __half2 ll = __floats2half2_rn(x0 - hf.x, x1 - hf.y);
+            o[i] = *reinterpret_cast<const uint32_t *>(&hh);
+            ol[i] = *reinterpret_cast<const uint32_t *>(&ll);
           }
           v = make_uint4(o[0], o[1], o[2], o[3]);
+          vl = make_uint4(ol[0], ol[1], ol[2], ol[3]);
         }
-        *reinterpret_cast<uint4 *>(sh.qtile + k8 * (N * 16) + (n >> 3) * 128 + (n & 7) * 16) = v;
+        const int qoff = k8 * (N * 16) + (n >> 3) * 128 + (n & 7) * 16;
+        *reinterpret_cast<uint4 *>(sh.qtile + qoff) = v;
+        *reinterpret_cast<uint4 *>(sh.qtile_lo + qoff) = vl;
       }
       fence_proxy_async_smem();
       if (smx) {
@@ -610,7 +639,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
                 const float2 dd = add_f32x2(make_float2(x[2 * e], x[2 * e + 1]),
                                             make_float2(-m[2 * e], -m[2 * e + 1]));
                 up |= (dd.x > kLazyRescale) | (dd.y > kLazyRescale);
-                h2[8 * c16 + e] = ex2_f16x2(dd.x, dd.y);  // 2^-inf = 0
+                h2[8 * c16 + e] = ex2_f32_to_f16x2(dd.x, dd.y);  // 2^-inf = 0
               }
             } else {
 #pragma unroll
@@ -689,7 +718,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
                 for (int e = 0; e < 8; ++e) {
                   const float2 dd = add_f32x2(make_float2(x[2 * e], x[2 * e + 1]),
                                               make_float2(-m[2 * e], -m[2 * e + 1]));
-                  h2[8 * c16 + e] = ex2_f16x2(dd.x, dd.y);
+                  h2[8 * c16 + e] = ex2_f32_to_f16x2(dd.x, dd.y);
                 }
               }
             }

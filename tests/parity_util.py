@@ -14,12 +14,13 @@ ATOL = 8e-3
 RTOL = 8e-3
 
 
-def oracle_outputs(wl: Workload, rows, nthreads=None, k8=False):
+def oracle_outputs(wl: Workload, rows, nthreads=None, k8=False, q=None):
     """rows: list of (b, t, hq).  Returns float64 [len(rows)][D]: the exact
     attention of query t of sequence b, head hq, over the sequence's keys
     0 .. ctx_b + t (all rows of the workload, quantised by the oracle; K in
-    the K8V4 cache's 8-bit row format when k8)."""
-    q = wl.queries()
+    the K8V4 cache's 8-bit row format when k8).  q: bf16 bits
+    [batch*T][Hq][D] replacing the workload's queries."""
+    q = wl.queries() if q is None else q
     G = wl.group
     kv = {}
     for b in sorted({r[0] for r in rows}):
@@ -34,12 +35,12 @@ def oracle_outputs(wl: Workload, rows, nthreads=None, k8=False):
     return out
 
 
-def oracle_outputs_dense(wl: Workload, rows):
+def oracle_outputs_dense(wl: Workload, rows, q=None):
     """As oracle_outputs, for many rows over long caches: the keys and values
     of each (sequence, kv-head) are quantised and dequantised once by the
     oracle (qdq_rows) and the rows are computed by oracle.attention_dense
     (pinned against the per-row oracle in test_oracle_dense_pins.py)."""
-    q = wl.queries()
+    q = wl.queries() if q is None else q
     G = wl.group
     out = np.zeros((len(rows), wl.head_dim), np.float64)
     by = {}

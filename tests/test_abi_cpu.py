@@ -282,3 +282,17 @@ def test_the_library_is_usable_from_plain_c(lib, tmp_path):
     r = subprocess.run([exe], capture_output=True, text=True, timeout=120)
     assert r.returncode == 0, r.stderr
     assert r.stdout.strip() == "ok"
+
+
+def test_decode_kernel_name_without_launch(lib):
+    """The dispatch query launches nothing; invalid shapes give "none",
+    valid ones one of the three kernel names (on a host without a GPU the
+    tensor-map encoder is missing, so it reports the CUDA-core kernel)."""
+    B = ctypes.byref
+    f = lib.nvkv_decode_kernel_name
+    assert f(None, 1, 24) == b"none"
+    assert f(B(cache(hkv=4, d=256)), 1, 25) == b"none"  # Hq % Hkv
+    assert f(B(cache(hkv=4, d=256)), 0, 24) == b"none"
+    for T in (1, 6, 16):
+        assert f(B(cache(hkv=4, d=256)), T, 24) in (b"decode_qk4", b"decode_tc", b"decode_simt")
+    assert f(B(cache(hkv=2, d=128)), 1, 8) == b"decode_simt"  # head_dim 128: CUDA cores only

@@ -9,6 +9,7 @@ import pytest
 import torch
 
 import nvfp4_quantized_kv_b200 as nv
+import oracle
 from nvfp4_quantized_kv_b200 import workload as W
 from nvfp4_quantized_kv_b200.harness import DeviceWorkload
 
@@ -80,6 +81,8 @@ def test_long_context_config_sampled(T):
     sequence, and for T=6 every head of the first query too."""
     wl = W.long_context(T=T)
     dw = run_step(wl)
+    assert nv.nvkv_decode_kernel_name(dw.cache, T, wl.num_q_heads) == (
+        "decode_qk4" if T == 1 else "decode_tc")
     ts = sorted({0, T - 1})
     rows = [(b, t, hq) for b in range(wl.batch) for t in ts for hq in range(wl.num_q_heads)]
     assert_close(gpu_rows(dw.out, wl, rows), oracle_outputs_dense(wl, rows), wl.name)
@@ -102,17 +105,67 @@ def test_rows_ending_on_page_unit_and_split_boundaries(T, num_splits):
     assert_close(gpu_rows(dw.out, wl, rows), oracle_outputs_dense(wl, rows), wl.name)
 
 
-def test_split_count_does_not_change_the_result():
+def split_count_bound(wl, rows, f16_exponent: bool):
+    """Largest difference the split count can make to an output element.
+
+    Split boundaries change which running maximum m each weight
+    p = 2^(x - m) is rounded against; the scores x (log2 units) themselves
+    do not change.  The combine merges the splits exactly up to fp32
+    rounding, so every split count computes o = sum_j P~_j v_j / sum_j P~_j
+    with P~_j the rounded weights in one global scale, and
+        o~ - o = sum_j (P~_j - P_j)(v_j - o) / sum_j P~_j.
+    A weight's error is at most e_j * p_j + 2^-25 (f16 subnormals, absolute
+    in units where the split's largest weight is >= 1, i.e. the lazy maximum
+    is at most 8 below the top score), with
+      e_j = 2^-11 + 2^-22             (fp32 exp2, one rounding to f16), or
+      e_j = 2^-9 + ln2 * 2^-11 * |x_j - m|,  |x_j - m| <= x_max - x_j + 8
+                                      (exponent argument rounded to f16, f16
+                                       exp2 and its rounding within 2^-9).
+    So |o~_d - o_d| <= sum_j w_j e_j |v_jd - o_d| + 2^-25 sum_j |v_jd - o_d|
+    (w_j the exact weights), plus fp32 accumulation (2^-20 of sum_j w_j
+    |v_jd|).  Two split counts differ by at most twice that, plus the two
+    bf16 roundings of the outputs (unit roundoff 2^-8, bf16 having 8
+    significant bits: 2^-8 |o| each).  All terms from the oracle's
+    dequantised keys and values in float64."""
+    q = wl.queries()
+    G = wl.group
+    bounds = np.zeros((len(rows), wl.head_dim))
+    cache = {}
+    for i, (b, t, hq) in enumerate(rows):
+        h = hq // G
+        if (b, h) not in cache:
+            k, v = wl.kv_rows(b, 0, int(wl.kv_lens[b]))
+            cache[(b, h)] = (oracle.qdq_rows(np.ascontiguousarray(k[:, h])),
+                             oracle.qdq_rows(np.ascontiguousarray(v[:, h])))
+        k_hat, v_hat = cache[(b, h)]
+        n = wl.query_position(b, t) + 1
+        qf = W.bf16_bits_to_f32(q[b * wl.T + t, hq]).astype(np.float64)
+        s = (k_hat[:n] @ qf) * wl.sm_scale
+        w = np.exp(s - s.max())
+        w /= w.sum()
+        o = w @ v_hat[:n]
+        x = s * np.log2(np.e)
+        if f16_exponent:
+            e = 2.0 ** -9 + np.log(2) * 2.0 ** -11 * (x.max() - x + 8)
+        else:
+            e = np.full(n, 2.0 ** -11 + 2.0 ** -22)
+        dev = np.abs(v_hat[:n] - o)
+        one = (w * e) @ dev + 2.0 ** -25 * dev.sum(axis=0) + 2.0 ** -20 * (w @ np.abs(v_hat[:n]))
+        bounds[i] = 2 * one + 2 * 2.0 ** -8 * np.abs(o) + 1e-7
+    return bounds
+
+
+@pytest.mark.parametrize("T,kernel", [(1, "decode_qk4"), (3, "decode_tc")])
+def test_split_count_does_not_change_the_result(T, kernel):
     """Combine metamorphic check: 1 split per pair up to more splits than
-    units.  Moving split boundaries changes the fp32 summation order and
-    which running max the f16 softmax weights are rounded against (relative
-    error up to 2^-11 per weight), so the outputs agree to the attention
-    tolerance rather than bit for bit; each is also checked against the
-    oracle by the other tests."""
-    wl = W.small("splits", 3, 24, 4, 256, 3, [2000, 50, 900], seed=4)
+    units give the same outputs within the bound derived in
+    split_count_bound (far tighter than the attention tolerance when the
+    weights are spread over many keys)."""
+    wl = W.small(f"splits_T{T}", 3, 24, 4, 256, T, [2000, 50, 900], seed=4)
     dw = DeviceWorkload(wl, num_splits=1)
     dw.fill_context()
     dw.load_step_inputs()
+    assert nv.nvkv_decode_kernel_name(dw.cache, T, wl.num_q_heads) == kernel
     dw.append()
     outs = []
     for S in (1, 2, 7, 64, 296, 5000):
@@ -122,10 +175,17 @@ def test_split_count_does_not_change_the_result():
                                            wl.head_dim, S), dtype=torch.uint8, device="cuda")
         dw.attend()
         torch.cuda.synchronize()
-        outs.append(dw.out.float().clone())
-    for o in outs[1:]:
-        diff = (o - outs[0]).abs()
-        assert (diff <= 8e-3 + 8e-3 * outs[0].abs()).all(), float(diff.max())
+        assert dw.err_bits() == 0
+        outs.append(dw.out.float().cpu().numpy().astype(np.float64))
+    rows = all_rows(wl)
+    bound = split_count_bound(wl, rows, f16_exponent=False)  # both: fp32 exp2, f16 weights
+    ref = np.stack([outs[0][b * wl.T + t, hq] for b, t, hq in rows])
+    for S, o in zip((2, 7, 64, 296, 5000), outs[1:]):
+        got = np.stack([o[b * wl.T + t, hq] for b, t, hq in rows])
+        ratio = np.abs(got - ref) / bound
+        assert ratio.max() <= 1.0, (S, float(ratio.max()))
+    # the bound is several times tighter than the parity tolerance
+    assert np.median(bound) < 2e-3
 
 
 def test_queries_without_keys_give_zeros():

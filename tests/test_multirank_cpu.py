@@ -67,13 +67,15 @@ def test_reference_arm_nonzero_rank_is_silent():
 def test_decode_traffic_tracks_the_captured_source(tmp_path, monkeypatch):
     import bench
     kv = 1_000_000
-    t = bench.decode_traffic(kv)
     cap = bench.DECODE_CAPTURE
+    t = bench.decode_traffic(kv, cap["kernel"])
     if t is not None:  # the source is the captured one: traffic scales with the KV bytes
         assert t == pytest.approx(kv * (cap["dram_bytes_read"] + cap["dram_bytes_write"]) /
                                   cap["kv_bytes"])
+    # another kernel ran: the capture does not describe it
+    assert bench.decode_traffic(kv, "decode_simt") is None
     monkeypatch.setitem(cap, "sha256", "0" * 64)
-    assert bench.decode_traffic(kv) is None
+    assert bench.decode_traffic(kv, cap["kernel"]) is None
 
 
 def test_reference_arm_rank0_prints_one_contract_line():
