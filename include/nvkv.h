@@ -157,13 +157,15 @@ nvkv_status nvkv_split_plan(const int32_t *kv_lens_host, int32_t batch, int32_t 
  *     p = 2^(x - m) from an fp32 exp2, rounded to f16 (relative error
  *     <= 2^-11; below 2^-14 f16 subnormals, absolute error <= 2^-25); the
  *     value sum is an f16 x f16 MMA with fp32 accumulation.
- *   decode_tc (D = 256, T*Hq/Hkv <= 48): q * sm_scale * log2(e) (fp32) as
+ *   decode_tc (D = 256, the other shapes with Hq/Hkv <= 48; more than 48
+ *     query rows per (sequence, kv-head) run as one launch per chunk of
+ *     queries, each reading the KV once): q * sm_scale * log2(e) (fp32) as
  *     two f16 terms hi + lo (about 22 significant bits; |q * sm_scale| must
  *     stay below about 45000, the f16 range, and elements below 2^-14 keep
  *     an absolute precision of 2^-25), K dequantised to f16, scores on the
  *     f16 MMA over both terms with fp32 accumulation; weights and value
  *     sum as for decode_qk4.
- *   decode_simt (every other shape, and NVKV_DECODE_KERNEL=simt): scores,
+ *   decode_simt (head_dim 128, and NVKV_DECODE_KERNEL=simt): scores,
  *     weights and value sums in fp32 on CUDA cores. */
 nvkv_status nvkv_decode_attn(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *q,
                              int32_t T, int32_t num_q_heads, float sm_scale, int32_t num_splits,

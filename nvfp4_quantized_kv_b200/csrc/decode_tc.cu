@@ -167,7 +167,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hkv,
                  const int32_t *__restrict__ page_table, int max_pages,
                  const int32_t *__restrict__ kv_lens, int B, int max_kv_len,
-                 const __nv_bfloat16 *__restrict__ q, int T, int Hq, float qscale, int S,
+                 const __nv_bfloat16 *__restrict__ q, int T, int t0, int T_all, int Hq,
+                 float qscale, int S,
                  float *__restrict__ ws_o, float *__restrict__ ws_lse, int32_t *err) {
   using C = Cfg<N>;
   constexpr int kStages = C::kStages;
@@ -201,7 +202,10 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int G = Hq / Hkv;
+  // This launch takes queries t0 .. t0+T-1 of the step's T_all (rows
+  // n < R = T*G of the chunk are rows t0*G + n of the step's R_all).
   const int R = T * G;
+  const int R_all = T_all * G;
 
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
@@ -417,7 +421,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
         if (n < R) {
           const int t = n / G, g = n % G;
           const uint4 raw = *reinterpret_cast<const uint4 *>(
-              q + ((size_t)(sg.b * T + t) * Hq + sg.h * G + g) * kD + k8 * 8);
+              q + ((size_t)(sg.b * T_all + t0 + t) * Hq + sg.h * G + g) * kD + k8 * 8);
           const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
           uint32_t o[4], ol[4];
 #pragma unroll
@@ -441,8 +445,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
       fence_proxy_async_smem();
       if (smx) {
         if (tid < N) {
-          // Keys visible to score row n (query t = n / G at kv_len - T + t).
-          sh.nvis_s[tid] = tid < R ? sg.kv_len - T + tid / G + 1 : 0;
+          // Keys visible to score row n (query t0 + n / G of the step, at
+          // position kv_len - T_all + t0 + n / G).
+          sh.nvis_s[tid] = tid < R ? sg.kv_len - T_all + t0 + tid / G + 1 : 0;
           sh.m_s[tid] = -INFINITY;
         }
 #pragma unroll
@@ -592,7 +597,7 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
           wait_bar(&sh.sready[uc & 1], (uc >> 1) & 1, sh.flags, err);
           tc_fence_after();
           const int pos = tok0 + 32 * lq + lane;
-          const bool vis_all = tok0 + kUnitTokens <= sg.kv_len - T + 1;
+          const bool vis_all = tok0 + kUnitTokens <= sg.kv_len - T_all + t0 + 1;
           const uint32_t sslot = tl + C::kColS + (uc & 1) * N;
           uint32_t *my_mask = sh.masks + ((uc & 1) * kSoftmaxWarps + lq) * 4;
           // Scores of one 16-row chunk, masked: invisible keys and padding
@@ -792,8 +797,9 @@ decode_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int Hk
             const int n = cb + j8 * 8 + j;
             if (n < R) {
               const float lv = sh.alpha_s[n];
-              ws_o[(slot * R + n) * kD + d] = lv > 0.f ? __uint_as_float(o[j]) / lv : 0.f;
-              if (d == 0) ws_lse[slot * R + n] = lv > 0.f ? sh.m_s[n] + log2f(lv) : -INFINITY;
+              ws_o[(slot * R_all + t0 * G + n) * kD + d] = lv > 0.f ? __uint_as_float(o[j]) / lv : 0.f;
+              if (d == 0)
+                ws_lse[slot * R_all + t0 * G + n] = lv > 0.f ? sh.m_s[n] + log2f(lv) : -INFINITY;
             }
           }
         }
@@ -829,25 +835,27 @@ EncodeTiledFn encode_fn() {
 
 template <int N>
 cudaError_t launch_n(const CUtensorMap &map, const nvkv_cache &c, const nvkv_seqs &s,
-                     const void *q, int T, int Hq, float qscale, int S, float *ws_o,
-                     float *ws_lse, cudaStream_t stream) {
+                     const void *q, int T, int t0, int T_all, int Hq, float qscale, int S,
+                     float *ws_o, float *ws_lse, cudaStream_t stream) {
   const int smem = Cfg<N>::kSmemBytes;
   cudaError_t e = cudaFuncSetAttribute(decode_tc_kernel<N>,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
   decode_tc_kernel<N><<<S, kThreads, smem, stream>>>(
       map, c.num_pages, c.num_kv_heads, s.page_table, s.max_pages_per_seq, s.kv_lens, s.batch,
-      s.max_kv_len, static_cast<const __nv_bfloat16 *>(q), T, Hq, qscale, S, ws_o, ws_lse,
-      s.err_word);
+      s.max_kv_len, static_cast<const __nv_bfloat16 *>(q), T, t0, T_all, Hq, qscale, S, ws_o,
+      ws_lse, s.err_word);
   return cudaGetLastError();
 }
 
 }  // namespace
 
-// True when the tensor-core decode kernel takes this shape.
+// True when the tensor-core decode kernel takes this shape: head_dim 256
+// and a GQA group of at most 48 query heads.  More than 48 query rows per
+// (sequence, kv-head) run as several launches over chunks of queries.
 bool decode_tc_supported(const nvkv_cache &c, int T, int Hq) {
-  const int R = T * (Hq / c.num_kv_heads);
-  return c.head_dim == kD && R >= 1 && R <= 48 && encode_fn() != nullptr;
+  const int G = Hq / c.num_kv_heads;
+  return c.head_dim == kD && T >= 1 && G >= 1 && G <= 48 && encode_fn() != nullptr;
 }
 
 // The pool as a 2-D byte tensor of 128-byte rows; one 36-row box is one
@@ -870,11 +878,25 @@ cudaError_t launch_decode_tc(const nvkv_cache &c, const nvkv_seqs &s, const void
                              cudaStream_t stream) {
   CUtensorMap map;
   if (!make_pool_tmap(c, &map)) return cudaErrorNotSupported;
-  const int R = T * (Hq / c.num_kv_heads);
+  const int G = Hq / c.num_kv_heads;
   const float qscale = sm_scale * 1.4426950408889634f;
-  if (R <= 16) return launch_n<16>(map, c, s, q, T, Hq, qscale, S, ws_o, ws_lse, stream);
-  if (R <= 32) return launch_n<32>(map, c, s, q, T, Hq, qscale, S, ws_o, ws_lse, stream);
-  return launch_n<48>(map, c, s, q, T, Hq, qscale, S, ws_o, ws_lse, stream);
+  // Queries in chunks of at most 48 rows: each launch reads the whole KV
+  // of the step and writes its rows of the shared workspace layout (the
+  // same split plan, so nvkv_combine merges them as one launch's).
+  const int Tc = 48 / G;
+  for (int t0 = 0; t0 < T; t0 += Tc) {
+    const int Tn = T - t0 < Tc ? T - t0 : Tc;
+    const int R = Tn * G;
+    cudaError_t e;
+    if (R <= 16)
+      e = launch_n<16>(map, c, s, q, Tn, t0, T, Hq, qscale, S, ws_o, ws_lse, stream);
+    else if (R <= 32)
+      e = launch_n<32>(map, c, s, q, Tn, t0, T, Hq, qscale, S, ws_o, ws_lse, stream);
+    else
+      e = launch_n<48>(map, c, s, q, Tn, t0, T, Hq, qscale, S, ws_o, ws_lse, stream);
+    if (e != cudaSuccess) return e;
+  }
+  return cudaSuccess;
 }
 
 }  // namespace nvkv
