@@ -671,8 +671,8 @@ def main():
         except Exception as exc:  # a failure here must not cost the lines above
             graph = {"error": repr(exc)[:300]}
 
-    # ---- the same decode step over a K8V4 cache (E4M3 K rows, NVFP4 V) on
-    # the CUDA-core kernels, on its own 3 x 60k context ----
+    # ---- the same decode step over a K8V4 cache (E4M3 K rows, NVFP4 V), on
+    # its own 3 x 60k context ----
     k8 = None
     if not args.no_k8v4:
         try:
@@ -699,11 +699,13 @@ def main():
             # K 1 byte per element + an fp32 scale per row, V 4.5 bits per element
             kvb = sum(int(c) + 1 for c in kw.ctx) * kw.num_kv_heads * (
                 kw.head_dim + 4 + kw.head_dim * 9 // 16)
-            k8 = {"workload": kw.name + "_k8v4", "kernel": "decode_simt (CUDA cores)",
+            k8 = {"workload": kw.name + "_k8v4",
+                  "kernel": nv.nvkv_decode_kernel_name(kdw.cache, kw.T, kw.num_q_heads),
                   "kv_bytes_per_step": kvb, "step_ms": step_ms,
                   "step_gbs": kvb / (step_ms * 1e-3) / 1e9, "attend_ms": attend_ms,
                   "attend_gbs": kvb / (attend_ms * 1e-3) / 1e9,
                   "attend_frac": kvb / (attend_ms * 1e-3) / 1e9 / peak,
+                  "l2": f"KV {kvb / 1e6:.0f} MB per step, L2 {l2_bytes / 1e6:.0f} MB",
                   "device_errors": kdw.err_bits()}
             del kdw
         except Exception as exc:  # a failure here must not cost the lines above

@@ -309,7 +309,15 @@ nvkv_status nvkv_pages_restore(const nvkv_cache *cache, const int32_t *page_ids,
  *   nvkv_pages_spill_k8v4, nvkv_pages_restore_k8v4 ~ nvkv_pages_spill,
  *                            nvkv_pages_restore, with arena slots of
  *                            nvkv_k8v4_page_bytes() bytes
- * The attention calls run on CUDA cores (one warp per query row).
+ * nvkv_decode_attn_k8v4 runs the decode_qk4 pipeline over this layout for
+ * head_dim 256 and T*Hq/Hkv <= 6: the scores on the E4M3 tensor-core MMA
+ * (kind::f8f6f4) straight from the cached K bytes, q * sm_scale * log2(e)
+ * entering as 8 stacked E4M3 terms after a power-of-two prescale of each
+ * row (term l weighted 2^-4l; remainder below 2^-28 of the row maximum),
+ * times each token's fp32 row scale in fp32; weights and value sum as for
+ * the NVFP4 cache.  Other decode shapes and the prefill run on CUDA cores
+ * (one warp per query row).  nvkv_decode_kernel_name_k8v4 names the kernel
+ * ("decode_qk4_k8v4" or "decode_simt"; "none" on invalid arguments).
  * nvkv_k8v4_page_bytes returns 0 for non-positive arguments. */
 size_t nvkv_k8v4_page_bytes(int32_t num_kv_heads, int32_t head_dim);
 nvkv_status nvkv_append_k8v4(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *k_new,
@@ -319,6 +327,8 @@ nvkv_status nvkv_decode_attn_k8v4(const nvkv_cache *cache, const nvkv_seqs *seqs
                                   int32_t T, int32_t num_q_heads, float sm_scale,
                                   int32_t num_splits, void *workspace, size_t workspace_bytes,
                                   nvkv_stream_t stream);
+const char *nvkv_decode_kernel_name_k8v4(const nvkv_cache *cache, int32_t T,
+                                         int32_t num_q_heads);
 nvkv_status nvkv_prefill_attn_k8v4(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *q,
                                    const int32_t *cu_q, int32_t total_q, int32_t max_q,
                                    int32_t num_q_heads, float sm_scale, void *out,

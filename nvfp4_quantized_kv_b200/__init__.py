@@ -74,6 +74,7 @@ def library():
             "nvkv_append": (ctypes.c_int, [cp, sp, vp, vp, vp, i32, i32, vp]),
             "nvkv_decode_attn": (ctypes.c_int, [cp, sp, vp, i32, i32, f32, i32, vp, sz, vp]),
             "nvkv_decode_kernel_name": (ctypes.c_char_p, [cp, i32, i32]),
+            "nvkv_decode_kernel_name_k8v4": (ctypes.c_char_p, [cp, i32, i32]),
             "nvkv_combine": (ctypes.c_int, [sp, vp, i32, i32, i32, i32, i32, vp, vp]),
             "nvkv_prefill_attn": (ctypes.c_int, [cp, sp, vp, vp, i32, i32, i32, f32, vp, vp]),
             "nvkv_decode_static_scratch_bytes": (sz, []),
@@ -257,11 +258,14 @@ def nvkv_decode_attn(cache: Cache, seqs: Seqs, q: torch.Tensor, T: int, num_q_he
 
 
 def nvkv_decode_kernel_name(cache: Cache, T: int, num_q_heads: int) -> str:
-    """The decode kernel nvkv_decode_attn launches for this cache and step
-    shape: "decode_qk4", "decode_tc" or "decode_simt"."""
-    _fmt(cache, "nvfp4", "nvkv_decode_kernel_name")
-    return library().nvkv_decode_kernel_name(ctypes.byref(cache._c), int(T),
-                                             int(num_q_heads)).decode()
+    """The decode kernel the decode call of this cache's format launches for
+    this step shape: "decode_qk4", "decode_tc" or "decode_simt" (NVFP4);
+    "decode_qk4_k8v4" or "decode_simt" (K8V4)."""
+    if cache.kv_format == "k8v4":
+        fn = library().nvkv_decode_kernel_name_k8v4
+    else:
+        fn = library().nvkv_decode_kernel_name
+    return fn(ctypes.byref(cache._c), int(T), int(num_q_heads)).decode()
 
 
 def nvkv_combine(seqs: Seqs, workspace: torch.Tensor, T: int, num_q_heads: int,

@@ -20,6 +20,8 @@ bool decode_tc_supported(const nvkv_cache &, int, int);
 bool decode_qk4_supported(const nvkv_cache &, int, int);
 cudaError_t launch_decode_qk4(const nvkv_cache &, const nvkv_seqs &, const void *, int, int, float,
                               int, float *, float *, cudaStream_t);
+cudaError_t launch_decode_qk4_k8v4(const nvkv_cache &, const nvkv_seqs &, const void *, int, int,
+                                   float, int, float *, float *, cudaStream_t);
 cudaError_t launch_decode_tc(const nvkv_cache &, const nvkv_seqs &, const void *, int, int, float,
                              int, float *, float *, cudaStream_t);
 bool prefill_tc_supported(const nvkv_cache &);
@@ -366,8 +368,21 @@ nvkv_status nvkv_decode_attn_k8v4(const nvkv_cache *cache, const nvkv_seqs *seqs
   const nvkv_status st = check_decode(cache, seqs, q, T, num_q_heads, sm_scale, num_splits,
                                       workspace, workspace_bytes, a);
   if (st != NVKV_OK) return st;
+  cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
+  if (!force_simt() && decode_qk4_supported(*cache, T, num_q_heads))
+    return cuda_status(launch_decode_qk4_k8v4(*cache, *seqs, q, T, num_q_heads, sm_scale, a.S,
+                                              a.ws_o, a.ws_lse, st_));
   return cuda_status(launch_decode_simt(*cache, *seqs, q, T, num_q_heads, sm_scale, a.S, a.ws_o,
-                                        a.ws_lse, reinterpret_cast<cudaStream_t>(stream), true));
+                                        a.ws_lse, st_, true));
+}
+
+const char *nvkv_decode_kernel_name_k8v4(const nvkv_cache *cache, int32_t T,
+                                         int32_t num_q_heads) {
+  if (!cache || cache->num_kv_heads <= 0 || T <= 0 || num_q_heads <= 0 ||
+      num_q_heads % cache->num_kv_heads != 0)
+    return "none";
+  if (!force_simt() && decode_qk4_supported(*cache, T, num_q_heads)) return "decode_qk4_k8v4";
+  return "decode_simt";
 }
 
 nvkv_status nvkv_prefill_attn_k8v4(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *q,

@@ -89,18 +89,21 @@ constexpr int kVRows = 18;               // V codes (16), V scales (2)
 constexpr int kKPageBytes = kKRows * 128;         // 2048
 constexpr int kVPageBytes = kVRows * 128;         // 2304
 constexpr int kKsPageBytes = kKsRows * 128;       // 256
-constexpr int kKTileBytes = kUnitPages * kKPageBytes;      // 16384
-constexpr int kStageBytes = kKTileBytes + kUnitPages * kVPageBytes;  // 34816
 constexpr int kVc = 0, kVs = 2048;       // V codes, V scales inside a page's V block
-constexpr int kStages = 5;
-constexpr int kKsSlots = 8;              // ring of the units' K scale bytes
 constexpr int kKsSlotBytes = kUnitPages * kKsPageBytes;    // 2048
+// K8V4 page block of one kv-head (head_dim 256): K codes [16][256] (4096 B),
+// K row scales [16] fp32 (64 B), then the V codes and scales as above.
+constexpr int kK8HeadBytes = 25 * kD + 64;   // 6464
+constexpr int kK8KsOff = 16 * kD;            // 4096
+constexpr int kK8VOff = kK8KsOff + 64;       // 4160
 
 constexpr int kRowsCap = 6;              // query rows per pair (T * G) this kernel takes
 constexpr int kTerms = 8;                // NVFP4 terms per query row
 constexpr int kNSMax = kRowsCap * kTerms;   // 48: largest N of the score MMA
 constexpr int kNP = 16;                  // N of the value MMA: the query rows, padded
 constexpr int kPSlots = 4;               // P ring depth
+constexpr int kPSlotBytes = 2 * 2048;    // rows 0..7, rows 8..15 (zero) x 128 tokens
+constexpr int kVscWarpBytes = kUnitPages * 2 * 8 * 4;   // 512
 constexpr int kVSlots = 3;               // V^T ring depth (Tensor Memory)
 
 constexpr int kDeqWarps = 8;             // warps 0..7
@@ -127,32 +130,48 @@ static_assert(kColV + kVSlots * 128 <= kColS && kColS + kNSMax <= kColO &&
                   kColSFB + 16 <= kTmemCols && kColSFA % 4 == 0 && kColSFB % 4 == 0,
               "tensor memory");
 
-// Shared memory (offsets from a 1024-byte aligned base).
-constexpr int kOffKs = kStages * kStageBytes;       // K scale ring [slot][page][token][16]
-constexpr int kOffQ = kOffKs + kKsSlots * kKsSlotBytes;  // query terms, kNSMax rows x 128 B, swizzled
-constexpr int kOffP = kOffQ + kNSMax * 128;         // P tiles [slot], MN-major f16
-constexpr int kPSlotBytes = 2 * 2048;               // rows 0..7, rows 8..15 (zero) x 128 tokens
-constexpr int kOffVsc = kOffP + kPSlots * kPSlotBytes;  // V scale pairs [warp][page][group][8]
-constexpr int kVscWarpBytes = kUnitPages * 2 * 8 * 4;   // 512
-constexpr int kOffSfb = kOffVsc + kDeqWarps * kVscWarpBytes;  // [kNSMax][16] term scale bytes
-constexpr int kOffFac = kOffSfb + kNSMax * 16;      // float [kRowsCap]: 2^-k of each row's terms
-constexpr int kOffRed = kOffFac + kNSMax * 4;       // float [quarter][kNP]
-constexpr int kOffMask = kOffRed + 4 * kNP * 4;     // u32 [parity][quarter]
-constexpr int kOffM = kOffMask + 2 * 4 * 4;         // float [kNP]
-constexpr int kOffAlpha = kOffM + kNP * 4;
-constexpr int kOffNvis = kOffAlpha + kNP * 4;
-constexpr int kOffFlags = kOffNvis + kNP * 4;       // int[4]: abort at [2]
-constexpr int kOffPages = kOffFlags + 16;           // int[stages][8]
-constexpr int kOffBars = kOffPages + kStages * kUnitPages * 4;
-constexpr int kNumBars = 2 * kStages + 2 * kKsSlots + 4 + 4 * kVSlots + 2 * kPSlots + 3;
-constexpr int kOffTmem = kOffBars + kNumBars * 8;
-constexpr int kSmemBytes = kOffTmem + 16 + 1024;    // + alignment slack
-static_assert(kSmemBytes <= 227 * 1024, "shared memory");
-static_assert(kOffQ % 1024 == 0 && kStageBytes % 1024 == 0 && kOffP % 128 == 0 &&
-                  kOffKs % 128 == 0 &&
-                  kOffVsc % 16 == 0 && kOffSfb % 16 == 0 && kOffPages % 16 == 0 &&
-                  kOffBars % 8 == 0,
-              "alignment");
+// Shared memory (offsets from a 1024-byte aligned base), per cache format.
+// NVFP4: a stage holds the unit's K code tile [128 tokens][128 B] and the 8
+// pages' V blocks; the K scale bytes go to their own ring.  K8V4: the K code
+// tile is two head_dim halves [2][128 tokens][128 B], then the V blocks, then
+// the 8 pages' K row scales ([8][128 B] slots, 16 fp32 used); no scale ring.
+template <bool K8>
+struct Fmt {
+  static constexpr int kKTileBytes = K8 ? 2 * kUnitPages * kKPageBytes : kUnitPages * kKPageBytes;
+  static constexpr int kVOff = kKTileBytes;                       // V blocks [page][2304]
+  static constexpr int kKsOff = kVOff + kUnitPages * kVPageBytes;  // K8: row scales [page][128 B]
+  static constexpr int kStageBytes = K8 ? 52224 : kKsOff;          // 1024-aligned
+  static constexpr int kStages = K8 ? 3 : 5;
+  static constexpr int kKsSlots = K8 ? 0 : 8;                      // K scale ring (NVFP4)
+  static constexpr int kQBytes = (K8 ? 2 : 1) * kNSMax * 128;      // query terms, swizzled
+  static constexpr int kOffKs = kStages * kStageBytes;
+  static constexpr int kOffQ = kOffKs + kKsSlots * kKsSlotBytes;
+  static constexpr int kOffP = kOffQ + kQBytes;                    // P tiles [slot], MN-major f16
+  static constexpr int kOffVsc = kOffP + kPSlots * kPSlotBytes;    // V scale pairs [warp][page][group][8]
+  static constexpr int kOffSfb = kOffVsc + kDeqWarps * kVscWarpBytes;  // [kNSMax][16] term scales
+  static constexpr int kOffFac = kOffSfb + kNSMax * 16;            // float: 2^-k of each row
+  static constexpr int kOffRed = kOffFac + kNSMax * 4;             // float [quarter][kNP]
+  static constexpr int kOffMask = kOffRed + 4 * kNP * 4;           // u32 [parity][quarter]
+  static constexpr int kOffM = kOffMask + 2 * 4 * 4;               // float [kNP]
+  static constexpr int kOffAlpha = kOffM + kNP * 4;
+  static constexpr int kOffNvis = kOffAlpha + kNP * 4;
+  static constexpr int kOffFlags = kOffNvis + kNP * 4;             // int[4]: abort at [2]
+  static constexpr int kOffPages = kOffFlags + 16;                 // int[stages][8]
+  static constexpr int kOffBars = kOffPages + kStages * kUnitPages * 4;
+  static constexpr int kNumBars = 2 * kStages + 2 * kKsSlots + 4 + 4 * kVSlots + 2 * kPSlots + 3;
+  static constexpr int kOffTmem = kOffBars + kNumBars * 8;
+  static constexpr int kSmemBytes = kOffTmem + 16 + 1024;          // + alignment slack
+  // (TMA destinations are 128-byte aligned: each page's 64 bytes of K row
+  // scales get a 128-byte slot)
+  static_assert(kKsOff + (K8 ? kUnitPages * 128 : 0) <= kStageBytes && kStageBytes % 1024 == 0 &&
+                    kKsOff % 128 == 0,
+                "stage");
+  static_assert(kSmemBytes <= 227 * 1024, "shared memory");
+  static_assert(kOffQ % 1024 == 0 && kOffP % 128 == 0 && kOffKs % 128 == 0 &&
+                    kOffVsc % 16 == 0 && kOffSfb % 16 == 0 && kOffPages % 16 == 0 &&
+                    kOffBars % 8 == 0,
+                "alignment");
+};
 
 struct Shared {
   uint8_t *stages, *ks, *qtile, *ptile, *sfb;
@@ -245,7 +264,12 @@ __device__ __forceinline__ uint32_t mul_f16x2(uint32_t a, uint32_t b) {
   return d;
 }
 
-template <int RM>
+// K8 selects the cache format: false = NVFP4 K (tmap_k: 16-row SW128 boxes of
+// K codes; tmap_ks: 2-row boxes of K scales; tmap_v: 18-row boxes of V codes
+// and scales, all over 128-byte rows of the pool), true = K8V4 (tmap_k: 3-D
+// [block][token][256 B], 128-byte SW128 boxes of 16 tokens, one per head_dim
+// half; tmap_ks: [block][64 B] row scales; tmap_v: [block][18][128 B]).
+template <int RM, bool K8>
 __global__ void __launch_bounds__(kThreads, 1)
 decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
                   const __grid_constant__ CUtensorMap tmap_ks,
@@ -258,6 +282,14 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
   // zero); the score MMA has N = RM * kTerms columns.
   static_assert(RM % 2 == 0 && RM >= 2 && RM <= kRowsCap, "rows");
   constexpr int NS = RM * kTerms;
+  using F = Fmt<K8>;
+  constexpr int kStages = F::kStages, kStageBytes = F::kStageBytes, kKTileBytes = F::kKTileBytes,
+                kKsSlots = F::kKsSlots;
+  constexpr int kOffKs = F::kOffKs, kOffQ = F::kOffQ, kOffP = F::kOffP, kOffVsc = F::kOffVsc,
+                kOffSfb = F::kOffSfb, kOffFac = F::kOffFac, kOffRed = F::kOffRed,
+                kOffMask = F::kOffMask, kOffM = F::kOffM, kOffAlpha = F::kOffAlpha,
+                kOffNvis = F::kOffNvis, kOffFlags = F::kOffFlags, kOffPages = F::kOffPages,
+                kOffBars = F::kOffBars, kOffTmem = F::kOffTmem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
                                               ~uintptr_t(1023));
@@ -300,7 +332,9 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
   if (threadIdx.x == 0) {
     for (int i = 0; i < kStages; ++i) {
       mbar_init(&sh.full[i], 1);
-      mbar_init(&sh.empty[i], 1 + kDeqWarps);  // the score MMAs' commit, the V^T writers
+      // the score MMAs' commit, the V^T writers (and, for K8V4, the softmax
+      // warps, which read their tokens' K row scales from the stage)
+      mbar_init(&sh.empty[i], 1 + kDeqWarps + (K8 ? kSmxWarps : 0));
     }
     for (int i = 0; i < kKsSlots; ++i) {
       mbar_init(&sh.ks_full[i], 1);
@@ -343,13 +377,15 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
   const int64_t u1 = U > 0 ? range_begin(c + 1, U, S) : 0;
   const uint32_t n_units = (uint32_t)(u1 - u0);
 
-  if (warp == kProducerWarp || warp == kKsProducerWarp) {
+  if (K8 && warp == kKsProducerWarp) {
+    // K8V4 has no K scale ring: this warp has nothing to do.
+  } else if (warp == kProducerWarp || warp == kKsProducerWarp) {
     // ------------------------------------------------------------------ TMA
     // Lane p < 8 owns page p of a unit; the page ids of unit u+1 are loaded
     // while unit u's copies are issued.  One warp fills the stage ring (K
-    // codes into the unit's contiguous K tile, V codes and scales), the
-    // other the deeper ring of K scale bytes, which the scale-factor
-    // writers read one unit ahead of the rest.
+    // codes into the unit's contiguous K tile, V codes and scales, and for
+    // K8V4 the K row scales), the other (NVFP4) the deeper ring of K scale
+    // bytes, which the scale-factor writers read one unit ahead of the rest.
     const bool big = warp == kProducerWarp;
     const int ring = big ? kStages : kKsSlots;
     uint64_t *fullb = big ? sh.full : sh.ks_full;
@@ -387,11 +423,21 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
       const bool mine = lane < kUnitPages && cur >= 0;
       if (big && lane < kUnitPages) sh.pages[slot * kUnitPages + lane] = cur;
       const uint32_t bytes = __popc(__ballot_sync(0xffffffffu, mine)) *
-                             (big ? kKPageBytes + kVPageBytes : kKsPageBytes);
+                             (!big ? kKsPageBytes : K8 ? kK8HeadBytes : kKPageBytes + kVPageBytes);
       __syncwarp();
       if (lane == 0) mbar_arrive_expect_tx(&fullb[slot], bytes);
       __syncwarp();
-      if (mine) {
+      if (mine && K8) {
+        // K halves [token][128 B] (x = 0 / 128 of the 256-byte rows), the V
+        // block and the 16 K row scales of this page's kv-head block
+        const int blk = cur * Hkv + sg.h;
+        uint8_t *st = sh.stages + slot * kStageBytes;
+        tma_load_3d(st + lane * kKPageBytes, &tmap_k, 0, 0, blk, &fullb[slot]);
+        tma_load_3d(st + kUnitPages * kKPageBytes + lane * kKPageBytes, &tmap_k, 128, 0, blk,
+                    &fullb[slot]);
+        tma_load_3d(st + F::kVOff + lane * kVPageBytes, &tmap_v, 0, 0, blk, &fullb[slot]);
+        tma_load_2d(st + F::kKsOff + lane * 128, &tmap_ks, 0, blk, &fullb[slot]);
+      } else if (mine) {
         const int y = (cur * Hkv + sg.h) * kRowsPerHead;
         if (big) {
           uint8_t *st = sh.stages + slot * kStageBytes;
@@ -426,7 +472,9 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
       int64_t seg_end = segment_at(u0, u1, kv_lens, B, Hkv, max_kv_len, max_pages).seg_end;
       bool issued = false;
       if (warp == kMmaWarp) {
-        const uint32_t idesc_qk = idesc_nvf4(128, NS);
+        // NVFP4: E2M1 x E2M1 block-scaled; K8V4: E4M3 x E4M3 (kind::f8f6f4,
+        // format 0 = E4M3), the same descriptor layout as the f16 kind.
+        const uint32_t idesc_qk = K8 ? idesc_f16_f32(128, NS, false, false) : idesc_nvf4(128, NS);
         const uint32_t qb = smem_u32(sh.qtile);
         const uint32_t kt0 = smem_u32(sh.stages);
         uint32_t seg_idx = 0;
@@ -440,17 +488,28 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
           if (opens) wait_bar(sh.qready, seg_idx & 1, sh.flags, err);
           const int stage = qk % kStages;
           wait_bar(&sh.full[stage], (qk / kStages) & 1, sh.flags, err);
-          wait_bar(&sh.sfa_ready[qk & 1], (qk >> 1) & 1, sh.flags, err);
+          if (!K8) wait_bar(&sh.sfa_ready[qk & 1], (qk >> 1) & 1, sh.flags, err);
           // S^T was read by the softmax of unit qk-1
           if (qk > 0) wait_bar(sh.sfree, (qk - 1) & 1, sh.flags, err);
           tc_fence_after();
           const uint32_t sslot = tmem + kColS;
           const uint32_t sfa = tmem + kColSFA + (qk & 1) * 16;
           const uint32_t kt = kt0 + stage * kStageBytes;
+          if constexpr (K8) {
+            // two head_dim halves of 128 bytes, 4 K steps of 32 elements each
 #pragma unroll
-          for (int ks = 0; ks < 4; ++ks)
-            mma_nvf4_ss(sslot, smem_desc_sw128(kt + 32 * ks), smem_desc_sw128(qb + 32 * ks),
-                        idesc_qk, ks > 0, sfa + 4 * ks, tmem + kColSFB + 4 * ks);
+            for (int hf = 0; hf < 2; ++hf)
+#pragma unroll
+              for (int ks = 0; ks < 4; ++ks)
+                mma_f8_ss(sslot, smem_desc_sw128(kt + hf * kUnitPages * kKPageBytes + 32 * ks),
+                          smem_desc_sw128(qb + hf * kNSMax * 128 + 32 * ks), idesc_qk,
+                          (hf | ks) > 0);
+          } else {
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks)
+              mma_nvf4_ss(sslot, smem_desc_sw128(kt + 32 * ks), smem_desc_sw128(qb + 32 * ks),
+                          idesc_qk, ks > 0, sfa + 4 * ks, tmem + kColSFB + 4 * ks);
+          }
           mma_commit(sh.sready);
           mma_commit(&sh.empty[stage]);  // the K tile has been read
           issued = true;
@@ -511,9 +570,10 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
     // Column 4*ks + m1, lane l: the 4 scale bytes of token 32*m1 + l for
     // head_dim elements 64*ks .. 64*ks+63.
     auto write_sfa = [&](uint32_t un) {
-      const int ksl = un % kKsSlots;
+      constexpr int kRing = kKsSlots > 0 ? kKsSlots : 1;  // (NVFP4 only)
+      const int ksl = un % kRing;
       const uint8_t *kb = sh.ks + ksl * kKsSlotBytes;
-      wait_bar(&sh.ks_full[ksl], (un / kKsSlots) & 1, sh.flags, err);
+      wait_bar(&sh.ks_full[ksl], (un / kRing) & 1, sh.flags, err);
       tc_fence_after();
       uint32_t w[16];
 #pragma unroll
@@ -533,7 +593,7 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
         mbar_arrive(&sh.ks_empty[ksl]);
       }
     };
-    if (smx && n_units > 0) write_sfa(0);
+    if (!K8 && smx && n_units > 0) write_sfa(0);
 
     uint32_t uc = 0;
     uint32_t seg_idx = 0;
@@ -585,7 +645,9 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
           // A row whose largest element is below the smallest normal float
           // (2^-126) is taken as zero: its scores would be below 2^-110.
           const int eb = (int)((__float_as_uint(a) >> 23) & 0xffu);  // biased exponent
-          const int k = 135 - eb;  // a in [2^(eb-127), 2^(eb-126)): a * 2^k in [256, 512)
+          // a in [2^(eb-127), 2^(eb-126)): a * 2^k in [256, 512) (NVFP4), in
+          // [128, 256) (K8V4, under the E4M3 maximum 448)
+          const int k = (K8 ? 134 : 135) - eb;
           if (eb > 0) {
 #pragma unroll
             for (int i = 0; i < 8; ++i) y[i] = scale_pow2(y[i], k);
@@ -593,6 +655,32 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
 #pragma unroll
             for (int i = 0; i < 8; ++i) y[i] = 0.f;
           }
+          if constexpr (K8) {
+            // Term l: E4M3 codes of y * 2^(4l), its value subtracted exactly.
+            // E4M3 rounding leaves at most 2^-4 of an element (or 2^-10 of
+            // the term's unit in the subnormal range), so y * 2^(4(l+1))
+            // stays below 256 and no term saturates; the MMA's column 8r + l
+            // carries weight 2^-4l, recombined in the softmax.
+#pragma unroll 1
+            for (int l = 0; l < kTerms; ++l) {
+              const int n = r * kTerms + l;
+              const float up = pow2f(4 * l), down = pow2f(-4 * l);
+              uint32_t pr[4];
+#pragma unroll
+              for (int i = 0; i < 4; ++i) {
+                pr[i] = f32x2_to_e4m3x2(y[2 * i] * up, y[2 * i + 1] * up);
+                const float2 v = f16x2_to_float2(e4m3x2_to_f16x2(pr[i]));
+                y[2 * i] -= v.x * down;  // exact
+                y[2 * i + 1] -= v.y * down;
+              }
+              // bytes 8*lane .. 8*lane+7 of the row: head_dim half lane/16,
+              // 128-byte swizzle
+              const int c16 = (lane & 15) >> 1;
+              *reinterpret_cast<uint2 *>(sh.qtile + (lane >> 4) * (kNSMax * 128) + n * 128 +
+                                         ((c16 ^ (n & 7)) << 4) + (lane & 1) * 8) =
+                  make_uint2(pr[0] | (pr[1] << 16), pr[2] | (pr[3] << 16));
+            }
+          } else {
 #pragma unroll 1
           for (int l = 0; l < kTerms; ++l) {
             const int n = r * kTerms + l;
@@ -620,6 +708,7 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
                                           (lane & 3) * 4) = codes;
             if ((lane & 1) == 0) sh.sfb[n * 16 + (lane >> 1)] = (uint8_t)sb;
           }
+          }
           if (lane == 0) sh.fac[r] = eb > 0 ? scale_pow2(1.f, -k) : 0.f;
         }
         fence_proxy_async_smem();
@@ -628,8 +717,11 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
         for (int i = 0; i < RM; ++i) facr[i] = sh.fac[i];
         // Scale factors of the terms into Tensor Memory (each lane quarter
         // holds all rows): column 4*ks + n1, lane l -> row 32*n1 + l (every
-        // K step's block starts on a multiple of 4 columns).
-        {
+        // K step's block starts on a multiple of 4 columns).  K8V4 has none.
+        if (K8) {
+          __syncwarp();
+          if (lane == 0) mbar_arrive(sh.qready);
+        } else {
           uint32_t w[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) w[i] = 0u;
@@ -720,7 +812,7 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
           // ---- softmax on S^T: thread = token tok0 + 32*lq + lane.
           // First the K scale factors of the next unit, while the scores of
           // this one are computed.
-          if (uc + 1 < n_units) write_sfa(uc + 1);
+          if (!K8 && uc + 1 < n_units) write_sfa(uc + 1);
           const int pos = tok0 + 32 * lq + lane;
           wait_bar(sh.sready, uc & 1, sh.flags, err);
           tc_fence_after();
@@ -737,16 +829,38 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(sh.sfree);  // S^T read
+            // K8V4: this token's K row scale, from the stage (then this
+            // warp's reads of the stage are done)
+            float ksc = 1.f;
+            if constexpr (K8) {
+              wait_bar(&sh.full[stage], (uc / kStages) & 1, sh.flags, err);
+              const int j = 32 * lq + lane;
+              ksc = *reinterpret_cast<const float *>(sh.stages + stage * kStageBytes + F::kKsOff +
+                                                     (j >> 4) * 128 + (j & 15) * 4);
+              __syncwarp();
+              if (lane == 0) mbar_arrive(&sh.empty[stage]);
+            }
             const bool vis_all = tok0 + kUnitTokens <= sg.kv_len - T + 1;
 #pragma unroll
             for (int j = 0; j < RM; ++j) {
               const uint32_t *c8 = rr + j * kTerms;
-              const float2 a0 = add_f32x2(make_float2(__uint_as_float(c8[0]), __uint_as_float(c8[1])),
-                                          make_float2(__uint_as_float(c8[2]), __uint_as_float(c8[3])));
-              const float2 a1 = add_f32x2(make_float2(__uint_as_float(c8[4]), __uint_as_float(c8[5])),
-                                          make_float2(__uint_as_float(c8[6]), __uint_as_float(c8[7])));
-              const float2 a2 = add_f32x2(a0, a1);
-              const float sc = (a2.x + a2.y) * facr[j];
+              float sc;
+              if constexpr (K8) {
+                // sum_l 2^-4l * column l, by Horner
+                float acc = __uint_as_float(c8[kTerms - 1]);
+#pragma unroll
+                for (int l = kTerms - 2; l >= 0; --l) acc = fmaf(acc, 0.0625f, __uint_as_float(c8[l]));
+                sc = acc * facr[j] * ksc;
+              } else {
+                const float2 a0 = add_f32x2(
+                    make_float2(__uint_as_float(c8[0]), __uint_as_float(c8[1])),
+                    make_float2(__uint_as_float(c8[2]), __uint_as_float(c8[3])));
+                const float2 a1 = add_f32x2(
+                    make_float2(__uint_as_float(c8[4]), __uint_as_float(c8[5])),
+                    make_float2(__uint_as_float(c8[6]), __uint_as_float(c8[7])));
+                const float2 a2 = add_f32x2(a0, a1);
+                sc = (a2.x + a2.y) * facr[j];
+              }
               const int nv = vis_all ? (j < R ? 0x7fffffff : 0) : sh.nvis_s[j];
               x[j] = pos < nv ? sc : -INFINITY;
             }
@@ -940,10 +1054,65 @@ bool make_map(const nvkv_cache &c, int rows, CUtensorMapSwizzle swz, CUtensorMap
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// K8V4 pool maps (head_dim 256): the pool as [block][...] with a block stride
+// of 6464 bytes (block = page * Hkv + h).  K: [block][16 tokens][256 B],
+// boxes of 128 B x 16 tokens, 128-byte swizzle (one box per head_dim half);
+// K row scales: [block][64 B] from byte 4096; V codes and scales:
+// [block][18][128 B] from byte 4160.
+bool make_k8_maps(const nvkv_cache &c, CUtensorMap *mk, CUtensorMap *mks, CUtensorMap *mv) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  const cuuint64_t nblk = (cuuint64_t)c.num_pages * c.num_kv_heads;
+  const cuuint32_t e1[3] = {1, 1, 1};
+  uint8_t *pool = static_cast<uint8_t *>(c.pool);
+  const cuuint64_t kd[3] = {256, 16, nblk}, ks[2] = {256, kK8HeadBytes};
+  const cuuint32_t kb[3] = {128, 16, 1};
+  const cuuint64_t sd[2] = {64, nblk}, ss[1] = {kK8HeadBytes};
+  const cuuint32_t sb[2] = {64, 1};
+  const cuuint64_t vd[3] = {128, kVRows, nblk}, vs[2] = {128, kK8HeadBytes};
+  const cuuint32_t vb[3] = {128, kVRows, 1};
+  return enc(mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, pool, kd, ks, kb, e1,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+             CUDA_SUCCESS &&
+         enc(mks, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, pool + kK8KsOff, sd, ss, sb, e1,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+             CUDA_SUCCESS &&
+         enc(mv, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, pool + kK8VOff, vd, vs, vb, e1,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) ==
+             CUDA_SUCCESS;
+}
+
+template <bool K8>
+cudaError_t launch_fmt(const nvkv_cache &c, const nvkv_seqs &s, const void *q, int T, int Hq,
+                       float sm_scale, int S, float *ws_o, float *ws_lse, cudaStream_t stream) {
+  CUtensorMap map_k, map_ks, map_v;
+  const bool ok = K8 ? make_k8_maps(c, &map_k, &map_ks, &map_v)
+                     : make_map(c, kKRows, CU_TENSOR_MAP_SWIZZLE_128B, &map_k) &&
+                           make_map(c, kKsRows, CU_TENSOR_MAP_SWIZZLE_NONE, &map_ks) &&
+                           make_map(c, kVRows, CU_TENSOR_MAP_SWIZZLE_NONE, &map_v);
+  if (!ok) return cudaErrorNotSupported;
+  const float qscale = sm_scale * 1.4426950408889634f;
+  const int R = T * (Hq / c.num_kv_heads);
+  auto kernel = R <= 2 ? decode_qk4_kernel<2, K8> : R <= 4 ? decode_qk4_kernel<4, K8>
+                                                             : decode_qk4_kernel<6, K8>;
+  const int smem = Fmt<K8>::kSmemBytes;
+  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  kernel<<<S, kThreads, smem, stream>>>(
+      map_k, map_ks, map_v, c.num_pages, c.num_kv_heads, s.page_table, s.max_pages_per_seq,
+      s.kv_lens, s.batch, s.max_kv_len, static_cast<const __nv_bfloat16 *>(q), T, Hq, qscale, S,
+      ws_o, ws_lse, s.err_word);
+  return cudaGetLastError();
+}
+
 }  // namespace
 
 // True when this kernel takes the shape: head_dim 256 and at most 6 query
-// rows (T * Hq/Hkv) per (sequence, kv-head).
+// rows (T * Hq/Hkv) per (sequence, kv-head).  The same holds for both cache
+// formats.
 bool decode_qk4_supported(const nvkv_cache &c, int T, int Hq) {
   const int R = T * (Hq / c.num_kv_heads);
   return c.head_dim == kD && R >= 1 && R <= kRowsCap && encode_fn() != nullptr;
@@ -952,23 +1121,15 @@ bool decode_qk4_supported(const nvkv_cache &c, int T, int Hq) {
 cudaError_t launch_decode_qk4(const nvkv_cache &c, const nvkv_seqs &s, const void *q, int T,
                               int Hq, float sm_scale, int S, float *ws_o, float *ws_lse,
                               cudaStream_t stream) {
-  CUtensorMap map_k, map_ks, map_v;
-  if (!make_map(c, kKRows, CU_TENSOR_MAP_SWIZZLE_128B, &map_k) ||
-      !make_map(c, kKsRows, CU_TENSOR_MAP_SWIZZLE_NONE, &map_ks) ||
-      !make_map(c, kVRows, CU_TENSOR_MAP_SWIZZLE_NONE, &map_v))
-    return cudaErrorNotSupported;
-  const float qscale = sm_scale * 1.4426950408889634f;
-  const int R = T * (Hq / c.num_kv_heads);
-  auto kernel = R <= 2 ? decode_qk4_kernel<2> : R <= 4 ? decode_qk4_kernel<4>
-                                                         : decode_qk4_kernel<6>;
-  cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       kSmemBytes);
-  if (e != cudaSuccess) return e;
-  kernel<<<S, kThreads, kSmemBytes, stream>>>(
-      map_k, map_ks, map_v, c.num_pages, c.num_kv_heads, s.page_table, s.max_pages_per_seq, s.kv_lens,
-      s.batch, s.max_kv_len, static_cast<const __nv_bfloat16 *>(q), T, Hq, qscale, S, ws_o,
-      ws_lse, s.err_word);
-  return cudaGetLastError();
+  return launch_fmt<false>(c, s, q, T, Hq, sm_scale, S, ws_o, ws_lse, stream);
+}
+
+// The same kernel over a K8V4 cache (E4M3 K rows with an fp32 row scale,
+// NVFP4 V): the scores on kind::f8f6f4 from the cached E4M3 bytes.
+cudaError_t launch_decode_qk4_k8v4(const nvkv_cache &c, const nvkv_seqs &s, const void *q, int T,
+                                   int Hq, float sm_scale, int S, float *ws_o, float *ws_lse,
+                                   cudaStream_t stream) {
+  return launch_fmt<true>(c, s, q, T, Hq, sm_scale, S, ws_o, ws_lse, stream);
 }
 
 }  // namespace nvkv

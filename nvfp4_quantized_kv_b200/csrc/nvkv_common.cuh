@@ -143,6 +143,14 @@ __device__ __forceinline__ uint32_t e4m3x2_to_f16x2(uint32_t two_bytes) {
   return out;
 }
 
+// Two floats -> two E4M3 bytes (a in the low byte), rounded to nearest with
+// ties to even and saturated at 448 by the hardware conversion.
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float a, float b) {
+  uint16_t out;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %2, %1;" : "=h"(out) : "f"(a), "f"(b));
+  return out;
+}
+
 // Two floats -> one byte of E2M1 codes (a in the low nibble), rounded to
 // nearest with ties to even and saturated at 6 by the hardware conversion.
 __device__ __forceinline__ uint32_t f32x2_to_e2m1x2(float a, float b) {

@@ -153,14 +153,47 @@ DECODE = [
 ]
 
 
+def k8_kernel(d, hq, hkv, T):
+    """The kernel nvkv_decode_attn_k8v4 picks: the tensor-core pipeline for
+    head_dim 256 and at most 6 query rows per kv-head, else CUDA cores."""
+    return "decode_qk4_k8v4" if d == 256 and T * (hq // hkv) <= 6 else "decode_simt"
+
+
 @pytest.mark.parametrize("case", DECODE, ids=[c[0] for c in DECODE])
 @pytest.mark.parametrize("num_splits", [0, 3])
 def test_decode_k8v4_all_rows(case, num_splits):
     name, b, hq, hkv, d, T, ctx = case
     wl = W.small(name, b, hq, hkv, d, T, ctx, seed=zlib.crc32(name.encode()) % 1000)
     dw = run_step(wl, num_splits)
+    assert nv.nvkv_decode_kernel_name(dw.cache, T, hq) == k8_kernel(d, hq, hkv, T)
     rows = all_rows(wl)
     assert_close(gpu_rows(dw.out, wl, rows), oracle_outputs(wl, rows, k8=True), name)
+
+
+TC_CASES = [c for c in DECODE if k8_kernel(c[4], c[2], c[3], c[5]) == "decode_qk4_k8v4"]
+
+
+@pytest.mark.parametrize("case", TC_CASES, ids=[c[0] for c in TC_CASES])
+def test_decode_k8v4_cuda_core_kernel_on_the_tensor_core_shapes(case, monkeypatch):
+    """The shapes the tensor-core K8V4 decode takes, forced onto the
+    CUDA-core kernel: both within tolerance of the oracle."""
+    name, b, hq, hkv, d, T, ctx = case
+    monkeypatch.setenv("NVKV_DECODE_KERNEL", "simt")
+    wl = W.small(name, b, hq, hkv, d, T, ctx, seed=zlib.crc32(name.encode()) % 1000 + 1)
+    dw = run_step(wl)
+    assert nv.nvkv_decode_kernel_name(dw.cache, T, hq) == "decode_simt"
+    rows = all_rows(wl)
+    assert_close(gpu_rows(dw.out, wl, rows), oracle_outputs(wl, rows, k8=True), name + "/simt")
+
+
+def test_decode_k8v4_tensor_core_long_context_sampled():
+    """3 x 60000 cached tokens, T=1, on the tensor-core K8V4 decode: many
+    units per split, several segments per CTA; sampled rows vs the oracle."""
+    wl = W.long_context(T=1, ctx=(60000, 60000, 60000))
+    dw = run_step(wl)
+    assert nv.nvkv_decode_kernel_name(dw.cache, 1, wl.num_q_heads) == "decode_qk4_k8v4"
+    rows = sample_rows(wl, 12, seed=9)
+    assert_close(gpu_rows(dw.out, wl, rows), oracle_outputs(wl, rows, k8=True), wl.name + "/k8v4")
 
 
 def test_decode_k8v4_batch2_verify_config():
