@@ -64,9 +64,9 @@ DATASHEET_BF16_TFLOPS = 2250.0  # dense
 DECODE_CAPTURE = {
     "kernel": "decode_qk4",
     "source": "nvfp4_quantized_kv_b200/csrc/decode_qk4.cu",
-    "sha256": "902d501081dd4c3a0763e90bdc0f6130c35acfbf9aa28bac0d9b03d8158469a2",
-    "dram_bytes_read": 207611904,
-    "dram_bytes_write": 3841792,
+    "sha256": "a9499a735164b17eb255cc502a9c3c5d9d42af8d0f5ffd5534031fc4879e4a01",
+    "dram_bytes_read": 207596288,
+    "dram_bytes_write": 4512000,
     "kv_bytes": 207363456,
 }
 

@@ -273,3 +273,23 @@ def test_k8v4_spill_restore_and_attention_after_restore(kind):
     torch.cuda.synchronize()
     assert torch.equal(dw.out, before)
     assert int(err.item()) == 0
+
+
+@pytest.mark.parametrize("scale", [1e4, 1e-4])
+def test_decode_k8v4_query_scale(scale):
+    """q scaled by 1e4 and by 1e-4 on the tensor-core K8V4 decode: the query
+    terms take any finite scale (power-of-two row prescale), against the
+    oracle at the attention tolerance."""
+    wl = W.small("k8_qscale", 2, 24, 4, 256, 1, [3000, 1500], seed=78)
+    dw = DeviceWorkload(wl, num_splits=5, kv_format="k8v4")
+    dw.fill_context()
+    dw.load_step_inputs()
+    assert nv.nvkv_decode_kernel_name(dw.cache, 1, wl.num_q_heads) == "decode_qk4_k8v4"
+    q = to_bf16_bits(W.bf16_bits_to_f32(dw.q_np) * np.float32(scale))
+    dw.q = bf16_tensor(q, dw.device)
+    dw.step()
+    torch.cuda.synchronize()
+    assert dw.err_bits() == 0
+    rows = all_rows(wl)
+    assert_close(gpu_rows(dw.out, wl, rows), oracle_outputs(wl, rows, k8=True, q=q),
+                 f"{wl.name} q x {scale:g}")
