@@ -585,15 +585,21 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
         w[3 * 4 + m1] = v.w;
       }
       tmem_st16(tl + kColSFA + (un & 1) * 16, w);
+      __syncwarp();  // every lane's loads are done (the store consumed them)
+      if (lane == 0) mbar_arrive(&sh.ks_empty[ksl]);
+    };
+    // Publishes the scale factors of unit un once the warp's stores are
+    // complete (the caller waits for them, together with its own loads).
+    auto finish_sfa = [&](uint32_t un) {
+      if (lane == 0) mbar_arrive(&sh.sfa_ready[un & 1]);
+    };
+    if (!K8 && smx && n_units > 0) {
+      write_sfa(0);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) {
-        mbar_arrive(&sh.sfa_ready[un & 1]);
-        mbar_arrive(&sh.ks_empty[ksl]);
-      }
-    };
-    if (!K8 && smx && n_units > 0) write_sfa(0);
+      finish_sfa(0);
+    }
 
     uint32_t uc = 0;
     uint32_t seg_idx = 0;
@@ -812,7 +818,8 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
           // ---- softmax on S^T: thread = token tok0 + 32*lq + lane.
           // First the K scale factors of the next unit, while the scores of
           // this one are computed.
-          if (!K8 && uc + 1 < n_units) write_sfa(uc + 1);
+          const bool sfa_next = !K8 && uc + 1 < n_units;
+          if (sfa_next) write_sfa(uc + 1);
           const int pos = tok0 + 32 * lq + lane;
           wait_bar(sh.sready, uc & 1, sh.flags, err);
           tc_fence_after();
@@ -826,9 +833,11 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
             for (int i = 0; i < NS / 16; ++i)
               tmem_ld16(scol + 16 * i, *reinterpret_cast<uint32_t(*)[16]>(rr + 16 * i));
             tmem_wait_ld();
+            if (sfa_next) tmem_wait_st();  // the next unit's scale factors
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(sh.sfree);  // S^T read
+            if (sfa_next) finish_sfa(uc + 1);
             // K8V4: this token's K row scale, from the stage (then this
             // warp's reads of the stage are done)
             float ksc = 1.f;
