@@ -151,8 +151,7 @@ struct Fmt {
   static constexpr int kOffSfb = kOffVsc + kDeqWarps * kVscWarpBytes;  // [kNSMax][16] term scales
   static constexpr int kOffFac = kOffSfb + kNSMax * 16;            // float: 2^-k of each row
   static constexpr int kOffRed = kOffFac + kNSMax * 4;             // float [quarter][kNP]
-  static constexpr int kOffMask = kOffRed + 4 * kNP * 4;           // u32 [parity][quarter]
-  static constexpr int kOffM = kOffMask + 2 * 4 * 4;               // float [kNP]
+  static constexpr int kOffM = kOffRed + 4 * kNP * 4;              // float [kNP]
   static constexpr int kOffAlpha = kOffM + kNP * 4;
   static constexpr int kOffNvis = kOffAlpha + kNP * 4;
   static constexpr int kOffFlags = kOffNvis + kNP * 4;             // int[4]: abort at [2]
@@ -178,7 +177,6 @@ struct Shared {
   uint32_t *vsc;
   float *fac, *red, *m_s, *alpha_s;
   int32_t *nvis_s, *pages;
-  uint32_t *masks;
   volatile int *flags;
   // A barrier of a ring slot completes once per unit that uses the slot.  A
   // parity wait for unit u on it is only valid once the unit before u on
@@ -287,7 +285,7 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 kKsSlots = F::kKsSlots;
   constexpr int kOffKs = F::kOffKs, kOffQ = F::kOffQ, kOffP = F::kOffP, kOffVsc = F::kOffVsc,
                 kOffSfb = F::kOffSfb, kOffFac = F::kOffFac, kOffRed = F::kOffRed,
-                kOffMask = F::kOffMask, kOffM = F::kOffM, kOffAlpha = F::kOffAlpha,
+                kOffM = F::kOffM, kOffAlpha = F::kOffAlpha,
                 kOffNvis = F::kOffNvis, kOffFlags = F::kOffFlags, kOffPages = F::kOffPages,
                 kOffBars = F::kOffBars, kOffTmem = F::kOffTmem;
   extern __shared__ uint8_t smem_raw[];
@@ -302,7 +300,6 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
   sh.sfb = smem + kOffSfb;
   sh.fac = reinterpret_cast<float *>(smem + kOffFac);
   sh.red = reinterpret_cast<float *>(smem + kOffRed);
-  sh.masks = reinterpret_cast<uint32_t *>(smem + kOffMask);
   sh.m_s = reinterpret_cast<float *>(smem + kOffM);
   sh.alpha_s = reinterpret_cast<float *>(smem + kOffAlpha);
   sh.nvis_s = reinterpret_cast<int32_t *>(smem + kOffNvis);
@@ -888,11 +885,8 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
             }
           };
           weights();
-          uint32_t *masks = sh.masks + (uc & 1) * 4;
-          const uint32_t wup = __ballot_sync(0xffffffffu, up);
-          if (lane == 0) masks[lq] = wup;
-          named_barrier(1, kSmxWarps * 32);
-          const uint32_t any = masks[0] | masks[1] | masks[2] | masks[3];
+          // one barrier of the 4 softmax warps that also ORs the votes
+          const bool any = named_barrier_or(1, kSmxWarps * 32, up);
           if (any) {
             // Slow path (the first unit of a segment and rare max raises):
             // exact row maxima, new running max, rescale of everything
