@@ -156,7 +156,8 @@ struct Fmt {
   static constexpr int kOffNvis = kOffAlpha + kNP * 4;
   static constexpr int kOffFlags = kOffNvis + kNP * 4;             // int[4]: abort at [2]
   static constexpr int kOffPages = kOffFlags + 16;                 // int[stages][8]
-  static constexpr int kOffBars = kOffPages + kStages * kUnitPages * 4;
+  static constexpr int kOffKsv = kOffPages + kStages * kUnitPages * 4;  // u32 [ks slot]: pages present
+  static constexpr int kOffBars = kOffKsv + ((kKsSlots > 0 ? kKsSlots : 1) * 4 + 7) / 8 * 8;
   static constexpr int kNumBars = 2 * kStages + 2 * kKsSlots + 4 + 4 * kVSlots + 2 * kPSlots + 3;
   static constexpr int kOffTmem = kOffBars + kNumBars * 8;
   static constexpr int kSmemBytes = kOffTmem + 16 + 1024;          // + alignment slack
@@ -177,6 +178,7 @@ struct Shared {
   uint32_t *vsc;
   float *fac, *red, *m_s, *alpha_s;
   int32_t *nvis_s, *pages;
+  uint32_t *ksv;  // [ks slot]: bit p set when page p of the unit is present (NVFP4)
   volatile int *flags;
   // A barrier of a ring slot completes once per unit that uses the slot.  A
   // parity wait for unit u on it is only valid once the unit before u on
@@ -287,6 +289,7 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 kOffSfb = F::kOffSfb, kOffFac = F::kOffFac, kOffRed = F::kOffRed,
                 kOffM = F::kOffM, kOffAlpha = F::kOffAlpha,
                 kOffNvis = F::kOffNvis, kOffFlags = F::kOffFlags, kOffPages = F::kOffPages,
+                kOffKsv = F::kOffKsv,
                 kOffBars = F::kOffBars, kOffTmem = F::kOffTmem;
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -305,6 +308,7 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
   sh.nvis_s = reinterpret_cast<int32_t *>(smem + kOffNvis);
   sh.flags = reinterpret_cast<volatile int *>(smem + kOffFlags);
   sh.pages = reinterpret_cast<int32_t *>(smem + kOffPages);
+  sh.ksv = reinterpret_cast<uint32_t *>(smem + kOffKsv);
   uint64_t *bars = reinterpret_cast<uint64_t *>(smem + kOffBars);
   sh.full = bars;
   sh.empty = bars + kStages;
@@ -419,7 +423,10 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
       }
       const bool mine = lane < kUnitPages && cur >= 0;
       if (big && lane < kUnitPages) sh.pages[slot * kUnitPages + lane] = cur;
-      const uint32_t bytes = __popc(__ballot_sync(0xffffffffu, mine)) *
+      const uint32_t present = __ballot_sync(0xffffffffu, mine);
+      // the K-scale ring carries the unit's present pages to the softmax
+      if (!big && lane == 0) sh.ksv[slot] = present;
+      const uint32_t bytes = __popc(present) *
                              (!big ? kKsPageBytes : K8 ? kK8HeadBytes : kKPageBytes + kVPageBytes);
       __syncwarp();
       if (lane == 0) mbar_arrive_expect_tx(&fullb[slot], bytes);
@@ -566,12 +573,14 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
     // unit un-2.  Every lane quarter holds the same rows.
     // Column 4*ks + m1, lane l: the 4 scale bytes of token 32*m1 + l for
     // head_dim elements 64*ks .. 64*ks+63.
-    auto write_sfa = [&](uint32_t un) {
+    // Returns the unit's present-page mask, which travels with its K scales.
+    auto write_sfa = [&](uint32_t un) -> uint32_t {
       constexpr int kRing = kKsSlots > 0 ? kKsSlots : 1;  // (NVFP4 only)
       const int ksl = un % kRing;
       const uint8_t *kb = sh.ks + ksl * kKsSlotBytes;
       wait_bar(&sh.ks_full[ksl], (un / kRing) & 1, sh.flags, err);
       tc_fence_after();
+      const uint32_t present = sh.ksv[ksl];
       uint32_t w[16];
 #pragma unroll
       for (int m1 = 0; m1 < 4; ++m1) {
@@ -584,14 +593,19 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
       tmem_st16(tl + kColSFA + (un & 1) * 16, w);
       __syncwarp();  // every lane's loads are done (the store consumed them)
       if (lane == 0) mbar_arrive(&sh.ks_empty[ksl]);
+      return present;
     };
     // Publishes the scale factors of unit un once the warp's stores are
     // complete (the caller waits for them, together with its own loads).
     auto finish_sfa = [&](uint32_t un) {
       if (lane == 0) mbar_arrive(&sh.sfa_ready[un & 1]);
     };
+    // Present pages of the softmax's current and next unit (NVFP4: from the
+    // K-scale ring; a token of an absent page is skipped like an invisible
+    // one).
+    uint32_t pm_cur = 0xffu, pm_next = 0xffu;
     if (!K8 && smx && n_units > 0) {
-      write_sfa(0);
+      pm_cur = write_sfa(0);
       tmem_wait_st();
       tc_fence_before();
       __syncwarp();
@@ -816,7 +830,7 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
           // First the K scale factors of the next unit, while the scores of
           // this one are computed.
           const bool sfa_next = !K8 && uc + 1 < n_units;
-          if (sfa_next) write_sfa(uc + 1);
+          if (sfa_next) pm_next = write_sfa(uc + 1);
           const int pos = tok0 + 32 * lq + lane;
           wait_bar(sh.sready, uc & 1, sh.flags, err);
           tc_fence_after();
@@ -838,15 +852,19 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
             // K8V4: this token's K row scale, from the stage (then this
             // warp's reads of the stage are done)
             float ksc = 1.f;
+            bool present;  // the token's page was loaded
             if constexpr (K8) {
               wait_bar(&sh.full[stage], (uc / kStages) & 1, sh.flags, err);
               const int j = 32 * lq + lane;
               ksc = *reinterpret_cast<const float *>(sh.stages + stage * kStageBytes + F::kKsOff +
                                                      (j >> 4) * 128 + (j & 15) * 4);
+              present = sh.pages[stage * kUnitPages + (j >> 4)] >= 0;
               __syncwarp();
               if (lane == 0) mbar_arrive(&sh.empty[stage]);
+            } else {
+              present = (pm_cur >> ((32 * lq + lane) >> 4)) & 1u;
             }
-            const bool vis_all = tok0 + kUnitTokens <= sg.kv_len - T + 1;
+            const bool vis_all = tok0 + kUnitTokens <= sg.kv_len - T + 1 && present;
 #pragma unroll
             for (int j = 0; j < RM; ++j) {
               const uint32_t *c8 = rr + j * kTerms;
@@ -868,7 +886,7 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
                 sc = (a2.x + a2.y) * facr[j];
               }
               const int nv = vis_all ? (j < R ? 0x7fffffff : 0) : sh.nvis_s[j];
-              x[j] = pos < nv ? sc : -INFINITY;
+              x[j] = pos < nv && present ? sc : -INFINITY;
             }
           }
           // Weights: p = 2^(score - running max) in fp32 (2^-inf = 0), as
@@ -971,6 +989,7 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&sh.pready[ps]);
+          pm_cur = pm_next;
         }
       }
 

@@ -243,3 +243,57 @@ def test_tensor_core_and_cuda_core_kernels_agree(case, monkeypatch):
             monkeypatch.setenv("NVKV_DECODE_KERNEL", "simt")
         dw = run_step(wl)
         assert_close(gpu_rows(dw.out, wl, rows), ref, f"{name}/{kernel}")
+
+
+@pytest.mark.parametrize("T,kernel", [(1, "decode_qk4"), (4, "decode_tc")])
+def test_tensor_core_kernels_report_bad_page_and_stay_finite(T, kernel):
+    """head_dim 256: an out-of-range page id in a visible range is reported
+    through the error word by the tensor-core kernels, its tokens are
+    skipped, and every output stays finite."""
+    dev = torch.device("cuda")
+    hkv, hq, d = 4, 24, 256
+    cache = nv.Cache.allocate(4, hkv, d, dev, fill=0)
+    pt = torch.tensor([[0, 1, 99, 2]], dtype=torch.int32, device=dev)  # page 99 does not exist
+    lens = torch.tensor([60], dtype=torch.int32, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    seqs = nv.Seqs(pt, lens, 64, err)
+    assert nv.nvkv_decode_kernel_name(cache, T, hq) == kernel
+    q = torch.randn((T, hq, d), device=dev).bfloat16()
+    S = 3
+    ws = torch.empty(nv.nvkv_decode_workspace_bytes(1, T, hq, hkv, d, S), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty((T, hq, d), dtype=torch.bfloat16, device=dev)
+    nv.nvkv_decode_attn(cache, seqs, q, T, hq, 0.0625, S, ws)
+    nv.nvkv_combine(seqs, ws, T, hq, hkv, d, S, out)
+    torch.cuda.synchronize()
+    assert int(err.item()) & nv.DEVERR_PAGE_ID
+    assert torch.isfinite(out.float()).all()
+    # the loaded pages are all zero (fill 0), so every row is a mean of zeros
+    assert (out.float() == 0).all()
+
+
+@pytest.mark.parametrize("T,kernel", [(1, "decode_qk4"), (4, "decode_tc")])
+def test_tensor_core_kernels_empty_sequence_gives_zeros(T, kernel):
+    """head_dim 256, a batch whose first sequence has no key at all and
+    whose second has fewer keys than queries: rows without a visible key
+    are zeros, the others match the oracle."""
+    wl = W.small(f"empty_T{T}", 2, 24, 4, 256, T, [0, 700], seed=12)
+    dw = DeviceWorkload(wl, num_splits=7)
+    dw.fill_context()
+    dw.load_step_inputs()
+    assert nv.nvkv_decode_kernel_name(dw.cache, T, wl.num_q_heads) == kernel
+    # no step append: sequence 0 has kv_len 0 (every row sees no key),
+    # sequence 1 its 700 cached rows
+    dw.kv_lens.copy_(torch.tensor([0, 700], dtype=torch.int32))
+    dw.attend()
+    torch.cuda.synchronize()
+    assert dw.err_bits() == 0
+    out = dw.out.float().cpu().numpy()
+    assert (out[:T] == 0).all()
+    rows = [(1, t, hq) for t in range(T) for hq in range(wl.num_q_heads)]
+    q = wl.queries()
+    got = np.stack([out[T + t, hq] for _, t, hq in rows]).astype(np.float64)
+    k, v = wl.kv_rows(1, 0, 700)
+    jobs = [(k, v, hq // wl.group, 700 - T + t + 1, q[T + t, hq]) for _, t, hq in rows]
+    ref, _, _ = oracle.attention_rows(jobs, wl.num_kv_heads, wl.head_dim, wl.sm_scale)
+    assert_close(got, ref, wl.name)

@@ -239,6 +239,31 @@ def test_decode_k8v4_reports_bad_page():
     assert torch.isfinite(out.float()).all()
 
 
+def test_decode_k8v4_tensor_core_reports_bad_page():
+    """head_dim 256 on the tensor-core K8V4 decode: an out-of-range page id
+    inside the visible range is reported, its tokens are skipped, and the
+    outputs equal the oracle over the remaining keys (a fill of 0 makes
+    every loaded key and value zero, so each row is the mean of zeros)."""
+    dev = torch.device("cuda")
+    hkv, hq, d = 4, 24, 256
+    cache = nv.Cache.allocate(4, hkv, d, dev, fill=0, kv_format="k8v4")
+    pt = torch.tensor([[0, 1, 99, 2]], dtype=torch.int32, device=dev)
+    lens = torch.tensor([60], dtype=torch.int32, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    seqs = nv.Seqs(pt, lens, 64, err)
+    assert nv.nvkv_decode_kernel_name(cache, 1, hq) == "decode_qk4_k8v4"
+    q = torch.randn((1, hq, d), device=dev).bfloat16()
+    ws = torch.empty(nv.nvkv_decode_workspace_bytes(1, 1, hq, hkv, d, 3), dtype=torch.uint8,
+                     device=dev)
+    out = torch.empty((1, hq, d), dtype=torch.bfloat16, device=dev)
+    nv.nvkv_decode_attn_k8v4(cache, seqs, q, 1, hq, 0.0625, 3, ws)
+    nv.nvkv_combine(seqs, ws, 1, hq, hkv, d, 3, out)
+    torch.cuda.synchronize()
+    assert int(err.item()) & nv.DEVERR_PAGE_ID
+    assert torch.isfinite(out.float()).all()
+    assert (out.float() == 0).all()
+
+
 @pytest.mark.parametrize("kind", ["device", "pinned"])
 def test_k8v4_spill_restore_and_attention_after_restore(kind):
     """Whole K8V4 pages (nvkv_k8v4_page_bytes each) move to arena slots and
