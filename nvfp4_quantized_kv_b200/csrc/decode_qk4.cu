@@ -629,6 +629,10 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
 #pragma unroll
         for (int i = 0; i < RM; ++i) l_part[i] = 0.f, mr[i] = -FLT_MAX;
+      }
+      {
+        // Query terms of the pair, one row per worker warp (rows are
+        // independent chains of conversions; the pipeline waits for them).
         // Row r of x = q * sm_scale * log2(e): one power-of-two prescale 2^k
         // puts the row maximum in [256, 512); then term l quantises the
         // residual y (group scale = E4M3 of its 16-element maximum / 6,
@@ -639,7 +643,7 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
         // columns r*8 .. r*8+7 summed and times 2^-k give the row's scores.
         // (Any rounding of the scales and codes would do: only the residual
         // bookkeeping has to be exact.)
-        for (int r = warp - kSmxWarp0; r < RM; r += kSmxWarps) {
+        for (int r = warp; r < RM; r += kDeqWarps + kSmxWarps) {
           float y[8];
           if (r < R) {
             const int t = r / G, g = r % G;
@@ -729,7 +733,9 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
           if (lane == 0) sh.fac[r] = eb > 0 ? scale_pow2(1.f, -k) : 0.f;
         }
         fence_proxy_async_smem();
-        named_barrier(1, kSmxWarps * 32);
+        named_barrier(2, kSegThreads);
+      }
+      if (smx) {
 #pragma unroll
         for (int i = 0; i < RM; ++i) facr[i] = sh.fac[i];
         // Scale factors of the terms into Tensor Memory (each lane quarter
