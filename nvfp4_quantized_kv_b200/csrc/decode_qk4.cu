@@ -114,7 +114,6 @@ constexpr int kMmaWarp = 13;             // issues the score MMAs
 constexpr int kPvWarp = 14;              // issues the value MMAs
 constexpr int kKsProducerWarp = 15;      // K scales
 constexpr int kThreads = 16 * 32;
-constexpr int kSegThreads = (kDeqWarps + kSmxWarps) * 32;
 constexpr uint32_t kTmemCols = 512;
 constexpr long long kWaitBudget = 2000000000LL;  // clock cycles (~1 s)
 constexpr float kLazyRescale = 8.0f;             // log2 units
@@ -158,7 +157,7 @@ struct Fmt {
   static constexpr int kOffPages = kOffFlags + 16;                 // int[stages][8]
   static constexpr int kOffKsv = kOffPages + kStages * kUnitPages * 4;  // u32 [ks slot]: pages present
   static constexpr int kOffBars = kOffKsv + ((kKsSlots > 0 ? kKsSlots : 1) * 4 + 7) / 8 * 8;
-  static constexpr int kNumBars = 2 * kStages + 2 * kKsSlots + 4 + 4 * kVSlots + 2 * kPSlots + 3;
+  static constexpr int kNumBars = 2 * kStages + 2 * kKsSlots + 4 + 4 * kVSlots + 2 * kPSlots + 5;
   static constexpr int kOffTmem = kOffBars + kNumBars * 8;
   static constexpr int kSmemBytes = kOffTmem + 16 + 1024;          // + alignment slack
   // (TMA destinations are 128-byte aligned: each page's 64 bytes of K row
@@ -191,23 +190,14 @@ struct Shared {
   uint64_t *vready, *pvdone;     // [kVSlots][half]: V^T written; value MMAs done
   uint64_t *pready, *pfree;      // [kPSlots]: P written; P read by the value MMAs
   uint64_t *qready, *final_bar, *final_pv;
+  uint64_t *qfree;     // every score MMA of the segment completed (query tiles free)
+  uint64_t *segstart;  // the softmax has taken the segment's row factors
   uint32_t *tmem_slot;
 };
 
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *flags,
                                          int32_t *err) {
-  if (flags[2]) return false;  // aborted: do not wait any more
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
-    if (flags[2]) return false;
-    if (clock64() - t0 > kWaitBudget) {
-      flags[2] = 1;
-      report(err, NVKV_DEVERR_TIMEOUT);
-      return false;
-    }
-  }
-  return true;
+  return guarded_wait(bar, parity, flags + 2, err, kWaitBudget);  // flags[2]: abort
 }
 
 // Segment of the CTA's range: units [u, seg_end) of pair (b, h).
@@ -324,6 +314,8 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
   sh.qready = sh.pfree + kPSlots;
   sh.final_bar = sh.qready + 1;
   sh.final_pv = sh.qready + 2;
+  sh.qfree = sh.qready + 3;
+  sh.segstart = sh.qready + 4;
   sh.tmem_slot = reinterpret_cast<uint32_t *>(smem + kOffTmem);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -352,7 +344,9 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
       mbar_init(&sh.pready[i], kSmxWarps);
       mbar_init(&sh.pfree[i], 1);
     }
-    mbar_init(sh.qready, kSmxWarps);
+    mbar_init(sh.qready, 4);  // the V^T writers of lane quarters 0..3
+    mbar_init(sh.qfree, 1);
+    mbar_init(sh.segstart, kSmxWarps);
     mbar_init(sh.final_bar, 1);
     mbar_init(sh.final_pv, 1);
     fence_mbar_init();
@@ -516,6 +510,9 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
           }
           mma_commit(sh.sready);
           mma_commit(&sh.empty[stage]);  // the K tile has been read
+          // the last score MMA of a segment that another follows: the V^T
+          // writers may build the next pair's query terms
+          if (uu + 1 >= seg_end && uu + 1 < u1) mma_commit(sh.qfree);
           issued = true;
         }
         if (issued) {
@@ -612,139 +609,119 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
       finish_sfa(0);
     }
 
-    uint32_t uc = 0;
-    uint32_t seg_idx = 0;
-    for (int64_t u = u0; u < u1; ++seg_idx) {
-      const Seg sg = segment_at(u, u1, kv_lens, B, Hkv, max_kv_len, max_pages);
-      if (sg.bad && threadIdx.x == 0) report(err, NVKV_DEVERR_LENGTH);
-      const int64_t seg_start = u;
-      const size_t slot = (size_t)c + (size_t)sg.b * Hkv + sg.h;
-
-      if (smx) {
-        // ---- query terms of this pair (the previous segment's score MMAs
-        // have completed: its last softmax waited for them) ----
-        if (stid < kNP) {
-          sh.nvis_s[stid] = stid < R ? sg.kv_len - T + stid / G + 1 : 0;
-          sh.m_s[stid] = -FLT_MAX;
+    // Query terms of pair pg, one row per V^T-writing warp (rows are
+    // independent chains of conversions), then their scale factors into
+    // Tensor Memory and the release of the pair's score MMAs.  The V^T
+    // writers build them for the next pair as soon as the current segment's
+    // last score MMA has completed, so the next segment's first scores are
+    // computed while the softmax finishes this one.
+    auto prep_q = [&](const Seg &pg) {
+      // Row r of x = q * sm_scale * log2(e): one power-of-two prescale 2^k
+      // puts the row maximum in [256, 512); then term l quantises the
+      // residual y (group scale = E4M3 of its 16-element maximum / 6,
+      // codes = nearest E2M1) and leaves y - term, exactly.  Each term
+      // shrinks every group's residual at least 5.6x, so the scales of the
+      // 8 terms stay inside the E4M3 range (448 down to 2^-9) until the
+      // remainder is below about 2^-15 of the row maximum.  The MMA's
+      // columns r*8 .. r*8+7 summed and times 2^-k give the row's scores.
+      // (Any rounding of the scales and codes would do: only the residual
+      // bookkeeping has to be exact.)
+      for (int r = warp; r < RM; r += kDeqWarps) {
+        float y[8];
+        if (r < R) {
+          const int t = r / G, g = r % G;
+          const uint4 raw = *reinterpret_cast<const uint4 *>(
+              q + ((size_t)(pg.b * T + t) * Hq + pg.h * G + g) * kD + 8 * lane);
+          const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            y[2 * i] = __uint_as_float(w[i] << 16) * qscale;
+            y[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u) * qscale;
+          }
+        } else {
+#pragma unroll
+          for (int i = 0; i < 8; ++i) y[i] = 0.f;
         }
+        float a = 0.f;
 #pragma unroll
-        for (int i = 0; i < RM; ++i) l_part[i] = 0.f, mr[i] = -FLT_MAX;
-      }
-      {
-        // Query terms of the pair, one row per worker warp (rows are
-        // independent chains of conversions; the pipeline waits for them).
-        // Row r of x = q * sm_scale * log2(e): one power-of-two prescale 2^k
-        // puts the row maximum in [256, 512); then term l quantises the
-        // residual y (group scale = E4M3 of its 16-element maximum / 6,
-        // codes = nearest E2M1) and leaves y - term, exactly.  Each term
-        // shrinks every group's residual at least 5.6x, so the scales of the
-        // 8 terms stay inside the E4M3 range (448 down to 2^-9) until the
-        // remainder is below about 2^-15 of the row maximum.  The MMA's
-        // columns r*8 .. r*8+7 summed and times 2^-k give the row's scores.
-        // (Any rounding of the scales and codes would do: only the residual
-        // bookkeeping has to be exact.)
-        for (int r = warp; r < RM; r += kDeqWarps + kSmxWarps) {
-          float y[8];
-          if (r < R) {
-            const int t = r / G, g = r % G;
-            const uint4 raw = *reinterpret_cast<const uint4 *>(
-                q + ((size_t)(sg.b * T + t) * Hq + sg.h * G + g) * kD + 8 * lane);
-            const uint32_t w[4] = {raw.x, raw.y, raw.z, raw.w};
+        for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(y[i]));
+        a = warp_max(a);
+        // A row whose largest element is below the smallest normal float
+        // (2^-126) is taken as zero: its scores would be below 2^-110.
+        const int eb = (int)((__float_as_uint(a) >> 23) & 0xffu);  // biased exponent
+        // a in [2^(eb-127), 2^(eb-126)): a * 2^k in [256, 512) (NVFP4), in
+        // [128, 256) (K8V4, under the E4M3 maximum 448)
+        const int k = (K8 ? 134 : 135) - eb;
+        if (eb > 0) {
 #pragma unroll
-            for (int i = 0; i < 4; ++i) {
-              y[2 * i] = __uint_as_float(w[i] << 16) * qscale;
-              y[2 * i + 1] = __uint_as_float(w[i] & 0xffff0000u) * qscale;
-            }
-          } else {
+          for (int i = 0; i < 8; ++i) y[i] = scale_pow2(y[i], k);
+        } else {
 #pragma unroll
-            for (int i = 0; i < 8; ++i) y[i] = 0.f;
-          }
-          float a = 0.f;
-#pragma unroll
-          for (int i = 0; i < 8; ++i) a = fmaxf(a, fabsf(y[i]));
-          a = warp_max(a);
-          // A row whose largest element is below the smallest normal float
-          // (2^-126) is taken as zero: its scores would be below 2^-110.
-          const int eb = (int)((__float_as_uint(a) >> 23) & 0xffu);  // biased exponent
-          // a in [2^(eb-127), 2^(eb-126)): a * 2^k in [256, 512) (NVFP4), in
-          // [128, 256) (K8V4, under the E4M3 maximum 448)
-          const int k = (K8 ? 134 : 135) - eb;
-          if (eb > 0) {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) y[i] = scale_pow2(y[i], k);
-          } else {
-#pragma unroll
-            for (int i = 0; i < 8; ++i) y[i] = 0.f;
-          }
-          if constexpr (K8) {
-            // Term l: E4M3 codes of y * 2^(4l), its value subtracted exactly.
-            // E4M3 rounding leaves at most 2^-4 of an element (or 2^-10 of
-            // the term's unit in the subnormal range), so y * 2^(4(l+1))
-            // stays below 256 and no term saturates; the MMA's column 8r + l
-            // carries weight 2^-4l, recombined in the softmax.
-#pragma unroll 1
-            for (int l = 0; l < kTerms; ++l) {
-              const int n = r * kTerms + l;
-              const float up = pow2f(4 * l), down = pow2f(-4 * l);
-              uint32_t pr[4];
-#pragma unroll
-              for (int i = 0; i < 4; ++i) {
-                pr[i] = f32x2_to_e4m3x2(y[2 * i] * up, y[2 * i + 1] * up);
-                const float2 v = f16x2_to_float2(e4m3x2_to_f16x2(pr[i]));
-                y[2 * i] -= v.x * down;  // exact
-                y[2 * i + 1] -= v.y * down;
-              }
-              // bytes 8*lane .. 8*lane+7 of the row: head_dim half lane/16,
-              // 128-byte swizzle
-              const int c16 = (lane & 15) >> 1;
-              *reinterpret_cast<uint2 *>(sh.qtile + (lane >> 4) * (kNSMax * 128) + n * 128 +
-                                         ((c16 ^ (n & 7)) << 4) + (lane & 1) * 8) =
-                  make_uint2(pr[0] | (pr[1] << 16), pr[2] | (pr[3] << 16));
-            }
-          } else {
+          for (int i = 0; i < 8; ++i) y[i] = 0.f;
+        }
+        if constexpr (K8) {
+          // Term l: E4M3 codes of y * 2^(4l), its value subtracted exactly.
+          // E4M3 rounding leaves at most 2^-4 of an element (or 2^-10 of
+          // the term's unit in the subnormal range), so y * 2^(4(l+1))
+          // stays below 256 and no term saturates; the MMA's column 8r + l
+          // carries weight 2^-4l, recombined in the softmax.
 #pragma unroll 1
           for (int l = 0; l < kTerms; ++l) {
             const int n = r * kTerms + l;
-            float ga = 0.f;
-#pragma unroll
-            for (int i = 0; i < 8; ++i) ga = fmaxf(ga, fabsf(y[i]));
-            ga = fmaxf(ga, __shfl_xor_sync(0xffffffffu, ga, 1));  // 16-element group
-            const uint32_t sb = (uint32_t)__nv_cvt_float_to_fp8(ga * (1.0f / 6.0f), __NV_SATFINITE,
-                                                                __NV_E4M3);
-            const float sv = e4m3_to_float((uint8_t)sb);
-            const float rs = sv > 0.f ? 1.0f / sv : 0.f;
-            uint32_t codes = 0;
+            const float up = pow2f(4 * l), down = pow2f(-4 * l);
+            uint32_t pr[4];
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
-              // codes of y/s (the hardware's rounding; any choice is exact
-              // bookkeeping below), then the chosen values, exact in f16
-              const uint32_t pair = f32x2_to_e2m1x2(y[2 * i] * rs, y[2 * i + 1] * rs);
-              codes |= pair << (8 * i);
-              const float2 v = f16x2_to_float2(e2m1x2_to_f16x2(pair));
-              y[2 * i] -= v.x * sv;  // the products are exact
-              y[2 * i + 1] -= v.y * sv;
+              pr[i] = f32x2_to_e4m3x2(y[2 * i] * up, y[2 * i + 1] * up);
+              const float2 v = f16x2_to_float2(e4m3x2_to_f16x2(pr[i]));
+              y[2 * i] -= v.x * down;  // exact
+              y[2 * i + 1] -= v.y * down;
             }
-            // Row n of the term tile: bytes 4*lane..4*lane+3, 128-byte swizzle.
-            *reinterpret_cast<uint32_t *>(sh.qtile + n * 128 + (((lane >> 2) ^ (n & 7)) << 4) +
-                                          (lane & 3) * 4) = codes;
-            if ((lane & 1) == 0) sh.sfb[n * 16 + (lane >> 1)] = (uint8_t)sb;
+            // bytes 8*lane .. 8*lane+7 of the row: head_dim half lane/16,
+            // 128-byte swizzle
+            const int c16 = (lane & 15) >> 1;
+            *reinterpret_cast<uint2 *>(sh.qtile + (lane >> 4) * (kNSMax * 128) + n * 128 +
+                                       ((c16 ^ (n & 7)) << 4) + (lane & 1) * 8) =
+                make_uint2(pr[0] | (pr[1] << 16), pr[2] | (pr[3] << 16));
           }
-          }
-          if (lane == 0) sh.fac[r] = eb > 0 ? scale_pow2(1.f, -k) : 0.f;
-        }
-        fence_proxy_async_smem();
-        named_barrier(2, kSegThreads);
-      }
-      if (smx) {
-#pragma unroll
-        for (int i = 0; i < RM; ++i) facr[i] = sh.fac[i];
-        // Scale factors of the terms into Tensor Memory (each lane quarter
-        // holds all rows): column 4*ks + n1, lane l -> row 32*n1 + l (every
-        // K step's block starts on a multiple of 4 columns).  K8V4 has none.
-        if (K8) {
-          __syncwarp();
-          if (lane == 0) mbar_arrive(sh.qready);
         } else {
+#pragma unroll 1
+        for (int l = 0; l < kTerms; ++l) {
+          const int n = r * kTerms + l;
+          float ga = 0.f;
+#pragma unroll
+          for (int i = 0; i < 8; ++i) ga = fmaxf(ga, fabsf(y[i]));
+          ga = fmaxf(ga, __shfl_xor_sync(0xffffffffu, ga, 1));  // 16-element group
+          const uint32_t sb = (uint32_t)__nv_cvt_float_to_fp8(ga * (1.0f / 6.0f), __NV_SATFINITE,
+                                                              __NV_E4M3);
+          const float sv = e4m3_to_float((uint8_t)sb);
+          const float rs = sv > 0.f ? 1.0f / sv : 0.f;
+          uint32_t codes = 0;
+#pragma unroll
+          for (int i = 0; i < 4; ++i) {
+            // codes of y/s (the hardware's rounding; any choice is exact
+            // bookkeeping below), then the chosen values, exact in f16
+            const uint32_t pair = f32x2_to_e2m1x2(y[2 * i] * rs, y[2 * i + 1] * rs);
+            codes |= pair << (8 * i);
+            const float2 v = f16x2_to_float2(e2m1x2_to_f16x2(pair));
+            y[2 * i] -= v.x * sv;  // the products are exact
+            y[2 * i + 1] -= v.y * sv;
+          }
+          // Row n of the term tile: bytes 4*lane..4*lane+3, 128-byte swizzle.
+          *reinterpret_cast<uint32_t *>(sh.qtile + n * 128 + (((lane >> 2) ^ (n & 7)) << 4) +
+                                        (lane & 3) * 4) = codes;
+          if ((lane & 1) == 0) sh.sfb[n * 16 + (lane >> 1)] = (uint8_t)sb;
+        }
+        }
+        if (lane == 0) sh.fac[r] = eb > 0 ? scale_pow2(1.f, -k) : 0.f;
+      }
+      fence_proxy_async_smem();
+      named_barrier(2, kDeqWarps * 32);
+      if (warp < 4) {
+        // Scale factors of the terms (each lane quarter holds all rows):
+        // column 4*ks + n1, lane l -> row 32*n1 + l (every K step's block
+        // starts on a multiple of 4 columns).  K8V4 has none.
+        if constexpr (!K8) {
           uint32_t w[16];
 #pragma unroll
           for (int i = 0; i < 16; ++i) w[i] = 0u;
@@ -759,9 +736,47 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
           tmem_st16(tl + kColSFB, w);
           tmem_wait_st();
           tc_fence_before();
-          __syncwarp();
-          if (lane == 0) mbar_arrive(sh.qready);
         }
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sh.qready);
+      }
+    };
+
+    uint32_t uc = 0;
+    uint32_t seg_idx = 0;
+    for (int64_t u = u0; u < u1; ++seg_idx) {
+      const Seg sg = segment_at(u, u1, kv_lens, B, Hkv, max_kv_len, max_pages);
+      if (sg.bad && threadIdx.x == 0) report(err, NVKV_DEVERR_LENGTH);
+      const int64_t seg_start = u;
+      const size_t slot = (size_t)c + (size_t)sg.b * Hkv + sg.h;
+
+      if (!smx) {
+        if (seg_idx > 0) {
+          // The V^T writers come here straight from the previous segment's
+          // units: its query terms are replaced once the softmax has taken
+          // its row factors (so the shared factors and the query-term
+          // barrier run one segment ahead at most) and its score MMAs have
+          // all completed.
+          wait_bar(sh.segstart, (seg_idx - 1) & 1, sh.flags, err);
+          wait_bar(sh.qfree, (seg_idx - 1) & 1, sh.flags, err);
+          tc_fence_after();
+        }
+        prep_q(sg);
+      } else {
+        // softmax state of the pair; its query terms' row factors (the V^T
+        // writers published them with the terms)
+        if (stid < kNP) {
+          sh.nvis_s[stid] = stid < R ? sg.kv_len - T + stid / G + 1 : 0;
+          sh.m_s[stid] = -FLT_MAX;
+        }
+#pragma unroll
+        for (int i = 0; i < RM; ++i) l_part[i] = 0.f, mr[i] = -FLT_MAX;
+        wait_bar(sh.qready, seg_idx & 1, sh.flags, err);
+#pragma unroll
+        for (int i = 0; i < RM; ++i) facr[i] = sh.fac[i];
+        __syncwarp();
+        if (lane == 0) mbar_arrive(sh.segstart);
+        named_barrier(1, kSmxWarps * 32);  // the row state is written
       }
 
       for (; u < sg.seg_end; ++u, ++uc) {
@@ -999,46 +1014,51 @@ decode_qk4_kernel(const __grid_constant__ CUtensorMap tmap_k,
         }
       }
 
-      // ---- end of segment: O^T / l -> workspace, lse ----
-      if (uc > 0) {
-        // the last unit's value MMAs, both halves (every worker has seen
-        // the value MMAs of unit uc-5 complete)
+
+      if (smx) {
+        // ---- end of segment: O^T / l -> workspace, lse (thread: head_dim
+        // rows d = 32*lq + lane and d + 128) ----
+        // the last unit's value MMAs, both halves (every softmax warp has
+        // seen the value MMAs of unit uc-5 complete)
         wait_bar(&sh.pfree[(uc - 1) % kPSlots], ((uc - 1) / kPSlots) & 1, sh.flags, err);
         tc_fence_after();
-      }
-      if (smx) {
 #pragma unroll
         for (int j = 0; j < RM; ++j) {
           const float ls = warp_sum(l_part[j]);
           if (lane == 0) sh.red[lq * kNP + j] = ls;
         }
-      }
-      named_barrier(2, kSegThreads);
-      if (smx && stid < RM) {
-        float l = 0.f;
-#pragma unroll
-        for (int w = 0; w < 4; ++w) l += sh.red[w * kNP + stid];
-        sh.alpha_s[stid] = l;
-      }
-      named_barrier(2, kSegThreads);
-      if (!smx) {
-        // The sums carry the 2^-14 of V^T: o = O * 2^14 / l, lse = m + log2(l).
-        const int d = 128 * hv + 32 * lq + lane;
-        uint32_t o8[8];
-        tmem_ld8(tl + kColO + hv * kNP, o8);
-        tmem_wait_ld();
+        named_barrier(1, kSmxWarps * 32);
+        float lv[RM];
 #pragma unroll
         for (int n = 0; n < RM; ++n) {
-          if (n < R) {
-            const float lv = sh.alpha_s[n];
-            const float v = __uint_as_float(o8[n]);
-            ws_o[(slot * R + n) * kD + d] = lv > 0.f ? v * 16384.f / lv : 0.f;
-            if (d == 0) ws_lse[slot * R + n] = lv > 0.f ? sh.m_s[n] + log2f(lv) : -INFINITY;
+          lv[n] = 0.f;
+#pragma unroll
+          for (int w = 0; w < 4; ++w) lv[n] += sh.red[w * kNP + n];
+        }
+        // The sums carry the 2^-14 of V^T: o = O * 2^14 / l, lse = m + log2(l).
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          uint32_t o8[8];
+          tmem_ld8(tl + kColO + half * kNP, o8);
+          tmem_wait_ld();
+          const int d = 128 * half + 32 * lq + lane;
+#pragma unroll
+          for (int n = 0; n < RM; ++n) {
+            if (n < R) {
+              const float v = __uint_as_float(o8[n]);
+              ws_o[(slot * R + n) * kD + d] = lv[n] > 0.f ? v * 16384.f / lv[n] : 0.f;
+            }
           }
         }
+        if (stid < R) {
+          float l = 0.f;
+#pragma unroll
+          for (int n = 0; n < RM; ++n) l = n == stid ? lv[n] : l;
+          ws_lse[slot * R + stid] = l > 0.f ? sh.m_s[stid] + log2f(l) : -INFINITY;
+        }
+        tc_fence_before();
+        named_barrier(1, kSmxWarps * 32);  // the sums and maxima have been read
       }
-      tc_fence_before();
-      named_barrier(2, kSegThreads);
     }
   }
 

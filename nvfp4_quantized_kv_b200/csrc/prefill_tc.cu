@@ -81,18 +81,7 @@ static_assert(kOffK % 1024 == 0 && kOffPages % 16 == 0 && kOffBars % 8 == 0, "al
 
 __device__ __forceinline__ bool wait_bar(uint64_t *bar, uint32_t parity, volatile int *flags,
                                          int32_t *err) {
-  if (flags[2]) return false;
-  if (mbar_try_wait(bar, parity)) return true;
-  const long long t0 = clock64();
-  while (!mbar_try_wait(bar, parity)) {
-    if (flags[2]) return false;
-    if (clock64() - t0 > kWaitBudget) {
-      flags[2] = 1;
-      report(err, NVKV_DEVERR_TIMEOUT);
-      return false;
-    }
-  }
-  return true;
+  return guarded_wait(bar, parity, flags + 2, err, kWaitBudget);  // flags[2]: abort
 }
 
 __device__ __forceinline__ uint32_t dup_scale(uint32_t byte) {

@@ -7,6 +7,8 @@
 #include <cuda.h>
 #include <stdint.h>
 
+#include "nvkv_common.cuh"
+
 namespace nvkv {
 namespace sm100 {
 
@@ -63,6 +65,33 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, long l
     if (clock64() - t0 > budget) return false;
   }
   return true;
+}
+
+// The pipeline wait of the tensor-core kernels: gives up after `budget`
+// clock cycles, raising the CTA's abort flag and reporting a timeout; once
+// the flag is up no wait blocks any more.  Only the first probe is inline:
+// the spin is a function of its own, so each of the many waits in the warp
+// roles' loops adds a few instructions, not a loop, to the code that the
+// roles' loops share an SM's instruction caches with.
+static __device__ __noinline__ bool guarded_wait_spin(uint64_t *bar, uint32_t parity,
+                                                      volatile int *abort, int32_t *err,
+                                                      long long budget) {
+  const long long t0 = clock64();
+  while (!mbar_try_wait(bar, parity)) {
+    if (*abort) return false;
+    if (clock64() - t0 > budget) {
+      *abort = 1;
+      report(err, NVKV_DEVERR_TIMEOUT);
+      return false;
+    }
+  }
+  return true;
+}
+__device__ __forceinline__ bool guarded_wait(uint64_t *bar, uint32_t parity, volatile int *abort,
+                                             int32_t *err, long long budget) {
+  if (*abort) return false;
+  if (__builtin_expect(mbar_try_wait(bar, parity), 1)) return true;
+  return guarded_wait_spin(bar, parity, abort, err, budget);
 }
 
 // ---------------------------------------------------------------------------
