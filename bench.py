@@ -31,6 +31,7 @@ from __future__ import annotations
 
 import argparse
 import datetime
+import hashlib
 import json
 import os
 import statistics
@@ -56,33 +57,43 @@ DATASHEET_HBM_GBS = 8000.0
 DATASHEET_BF16_TFLOPS = 2250.0  # dense
 
 # DRAM traffic of one decode-attention launch, from one ncu capture of the
-# kernel source with this SHA-256 (profiles/decode_qk4_long_ctx_3x60k_T1.md:
-# 3 x 60000 cached tokens, T=1, 24/4 heads, d 256).  Traffic grows with the
-# KV bytes attended, so it is scaled by them to the benchmarked workload; it
-# applies only to that kernel, and once its source changes the figure no
+# kernel built from the sources whose SHA-256 (of their concatenation, in this
+# order) is recorded here (profiles/decode_qk4_long_ctx_3x60k_T1.md: 3 x 60000
+# cached tokens, T=1, 24/4 heads, d 256).  Traffic grows with the KV bytes
+# attended, so it is scaled by them to the benchmarked workload; it applies
+# only to that kernel, and once any of its sources changes the figure no
 # longer applies and is reported null.
 DECODE_CAPTURE = {
     "kernel": "decode_qk4",
-    "source": "nvfp4_quantized_kv_b200/csrc/decode_qk4.cu",
-    "sha256": "a9499a735164b17eb255cc502a9c3c5d9d42af8d0f5ffd5534031fc4879e4a01",
-    "dram_bytes_read": 207596288,
-    "dram_bytes_write": 4512000,
+    "sources": ["nvfp4_quantized_kv_b200/csrc/decode_qk4.cu",
+                "nvfp4_quantized_kv_b200/csrc/sm100.cuh",
+                "nvfp4_quantized_kv_b200/csrc/nvkv_common.cuh",
+                "include/nvkv.h"],
+    "sha256": "",
+    "dram_bytes_read": 0,
+    "dram_bytes_write": 0,
     "kv_bytes": 207363456,
 }
 
 
-def decode_traffic(kv_bytes, kernel):
-    """Per-launch DRAM bytes of the decode kernel scaled from the capture, or
-    None when another kernel ran or its source is not the captured one."""
-    import hashlib
-    if kernel != DECODE_CAPTURE["kernel"] or not DECODE_CAPTURE["sha256"]:
-        return None
+def sources_sha256(paths):
+    """SHA-256 of the concatenated files (None when one is missing)."""
+    h = hashlib.sha256()
     try:
-        with open(os.path.join(ROOT, DECODE_CAPTURE["source"]), "rb") as f:
-            digest = hashlib.sha256(f.read()).hexdigest()
+        for rel in paths:
+            with open(os.path.join(ROOT, rel), "rb") as f:
+                h.update(f.read())
     except OSError:
         return None
-    if digest != DECODE_CAPTURE["sha256"]:
+    return h.hexdigest()
+
+
+def decode_traffic(kv_bytes, kernel):
+    """DRAM bytes (read + write) of one decode launch attending kv_bytes, or
+    None when the kernel or its sources differ from the captured ones."""
+    if kernel != DECODE_CAPTURE["kernel"] or not DECODE_CAPTURE["sha256"]:
+        return None
+    if sources_sha256(DECODE_CAPTURE["sources"]) != DECODE_CAPTURE["sha256"]:
         return None
     per_byte = (DECODE_CAPTURE["dram_bytes_read"] + DECODE_CAPTURE["dram_bytes_write"]) / \
         DECODE_CAPTURE["kv_bytes"]
@@ -548,7 +559,9 @@ def main():
         torch.cuda.empty_cache()
     if not args.no_prefill:
         pw = W.chunked_prefill()
-        pdw = DeviceWorkload(pw, dev, fill=None)
+        # the key-split call with the automatic split count (3 on 148 SMs:
+        # 384 tile CTAs fill 2.59 of 3 waves, 1152 third-length ones 7.78 of 8)
+        pdw = DeviceWorkload(pw, dev, fill=None, prefill_splits=0)
         pdw.fill_context()
         pdw.load_step_inputs()
         pdw.append(stream)
@@ -567,7 +580,10 @@ def main():
         pairs = sum(int(pw.ctx[0]) + i + 1 for i in range(pw.T))  # causal (query, key) pairs
         flops = 4.0 * pw.head_dim * pw.num_q_heads * pairs
         tf_peak, tf_kind = bf16_peak()
-        prefill = {"workload": pw.name, "ms": p_ms, "tflops": flops / (p_ms * 1e-3) / 1e12,
+        prefill = {"workload": pw.name, "kernel": "prefill_tc",
+                   "num_splits": nv.nvkv_prefill_num_splits(pdw.cache, pw.batch, pw.T,
+                                                            pw.num_q_heads),
+                   "ms": p_ms, "tflops": flops / (p_ms * 1e-3) / 1e12,
                    "flop_per_call": flops, "bound": "tensor", "peak_tflops": tf_peak,
                    "peak_kind": tf_kind, "frac": flops / (p_ms * 1e-3) / 1e12 / tf_peak,
                    "frac_datasheet": flops / (p_ms * 1e-3) / 1e12 / DATASHEET_BF16_TFLOPS,

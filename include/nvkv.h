@@ -231,6 +231,46 @@ nvkv_status nvkv_prefill_attn(const nvkv_cache *cache, const nvkv_seqs *seqs, co
                               int32_t num_q_heads, float sm_scale, void *out,
                               nvkv_stream_t stream);
 
+/* The same chunked prefill with each query tile's keys split into
+ * num_splits equal runs of 64-key tiles, one CTA each, so that the grid of
+ * tile CTAs fills the GPU's last wave (one CTA of the head_dim-256
+ * tensor-core kernel per SM).  Every split leaves, per query row, its
+ * softmax-normalised partial output O_s and lse_s = log2 of its sum of
+ * weights (in the base-2 score scale), and a merge kernel writes
+ * out = sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M), M = max_s lse_s:
+ * the log-sum-exp combination of partial softmax results, the same merge
+ * the decode splits use (the result equals one pass up to fp32 rounding;
+ * a row no split sees a key of is 0).
+ *   num_splits: 0 = automatic -- the count in 1..4 whose CTAs fill their
+ *               last wave best on this device, 1 only unless another raises
+ *               that fill by more than 3 % (nvkv_prefill_num_splits tells
+ *               which); 1..4 = that count; others NVKV_ERR_INVALID_ARG.
+ *   workspace:  device, 16-byte aligned, caller-owned, at least
+ *               nvkv_prefill_workspace_bytes(total_q, Hq, D, num_splits)
+ *               bytes when the resolved count is above 1 (else unused, may
+ *               be NULL); NVKV_ERR_WORKSPACE otherwise.  Layout: fp32
+ *               [S][total_q][Hq][D] partial outputs, then (at a 256-byte
+ *               boundary) fp32 [S][total_q][Hq] lse.  Its contents need no
+ *               initialisation.
+ * Shapes the tensor-core kernel does not take (head_dim 128), and
+ * NVKV_DECODE_KERNEL=simt, run the CUDA-core kernel of nvkv_prefill_attn
+ * and ignore the workspace.
+ * nvkv_prefill_workspace_bytes: bytes for num_splits (0: for the largest
+ * count the automatic choice takes, 4); 0 when no workspace is needed
+ * (num_splits 1) and on invalid arguments.
+ * nvkv_prefill_num_splits: the count num_splits = 0 resolves to for batch
+ * sequences of at most max_q new queries (1 where the CUDA-core kernel
+ * runs); 0 on invalid arguments. */
+size_t nvkv_prefill_workspace_bytes(int32_t total_q, int32_t num_q_heads, int32_t head_dim,
+                                    int32_t num_splits);
+int32_t nvkv_prefill_num_splits(const nvkv_cache *cache, int32_t batch, int32_t max_q,
+                                int32_t num_q_heads);
+nvkv_status nvkv_prefill_attn_split(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *q,
+                                    const int32_t *cu_q, int32_t total_q, int32_t max_q,
+                                    int32_t num_q_heads, float sm_scale, int32_t num_splits,
+                                    void *workspace, size_t workspace_bytes, void *out,
+                                    nvkv_stream_t stream);
+
 /* Rotary position embedding of K fused with the quantise-append: the YaRN
  * context extension of the "gzenz/ninfer" README, "Fork changes vs
  * upstream" -> "Context and model", stated there as linear RoPE scaling

@@ -25,7 +25,8 @@ __all__ = [
     "nvkv_decode_static_scratch_bytes", "nvkv_rope_table", "nvkv_append_rope",
     "nvkv_pages_spill", "nvkv_pages_restore", "nvkv_k8v4_page_bytes", "nvkv_append_k8v4",
     "nvkv_decode_attn_k8v4", "nvkv_prefill_attn_k8v4", "nvkv_pages_spill_k8v4",
-    "nvkv_pages_restore_k8v4",
+    "nvkv_pages_restore_k8v4", "nvkv_prefill_attn_split", "nvkv_prefill_workspace_bytes",
+    "nvkv_prefill_num_splits",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -77,6 +78,10 @@ def library():
             "nvkv_decode_kernel_name_k8v4": (ctypes.c_char_p, [cp, i32, i32]),
             "nvkv_combine": (ctypes.c_int, [sp, vp, i32, i32, i32, i32, i32, vp, vp]),
             "nvkv_prefill_attn": (ctypes.c_int, [cp, sp, vp, vp, i32, i32, i32, f32, vp, vp]),
+            "nvkv_prefill_workspace_bytes": (sz, [i32, i32, i32, i32]),
+            "nvkv_prefill_num_splits": (i32, [cp, i32, i32, i32]),
+            "nvkv_prefill_attn_split": (ctypes.c_int, [cp, sp, vp, vp, i32, i32, i32, f32, i32, vp,
+                                                       sz, vp, vp]),
             "nvkv_decode_static_scratch_bytes": (sz, []),
             "nvkv_decode_attn_static": (ctypes.c_int, [cp, sp, vp, i32, i32, f32, i32, vp, vp]),
             "nvkv_rope_table": (ctypes.c_int, [vp, i32, i32, ctypes.c_double, ctypes.c_double, vp]),
@@ -285,6 +290,35 @@ def nvkv_prefill_attn(cache: Cache, seqs: Seqs, q: torch.Tensor, cu_q: torch.Ten
         ctypes.byref(cache._c), ctypes.byref(seqs._c), _dev(q, torch.bfloat16, "q"),
         _dev(cu_q, torch.int32, "cu_q"), int(total_q), int(max_q), int(num_q_heads),
         float(sm_scale), _dev(out, torch.bfloat16, "out"), _stream(stream)), "nvkv_prefill_attn")
+
+
+def nvkv_prefill_workspace_bytes(total_q: int, num_q_heads: int, head_dim: int,
+                                 num_splits: int) -> int:
+    return int(library().nvkv_prefill_workspace_bytes(int(total_q), int(num_q_heads),
+                                                      int(head_dim), int(num_splits)))
+
+
+def nvkv_prefill_num_splits(cache: Cache, batch: int, max_q: int, num_q_heads: int) -> int:
+    """The key-split count nvkv_prefill_attn_split takes for num_splits = 0."""
+    return int(library().nvkv_prefill_num_splits(ctypes.byref(cache._c), int(batch), int(max_q),
+                                                 int(num_q_heads)))
+
+
+def nvkv_prefill_attn_split(cache: Cache, seqs: Seqs, q: torch.Tensor, cu_q: torch.Tensor,
+                            total_q: int, max_q: int, num_q_heads: int, sm_scale: float,
+                            num_splits: int, workspace: "torch.Tensor | None", out: torch.Tensor,
+                            stream=None) -> None:
+    """Chunked prefill with the keys of each query tile split over num_splits
+    CTAs (0: automatic) and merged; workspace: uint8 device tensor of at least
+    nvkv_prefill_workspace_bytes(...) bytes (None when the count is 1)."""
+    _fmt(cache, "nvfp4", "nvkv_prefill_attn_split")
+    ws = _dev(workspace, torch.uint8, "workspace") if workspace is not None else None
+    nbytes = workspace.numel() if workspace is not None else 0
+    _check(library().nvkv_prefill_attn_split(
+        ctypes.byref(cache._c), ctypes.byref(seqs._c), _dev(q, torch.bfloat16, "q"),
+        _dev(cu_q, torch.int32, "cu_q"), int(total_q), int(max_q), int(num_q_heads),
+        float(sm_scale), int(num_splits), ws, nbytes, _dev(out, torch.bfloat16, "out"),
+        _stream(stream)), "nvkv_prefill_attn_split")
 
 
 def nvkv_decode_static_scratch_bytes() -> int:

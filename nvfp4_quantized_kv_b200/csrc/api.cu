@@ -26,7 +26,10 @@ cudaError_t launch_decode_tc(const nvkv_cache &, const nvkv_seqs &, const void *
                              int, float *, float *, cudaStream_t);
 bool prefill_tc_supported(const nvkv_cache &);
 cudaError_t launch_prefill_tc(const nvkv_cache &, const nvkv_seqs &, const void *, const int32_t *,
-                              int, int, int, float, void *, cudaStream_t);
+                              int, int, int, float, void *, int, float *, float *, cudaStream_t);
+int prefill_max_splits();
+int prefill_auto_splits(int64_t, int);
+int prefill_tc_items(const nvkv_cache &, const nvkv_seqs &, int, int);
 cudaError_t launch_combine(const nvkv_seqs &, const void *, const void *, int, int, int, int, int,
                            void *, cudaStream_t);
 cudaError_t launch_prefill_simt(const nvkv_cache &, const nvkv_seqs &, const void *,
@@ -170,6 +173,17 @@ nvkv_status check_prefill(const nvkv_cache *cache, const nvkv_seqs *seqs, const 
   if (total_q == 0) return NVKV_OK;
   if (!q || !cu_q || !out || !aligned16(q) || !aligned16(out)) return NVKV_ERR_INVALID_ARG;
   return NVKV_OK;
+}
+
+// Workspace of the key-split prefill: S planes of total_q * Hq rows, the
+// rows' O / l (fp32, head_dim each) and then their lse (fp32).
+struct PrefillLayout {
+  size_t lse_off, total;
+};
+PrefillLayout prefill_layout(int64_t total_q, int Hq, int D, int S) {
+  const size_t rows = (size_t)total_q * Hq * S;
+  const size_t lse_off = align256(rows * D * sizeof(float));
+  return {lse_off, lse_off + align256(rows * sizeof(float))};
 }
 
 // NVKV_DECODE_KERNEL=simt forces the CUDA-core decode and prefill kernels;
@@ -335,9 +349,60 @@ nvkv_status nvkv_prefill_attn(const nvkv_cache *cache, const nvkv_seqs *seqs, co
   cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
   if (!force_simt() && prefill_tc_supported(*cache))
     return cuda_status(launch_prefill_tc(*cache, *seqs, q, cu_q, total_q, max_q, num_q_heads,
-                                         sm_scale, out, st_));
+                                         sm_scale, out, 1, nullptr, nullptr, st_));
   return cuda_status(launch_prefill_simt(*cache, *seqs, q, cu_q, total_q, num_q_heads, sm_scale,
                                          out, st_, false));
+}
+
+size_t nvkv_prefill_workspace_bytes(int32_t total_q, int32_t num_q_heads, int32_t head_dim,
+                                    int32_t num_splits) {
+  if (total_q < 0 || num_q_heads <= 0 || head_dim <= 0 || num_splits < 0 ||
+      num_splits > prefill_max_splits())
+    return 0;
+  const int S = num_splits == 0 ? prefill_max_splits() : num_splits;
+  return S > 1 ? prefill_layout(total_q, num_q_heads, head_dim, S).total : 0;
+}
+
+int32_t nvkv_prefill_num_splits(const nvkv_cache *cache, int32_t batch, int32_t max_q,
+                                int32_t num_q_heads) {
+  if (check_cache(cache) != NVKV_OK || batch <= 0 || max_q < 0 || num_q_heads <= 0 ||
+      num_q_heads % cache->num_kv_heads != 0)
+    return 0;
+  if (force_simt() || !prefill_tc_supported(*cache)) return 1;
+  nvkv_seqs s{};
+  s.batch = batch;
+  return prefill_auto_splits(prefill_tc_items(*cache, s, max_q, num_q_heads),
+                             nvkv_default_num_splits());
+}
+
+nvkv_status nvkv_prefill_attn_split(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *q,
+                                    const int32_t *cu_q, int32_t total_q, int32_t max_q,
+                                    int32_t num_q_heads, float sm_scale, int32_t num_splits,
+                                    void *workspace, size_t workspace_bytes, void *out,
+                                    nvkv_stream_t stream) {
+  const nvkv_status st =
+      check_prefill(cache, seqs, q, cu_q, total_q, max_q, num_q_heads, sm_scale, out);
+  if (st != NVKV_OK) return st;
+  if (num_splits < 0 || num_splits > prefill_max_splits()) return NVKV_ERR_INVALID_ARG;
+  if (total_q == 0) return NVKV_OK;
+  cudaStream_t st_ = reinterpret_cast<cudaStream_t>(stream);
+  if (force_simt() || !prefill_tc_supported(*cache))
+    return cuda_status(launch_prefill_simt(*cache, *seqs, q, cu_q, total_q, num_q_heads, sm_scale,
+                                           out, st_, false));
+  const int S = num_splits > 0 ? num_splits
+                               : prefill_auto_splits(
+                                     prefill_tc_items(*cache, *seqs, max_q, num_q_heads),
+                                     nvkv_default_num_splits());
+  float *ws_o = nullptr, *ws_lse = nullptr;
+  if (S > 1) {
+    const PrefillLayout w = prefill_layout(total_q, num_q_heads, cache->head_dim, S);
+    if (!workspace || !aligned16(workspace) || workspace_bytes < w.total)
+      return NVKV_ERR_WORKSPACE;
+    ws_o = static_cast<float *>(workspace);
+    ws_lse = reinterpret_cast<float *>(static_cast<char *>(workspace) + w.lse_off);
+  }
+  return cuda_status(launch_prefill_tc(*cache, *seqs, q, cu_q, total_q, max_q, num_q_heads,
+                                       sm_scale, out, S, ws_o, ws_lse, st_));
 }
 
 size_t nvkv_k8v4_page_bytes(int32_t num_kv_heads, int32_t head_dim) {

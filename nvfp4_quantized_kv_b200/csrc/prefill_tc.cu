@@ -94,8 +94,13 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int H
                   const int32_t *__restrict__ kv_lens, int max_kv_len,
                   const __nv_bfloat16 *__restrict__ q, const int32_t *__restrict__ cu_q,
                   int total_q, int Hq, float qscale, __nv_bfloat16 *__restrict__ out,
+                  int num_splits, float *__restrict__ ws_o, float *__restrict__ ws_lse,
                   int32_t *err) {
-  const int mt = blockIdx.x, h = blockIdx.y, b = blockIdx.z;
+  // blockIdx.x = m-tile * num_splits + split: split s of an m-tile takes the
+  // s-th of num_splits equal runs of its key tiles and, when num_splits > 1,
+  // leaves O / l and log2(l) + m of its rows in the workspace for the merge.
+  const int mt = blockIdx.x / num_splits, split = blockIdx.x % num_splits;
+  const int h = blockIdx.y, b = blockIdx.z;
   const int G = Hq / Hkv;
   const int q0 = cu_q[b];
   const int n_b = cu_q[b + 1] - q0;
@@ -106,9 +111,14 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int H
                    kv_len > max_kv_len || kv_len > max_pages * kPageTokens;
   const int i_first = (128 * mt) / G;
   const int i_last = min(n_b - 1, (128 * mt + 127) / G);
-  const int pos_first = kv_len - n_b + i_first;   // position of the tile's first query token
   const int pos_last = kv_len - n_b + i_last;     // keys 0 .. pos_last are needed
-  const int ntiles = bad ? 0 : pos_last / kTileTokens + 1;
+  const int ntiles_all = bad ? 0 : pos_last / kTileTokens + 1;
+  // This CTA's key tiles j0 .. j0 + ntiles - 1; every ring and barrier below
+  // counts from its first tile.
+  const int j0 = (int)((int64_t)split * ntiles_all / num_splits);
+  const int ntiles = (int)((int64_t)(split + 1) * ntiles_all / num_splits) - j0;
+  // Output rows exist only when the chunk lies inside the total_q rows.
+  const bool rows_ok = n_b >= 0 && q0 >= 0 && q0 + n_b <= total_q;
 
   extern __shared__ uint8_t smem_raw[];
   uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) &
@@ -169,10 +179,10 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int H
       }
       return pg;
     };
-    int cur = ntiles > 0 ? page_for(0) : -1;
+    int cur = ntiles > 0 ? page_for(j0) : -1;
     for (int j = 0; j < ntiles; ++j) {
       const int stage = j % kStages;
-      const int nxt = j + 1 < ntiles ? page_for(j + 1) : -1;
+      const int nxt = j + 1 < ntiles ? page_for(j0 + j + 1) : -1;
       if (j >= kStages) {
         if (lane == 0) wait_bar(&empty[stage], ((j / kStages) + 1) & 1, flags, err);
         __syncwarp();
@@ -261,7 +271,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int H
       wait_bar(&full[stage], (j / kStages) & 1, flags, err);
       const int4 pg4 = *reinterpret_cast<const int4 *>(spages + stage * kTilePages);
       const int pgs[4] = {pg4.x, pg4.y, pg4.z, pg4.w};
-      const int tok0 = j * kTileTokens;
+      const int tok0 = (j0 + j) * kTileTokens;
       {
         // This tile's V scales, converted once: thread t takes 4 consecutive
         // tokens of one (page, group); the 16 V^T rows of a group share them.
@@ -437,7 +447,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int H
           x[48 + e] = __uint_as_float(r3[e]);
         }
       }
-      const int key0 = j * kTileTokens;
+      const int key0 = (j0 + j) * kTileTokens;
       float tmax = -INFINITY;
       if (valid && key0 + kTileTokens - 1 <= pos) {
 #pragma unroll
@@ -502,7 +512,12 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int H
       tc_fence_after();
     }
     const float inv = l > 0.f ? 1.f / l : 0.f;
-    __nv_bfloat16 *orow = out + ((size_t)(q0 + i) * Hq + h * G + g) * kD;
+    const size_t orow_idx = (size_t)(q0 + i) * Hq + h * G + g;
+    const bool write = gr < rows && rows_ok;
+    // Split partial: O / l (fp32) and lse = m + log2(l), -inf without a
+    // visible key, in the split's plane of total_q * Hq rows.
+    const size_t plane = (size_t)split * total_q * Hq;
+    if (ws_o && write) ws_lse[plane + orow_idx] = l > 0.f ? m + log2f(l) : -INFINITY;
 #pragma unroll 1
     for (int c16 = 0; c16 < kD / 16; ++c16) {
       uint32_t rr[16];
@@ -513,14 +528,23 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int H
 #pragma unroll
         for (int e = 0; e < 16; ++e) rr[e] = 0u;
       }
-      uint32_t ow[8];
+      if (!write) continue;
+      if (ws_o) {
+        float4 *dst = reinterpret_cast<float4 *>(ws_o + (plane + orow_idx) * kD + c16 * 16);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(rr[2 * e]) * inv,
-                                                  __uint_as_float(rr[2 * e + 1]) * inv);
-        ow[e] = *reinterpret_cast<uint32_t *>(&b2);
-      }
-      if (gr < rows) {
+        for (int e4 = 0; e4 < 4; ++e4)
+          dst[e4] = make_float4(__uint_as_float(rr[4 * e4]) * inv, __uint_as_float(rr[4 * e4 + 1]) * inv,
+                                __uint_as_float(rr[4 * e4 + 2]) * inv,
+                                __uint_as_float(rr[4 * e4 + 3]) * inv);
+      } else {
+        uint32_t ow[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          __nv_bfloat162 b2 = __floats2bfloat162_rn(__uint_as_float(rr[2 * e]) * inv,
+                                                    __uint_as_float(rr[2 * e + 1]) * inv);
+          ow[e] = *reinterpret_cast<uint32_t *>(&b2);
+        }
+        __nv_bfloat16 *orow = out + orow_idx * kD;
         *reinterpret_cast<uint4 *>(orow + c16 * 16) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
         *reinterpret_cast<uint4 *>(orow + c16 * 16 + 8) = make_uint4(ow[4], ow[5], ow[6], ow[7]);
       }
@@ -533,25 +557,109 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int H
   if (warp == kMmaWarp) tmem_dealloc(tmem, kTmemCols);
 }
 
+// Merge of the key splits: row (token q0 + i, head hq) of sequence b is
+// sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M) with M the largest lse (the
+// log-sum-exp combination of partial softmax results; zero when no split saw
+// a key).  One warp per row, 8 head_dim elements per lane.
+constexpr int kMaxSplits = 4;
+constexpr int kMergeWarps = 8;
+
+__global__ void __launch_bounds__(kMergeWarps * 32)
+prefill_merge_kernel(const float *__restrict__ ws_o, const float *__restrict__ ws_lse,
+                     int num_splits, const int32_t *__restrict__ cu_q, int total_q, int Hq,
+                     int G, int row_cap, __nv_bfloat16 *__restrict__ out) {
+  const int b = blockIdx.y;
+  const int q0 = cu_q[b], n_b = cu_q[b + 1] - q0;
+  if (n_b <= 0 || q0 < 0 || q0 + n_b > total_q) return;  // no output rows (as in the attention)
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t idx = (int64_t)blockIdx.x * kMergeWarps + warp;  // token idx / Hq, head idx % Hq
+  if (idx >= (int64_t)n_b * Hq) return;
+  // only the rows the attention grid covers (tile rows i*G + g < row_cap)
+  if ((idx / Hq) * G + (idx % Hq) % G >= row_cap) return;
+  const size_t row = (size_t)q0 * Hq + idx;
+  const size_t plane = (size_t)total_q * Hq;
+  float lse[kMaxSplits], mx = -INFINITY;
+#pragma unroll
+  for (int s = 0; s < kMaxSplits; ++s) {
+    lse[s] = s < num_splits ? ws_lse[s * plane + row] : -INFINITY;
+    mx = fmaxf(mx, lse[s]);
+  }
+  float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f}, wsum = 0.f;
+  if (mx > -INFINITY) {
+#pragma unroll
+    for (int s = 0; s < kMaxSplits; ++s) {
+      if (s < num_splits && lse[s] > -INFINITY) {
+        const float w = exp2f(lse[s] - mx);
+        const float4 *src = reinterpret_cast<const float4 *>(ws_o + (s * plane + row) * kD + 8 * lane);
+        const float4 a = src[0], c = src[1];
+        acc[0] += w * a.x; acc[1] += w * a.y; acc[2] += w * a.z; acc[3] += w * a.w;
+        acc[4] += w * c.x; acc[5] += w * c.y; acc[6] += w * c.z; acc[7] += w * c.w;
+        wsum += w;
+      }
+    }
+  }
+  const float inv = wsum > 0.f ? 1.f / wsum : 0.f;
+  uint32_t ow[4];
+#pragma unroll
+  for (int e = 0; e < 4; ++e) {
+    __nv_bfloat162 b2 = __floats2bfloat162_rn(acc[2 * e] * inv, acc[2 * e + 1] * inv);
+    ow[e] = *reinterpret_cast<uint32_t *>(&b2);
+  }
+  *reinterpret_cast<uint4 *>(out + row * kD + 8 * lane) = make_uint4(ow[0], ow[1], ow[2], ow[3]);
+}
+
 }  // namespace
 
 bool prefill_tc_supported(const nvkv_cache &c) { return c.head_dim == kD; }
 
+int prefill_max_splits() { return kMaxSplits; }
+
+// Key splits for a grid of `items` (m-tile, kv-head, sequence) CTAs on `sms`
+// SMs (one CTA per SM): the count in 1 .. kMaxSplits whose CTAs fill their
+// last wave best, taken only when it raises the fill by more than 3 % (each
+// split writes and merges a partial result of its rows).
+int prefill_auto_splits(int64_t items, int sms) {
+  if (items <= 0 || sms <= 0) return 1;
+  auto fill = [&](int k) {
+    const int64_t n = items * k;
+    return (double)n / (double)(((n + sms - 1) / sms) * sms);
+  };
+  int best = 1;
+  for (int k = 2; k <= kMaxSplits; ++k)
+    if (fill(k) > fill(best) + 0.03) best = k;
+  return best;
+}
+
+int prefill_tc_items(const nvkv_cache &c, const nvkv_seqs &s, int max_q, int Hq) {
+  const int G = Hq / c.num_kv_heads;
+  return (int)(((int64_t)max_q * G + 127) / 128) * c.num_kv_heads * s.batch;
+}
+
 cudaError_t launch_prefill_tc(const nvkv_cache &c, const nvkv_seqs &s, const void *q,
                               const int32_t *cu_q, int total_q, int max_q, int Hq,
-                              float sm_scale, void *out, cudaStream_t stream) {
+                              float sm_scale, void *out, int num_splits, float *ws_o,
+                              float *ws_lse, cudaStream_t stream) {
   CUtensorMap map;
   if (!make_pool_tmap(c, &map)) return cudaErrorNotSupported;
+  if (num_splits < 1 || num_splits > kMaxSplits || (num_splits > 1 && (!ws_o || !ws_lse)))
+    return cudaErrorInvalidValue;
   const int G = Hq / c.num_kv_heads;
   const int mtiles = (max_q * G + 127) / 128;
   cudaError_t e = cudaFuncSetAttribute(prefill_tc_kernel,
                                        cudaFuncAttributeMaxDynamicSharedMemorySize, kSmemBytes);
   if (e != cudaSuccess) return e;
-  dim3 grid((unsigned)mtiles, (unsigned)c.num_kv_heads, (unsigned)s.batch);
+  dim3 grid((unsigned)(mtiles * num_splits), (unsigned)c.num_kv_heads, (unsigned)s.batch);
   prefill_tc_kernel<<<grid, kThreads, kSmemBytes, stream>>>(
       map, c.num_pages, c.num_kv_heads, s.page_table, s.max_pages_per_seq, s.kv_lens,
       s.max_kv_len, static_cast<const __nv_bfloat16 *>(q), cu_q, total_q, Hq,
-      sm_scale * 1.4426950408889634f, static_cast<__nv_bfloat16 *>(out), s.err_word);
+      sm_scale * 1.4426950408889634f, static_cast<__nv_bfloat16 *>(out), num_splits,
+      num_splits > 1 ? ws_o : nullptr, ws_lse, s.err_word);
+  if ((e = cudaGetLastError()) != cudaSuccess || num_splits == 1) return e;
+  const dim3 mgrid((unsigned)(((int64_t)max_q * Hq + kMergeWarps - 1) / kMergeWarps),
+                   (unsigned)s.batch);
+  prefill_merge_kernel<<<mgrid, kMergeWarps * 32, 0, stream>>>(
+      ws_o, ws_lse, num_splits, cu_q, total_q, Hq, G, 128 * mtiles,
+      static_cast<__nv_bfloat16 *>(out));
   return cudaGetLastError();
 }
 

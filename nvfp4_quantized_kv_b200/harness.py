@@ -13,7 +13,7 @@ import torch
 
 from . import (Cache, Seqs, nvkv_append, nvkv_append_k8v4, nvkv_combine, nvkv_decode_attn,
                nvkv_decode_attn_k8v4, nvkv_decode_workspace_bytes, nvkv_prefill_attn,
-               nvkv_prefill_attn_k8v4)
+               nvkv_prefill_attn_k8v4, nvkv_prefill_attn_split, nvkv_prefill_workspace_bytes)
 
 # The calls of each cache format: (append, decode partials, prefill).
 _CALLS = {
@@ -37,11 +37,13 @@ def bf16_tensor(bits: np.ndarray, device) -> torch.Tensor:
 class DeviceWorkload:
     def __init__(self, wl: Workload, device="cuda", fill: int | None = 0xA5, num_splits: int = 0,
                  err_word: bool = True, cache_from: "DeviceWorkload | None" = None,
-                 kv_format: str = "nvfp4"):
+                 kv_format: str = "nvfp4", prefill_splits: "int | None" = None):
         """cache_from: reuse the (already filled) pool of another workload
         with the same cached context -- same seed, lengths, heads and page
         table -- under a different step shape (T=1 decode and T=6 verify).
-        kv_format: "nvfp4" (the default) or "k8v4"."""
+        kv_format: "nvfp4" (the default) or "k8v4".
+        prefill_splits: None runs nvkv_prefill_attn; a count (0: automatic)
+        runs nvkv_prefill_attn_split with a workspace (NVFP4 only)."""
         if kv_format not in _CALLS:
             raise ValueError(f"kv_format must be one of {tuple(_CALLS)}")
         self.kv_format = kv_format
@@ -74,6 +76,13 @@ class DeviceWorkload:
             self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=self.device)
         else:
             self.workspace = None
+        self.prefill_splits = prefill_splits
+        if wl.mode != "decode" and prefill_splits is not None:
+            if kv_format != "nvfp4":
+                raise ValueError("the key-split prefill takes an NVFP4 cache")
+            nbytes = nvkv_prefill_workspace_bytes(rows, wl.num_q_heads, wl.head_dim,
+                                                  prefill_splits)
+            self.workspace = torch.empty(max(nbytes, 16), dtype=torch.uint8, device=self.device)
         self.k_new = self.v_new = self.cu_new = self.q = None
 
     # ---- context ---------------------------------------------------------
@@ -115,6 +124,10 @@ class DeviceWorkload:
                          self.num_splits, self.workspace, stream)
             nvkv_combine(self.seqs, self.workspace, wl.T, wl.num_q_heads, wl.num_kv_heads,
                          wl.head_dim, self.num_splits, self.out, stream)
+        elif self.prefill_splits is not None:
+            nvkv_prefill_attn_split(self.cache, self.seqs, self.q, self.cu_new, wl.batch * wl.T,
+                                    wl.T, wl.num_q_heads, wl.sm_scale, self.prefill_splits,
+                                    self.workspace, self.out, stream)
         else:
             self._prefill(self.cache, self.seqs, self.q, self.cu_new, wl.batch * wl.T, wl.T,
                           wl.num_q_heads, wl.sm_scale, self.out, stream)

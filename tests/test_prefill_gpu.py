@@ -1,8 +1,9 @@
-"""GPU parity of chunked-prefill attention (nvkv_prefill_attn) against the
-float64 oracle: a chunk of new queries, appended first, attends causally to
-the whole cache of its sequence.  head_dim 256 runs on the tensor-core
-kernel, head_dim 128 on the CUDA-core kernel; NVKV_DECODE_KERNEL=simt forces
-the latter for cross-checks."""
+"""GPU parity of chunked-prefill attention (nvkv_prefill_attn and the
+key-split nvkv_prefill_attn_split) against the float64 oracle: a chunk of new
+queries, appended first, attends causally to the whole cache of its
+sequence.  head_dim 256 runs on the tensor-core kernel, head_dim 128 on the
+CUDA-core kernel; NVKV_DECODE_KERNEL=simt forces the latter for
+cross-checks."""
 import zlib
 
 import numpy as np
@@ -27,8 +28,8 @@ SMALL = [
 ]
 
 
-def run(wl):
-    dw = DeviceWorkload(wl)
+def run(wl, prefill_splits=None):
+    dw = DeviceWorkload(wl, prefill_splits=prefill_splits)
     dw.fill_context()
     dw.load_step_inputs()
     dw.step()
@@ -63,11 +64,20 @@ def test_prefill_kernels_agree(case, monkeypatch):
         assert_close(gpu_rows(dw.out, wl, rows), ref, f"{name}/{kernel}")
 
 
-def test_chunked_prefill_config_sampled():
+@pytest.mark.parametrize("splits", [None, 0], ids=["unsplit", "auto_split"])
+def test_chunked_prefill_config_sampled(splits):
     """65536 cached tokens + a 2048-token chunk, 24/4 heads, head_dim 256:
-    the first 64, the last 64 and every 31st chunk query, all heads."""
+    the first 64, the last 64 and every 31st chunk query, all heads; through
+    nvkv_prefill_attn and through the key-split call with the automatic
+    count (the launch the benchmark times: 3 splits on 148 SMs)."""
+    import nvfp4_quantized_kv_b200 as nv
     wl = W.chunked_prefill()
-    dw = run(wl)
+    dw = run(wl, prefill_splits=splits)
+    if splits == 0:
+        S = nv.nvkv_prefill_num_splits(dw.cache, wl.batch, wl.T, wl.num_q_heads)
+        assert 1 <= S <= 4
+        if torch.cuda.get_device_properties(0).multi_processor_count == 148:
+            assert S == 3
     rows = [(0, t, hq) for t in prefill_sample_queries(wl.T) for hq in range(wl.num_q_heads)]
     assert_close(gpu_rows(dw.out, wl, rows), oracle_outputs_dense(wl, rows), wl.name)
 
@@ -105,3 +115,50 @@ def test_prefill_reports_bad_page(kernel, monkeypatch):
     assert int(err.item()) & nv.DEVERR_PAGE_ID
     assert torch.isfinite(out.float()).all()
     assert (out == 0).all()  # an all-zero pool dequantises to 0
+
+
+SPLIT_CASES = [c for c in SMALL if c[4] == 256]
+
+
+@pytest.mark.parametrize("splits", [2, 3, 4])
+@pytest.mark.parametrize("case", SPLIT_CASES, ids=[c[0] for c in SPLIT_CASES])
+def test_prefill_split_small(case, splits):
+    """Every key-split count on the small chunks: ragged chunks, several
+    m-tiles, and chunks with fewer 64-key tiles than splits (empty splits
+    leave lse = -inf, which the merge skips)."""
+    name, b, hq, hkv, d, T, ctx = case
+    wl = W.small(name, b, hq, hkv, d, T, ctx, mode="prefill", seed=seed_of(name))
+    dw = run(wl, prefill_splits=splits)
+    rows = all_rows(wl) if len(all_rows(wl)) <= 2500 else sample_rows(wl, 400, seed=3)
+    assert_close(gpu_rows(dw.out, wl, rows), oracle_outputs(wl, rows), f"{name}/S{splits}")
+
+
+@pytest.mark.parametrize("mode", ["default", "split", "simt"])
+def test_prefill_chunk_past_total_q_writes_no_row_beyond(mode, monkeypatch):
+    """cu_q claims 20 rows but total_q is 12: nothing is written past row 12
+    of out (the tensor-core kernels also report the sequence with
+    NVKV_DEVERR_LENGTH and leave its rows alone)."""
+    import nvfp4_quantized_kv_b200 as nv
+    if mode == "simt":
+        monkeypatch.setenv("NVKV_DECODE_KERNEL", "simt")
+    dev = torch.device("cuda")
+    hkv, hq, d, n, total_q = 2, 12, 256, 20, 12
+    cache = nv.Cache.allocate(2, hkv, d, dev, fill=0)
+    pt = torch.tensor([[0, 1]], dtype=torch.int32, device=dev)
+    lens = torch.tensor([n], dtype=torch.int32, device=dev)
+    err = torch.zeros(1, dtype=torch.int32, device=dev)
+    seqs = nv.Seqs(pt, lens, n, err)
+    q = torch.zeros((n, hq, d), dtype=torch.bfloat16, device=dev)
+    cu = torch.tensor([0, n], dtype=torch.int32, device=dev)
+    out_full = torch.full((n, hq, d), 7.0, dtype=torch.bfloat16, device=dev)
+    out = out_full[:total_q]
+    if mode == "split":
+        ws = torch.empty(nv.nvkv_prefill_workspace_bytes(total_q, hq, d, 2), dtype=torch.uint8,
+                         device=dev)
+        nv.nvkv_prefill_attn_split(cache, seqs, q, cu, total_q, n, hq, 0.0625, 2, ws, out)
+    else:
+        nv.nvkv_prefill_attn(cache, seqs, q, cu, total_q, n, hq, 0.0625, out)
+    torch.cuda.synchronize()
+    assert (out_full[total_q:].float() == 7.0).all()
+    if mode != "simt":
+        assert int(err.item()) & nv.DEVERR_LENGTH
