@@ -559,8 +559,8 @@ def main():
         torch.cuda.empty_cache()
     if not args.no_prefill:
         pw = W.chunked_prefill()
-        # the key-split call with the automatic split count (3 on 148 SMs:
-        # 384 tile CTAs fill 2.59 of 3 waves, 1152 third-length ones 7.78 of 8)
+        # the key-split call with the automatic split count (5 on 148 SMs:
+        # 384 tile CTAs fill 2.59 of 3 waves, 1920 fifth-length ones 12.97 of 13)
         pdw = DeviceWorkload(pw, dev, fill=None, prefill_splits=0)
         pdw.fill_context()
         pdw.load_step_inputs()

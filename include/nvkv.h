@@ -241,10 +241,11 @@ nvkv_status nvkv_prefill_attn(const nvkv_cache *cache, const nvkv_seqs *seqs, co
  * the log-sum-exp combination of partial softmax results, the same merge
  * the decode splits use (the result equals one pass up to fp32 rounding;
  * a row no split sees a key of is 0).
- *   num_splits: 0 = automatic -- the count in 1..4 whose CTAs fill their
- *               last wave best on this device, 1 only unless another raises
- *               that fill by more than 3 % (nvkv_prefill_num_splits tells
- *               which); 1..4 = that count; others NVKV_ERR_INVALID_ARG.
+ *   num_splits: 0 = automatic -- the count in 1..8 whose CTAs fill their
+ *               last wave best on this device, a larger count only where it
+ *               raises that fill by more than 1 % (nvkv_prefill_num_splits
+ *               tells which); 1..8 = that count; others
+ *               NVKV_ERR_INVALID_ARG.
  *   workspace:  device, 16-byte aligned, caller-owned, at least
  *               nvkv_prefill_workspace_bytes(total_q, Hq, D, num_splits)
  *               bytes when the resolved count is above 1 (else unused, may
@@ -256,7 +257,7 @@ nvkv_status nvkv_prefill_attn(const nvkv_cache *cache, const nvkv_seqs *seqs, co
  * NVKV_DECODE_KERNEL=simt, run the CUDA-core kernel of nvkv_prefill_attn
  * and ignore the workspace.
  * nvkv_prefill_workspace_bytes: bytes for num_splits (0: for the largest
- * count the automatic choice takes, 4); 0 when no workspace is needed
+ * count the automatic choice takes, 8); 0 when no workspace is needed
  * (num_splits 1) and on invalid arguments.
  * nvkv_prefill_num_splits: the count num_splits = 0 resolves to for batch
  * sequences of at most max_q new queries (1 where the CUDA-core kernel

@@ -309,7 +309,7 @@ def nvkv_prefill_attn_split(cache: Cache, seqs: Seqs, q: torch.Tensor, cu_q: tor
                             num_splits: int, workspace: "torch.Tensor | None", out: torch.Tensor,
                             stream=None) -> None:
     """Chunked prefill with the keys of each query tile split over num_splits
-    CTAs (0: automatic) and merged; workspace: uint8 device tensor of at least
+    (1..8) CTAs (0: automatic) and merged; workspace: uint8 device tensor of at least
     nvkv_prefill_workspace_bytes(...) bytes (None when the count is 1)."""
     _fmt(cache, "nvfp4", "nvkv_prefill_attn_split")
     ws = _dev(workspace, torch.uint8, "workspace") if workspace is not None else None

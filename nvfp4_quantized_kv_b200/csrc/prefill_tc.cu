@@ -561,7 +561,7 @@ prefill_tc_kernel(const __grid_constant__ CUtensorMap tmap, int num_pages, int H
 // sum_s 2^(lse_s - M) O_s / sum_s 2^(lse_s - M) with M the largest lse (the
 // log-sum-exp combination of partial softmax results; zero when no split saw
 // a key).  One warp per row, 8 head_dim elements per lane.
-constexpr int kMaxSplits = 4;
+constexpr int kMaxSplits = 8;
 constexpr int kMergeWarps = 8;
 
 __global__ void __launch_bounds__(kMergeWarps * 32)
@@ -616,8 +616,10 @@ int prefill_max_splits() { return kMaxSplits; }
 
 // Key splits for a grid of `items` (m-tile, kv-head, sequence) CTAs on `sms`
 // SMs (one CTA per SM): the count in 1 .. kMaxSplits whose CTAs fill their
-// last wave best, taken only when it raises the fill by more than 3 % (each
-// split writes and merges a partial result of its rows).
+// last wave best, a larger count taken only when it raises the fill by more
+// than 1 % (each split writes and merges a partial result of its rows).  The
+// 384 CTAs of a 2048-token chunk at 24/4 heads fill 2.59 of 3 waves; 5
+// splits fill 12.97 of 13.
 int prefill_auto_splits(int64_t items, int sms) {
   if (items <= 0 || sms <= 0) return 1;
   auto fill = [&](int k) {
@@ -626,7 +628,7 @@ int prefill_auto_splits(int64_t items, int sms) {
   };
   int best = 1;
   for (int k = 2; k <= kMaxSplits; ++k)
-    if (fill(k) > fill(best) + 0.03) best = k;
+    if (fill(k) > fill(best) + 0.01) best = k;
   return best;
 }
 

@@ -113,23 +113,23 @@ def test_split_prefill_host_logic(lib):
     """Workspace bytes of the key-split prefill, its argument checks (before
     any launch) and the automatic split count (148 SMs when no GPU is
     visible): the chunked-prefill grid of 96 m-tiles x 4 kv-heads = 384 CTAs
-    fills 2.59 of 3 waves, 3 splits fill 7.78 of 8; a 148-CTA grid stays
-    whole; a 100-CTA grid fills 0.68 whole, split in 2 or 3 the same, in 4
-    0.90."""
+    fills 2.59 of 3 waves, 3 splits fill 7.78 of 8 (0.973), 5 splits 12.97
+    of 13 (0.998); a 148-CTA grid stays whole; a 100-CTA grid fills 0.68
+    whole, 0.90 in 4 splits, 0.95 in 7."""
     B = ctypes.byref
     a256 = lambda x: (x + 255) // 256 * 256
     for tq, hq, d, S in [(2048, 24, 256, 3), (37, 12, 256, 2), (1, 8, 128, 4)]:
         rows = tq * hq * S
         assert lib.nvkv_prefill_workspace_bytes(tq, hq, d, S) == a256(rows * d * 4) + a256(rows * 4)
     assert lib.nvkv_prefill_workspace_bytes(2048, 24, 256, 0) == \
-        lib.nvkv_prefill_workspace_bytes(2048, 24, 256, 4)
+        lib.nvkv_prefill_workspace_bytes(2048, 24, 256, 8)
     assert lib.nvkv_prefill_workspace_bytes(2048, 24, 256, 1) == 0
-    assert lib.nvkv_prefill_workspace_bytes(2048, 24, 256, 5) == 0
+    assert lib.nvkv_prefill_workspace_bytes(2048, 24, 256, 9) == 0
     assert lib.nvkv_prefill_workspace_bytes(-1, 24, 256, 2) == 0
     c, s = cache(hkv=4, d=256), seqs()
     f = lib.nvkv_prefill_attn_split
     need = lib.nvkv_prefill_workspace_bytes(10, 24, 256, 2)
-    assert f(B(c), B(s), 0x100, 0x200, 10, 10, 24, 0.1, 5, None, 0, 0x300, None) == nv.ERR_INVALID_ARG
+    assert f(B(c), B(s), 0x100, 0x200, 10, 10, 24, 0.1, 9, None, 0, 0x300, None) == nv.ERR_INVALID_ARG
     assert f(B(c), B(s), 0x100, 0x200, 10, 10, 24, 0.1, -1, None, 0, 0x300, None) == nv.ERR_INVALID_ARG
     assert f(B(c), B(s), 0x100, 0x200, 10, 10, 25, 0.1, 2, None, 0, 0x300, None) == nv.ERR_INVALID_ARG
     assert f(B(c), B(s), 0x100, 0x200, 10, 10, 24, 0.1, 2, None, 0, 0x300, None) == nv.ERR_WORKSPACE
@@ -139,9 +139,9 @@ def test_split_prefill_host_logic(lib):
         nv.ERR_WORKSPACE
     assert f(B(c), B(s), None, None, 0, 0, 24, 0.1, 2, None, 0, None, None) == nv.OK
     n = lib.nvkv_prefill_num_splits
-    assert n(B(c), 1, 2048, 24) == 3
+    assert n(B(c), 1, 2048, 24) == 5
     assert n(B(c), 1, 789, 24) == 1      # ceil(789 * 6 / 128) = 37 m-tiles x 4 = 148 CTAs
-    assert n(B(c), 1, 533, 24) == 4      # 25 m-tiles x 4 = 100 CTAs
+    assert n(B(c), 1, 533, 24) == 7      # 25 m-tiles x 4 = 100 CTAs
     assert n(B(cache(hkv=4, d=128)), 1, 2048, 24) == 1  # CUDA-core kernel
     assert n(B(c), 1, 2048, 25) == 0 and n(None, 1, 2048, 24) == 0
 

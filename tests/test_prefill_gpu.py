@@ -69,15 +69,15 @@ def test_chunked_prefill_config_sampled(splits):
     """65536 cached tokens + a 2048-token chunk, 24/4 heads, head_dim 256:
     the first 64, the last 64 and every 31st chunk query, all heads; through
     nvkv_prefill_attn and through the key-split call with the automatic
-    count (the launch the benchmark times: 3 splits on 148 SMs)."""
+    count (the launch the benchmark times: 5 splits on 148 SMs)."""
     import nvfp4_quantized_kv_b200 as nv
     wl = W.chunked_prefill()
     dw = run(wl, prefill_splits=splits)
     if splits == 0:
         S = nv.nvkv_prefill_num_splits(dw.cache, wl.batch, wl.T, wl.num_q_heads)
-        assert 1 <= S <= 4
+        assert 1 <= S <= 8
         if torch.cuda.get_device_properties(0).multi_processor_count == 148:
-            assert S == 3
+            assert S == 5
     rows = [(0, t, hq) for t in prefill_sample_queries(wl.T) for hq in range(wl.num_q_heads)]
     assert_close(gpu_rows(dw.out, wl, rows), oracle_outputs_dense(wl, rows), wl.name)
 
@@ -120,7 +120,7 @@ def test_prefill_reports_bad_page(kernel, monkeypatch):
 SPLIT_CASES = [c for c in SMALL if c[4] == 256]
 
 
-@pytest.mark.parametrize("splits", [2, 3, 4])
+@pytest.mark.parametrize("splits", [2, 3, 5, 8])
 @pytest.mark.parametrize("case", SPLIT_CASES, ids=[c[0] for c in SPLIT_CASES])
 def test_prefill_split_small(case, splits):
     """Every key-split count on the small chunks: ragged chunks, several
