@@ -225,7 +225,11 @@ nvkv_status nvkv_decode_attn_static(const nvkv_cache *cache, const nvkv_seqs *se
  *         cu_q[b] .. cu_q[b+1]-1 are the n_b newest positions of sequence b
  *         (kv_lens[b]-n_b .. kv_lens[b]-1).
  *   total_q = cu_q[batch] (host), max_q >= every n_b (host bound).
- *   out:  device bf16 [total_q][Hq][D]. */
+ *   out:  device bf16 [total_q][Hq][D].
+ * Device-side: a page id outside the pool sets NVKV_DEVERR_PAGE_ID (its keys
+ * read as absent); a kv_len beyond max_kv_len or the page table, or (on the
+ * tensor-core kernel) a chunk reaching past total_q, sets
+ * NVKV_DEVERR_LENGTH.  No row at or past total_q is ever written. */
 nvkv_status nvkv_prefill_attn(const nvkv_cache *cache, const nvkv_seqs *seqs, const void *q,
                               const int32_t *cu_q, int32_t total_q, int32_t max_q,
                               int32_t num_q_heads, float sm_scale, void *out,
