@@ -69,9 +69,9 @@ DECODE_CAPTURE = {
                 "nvfp4_quantized_kv_b200/csrc/sm100.cuh",
                 "nvfp4_quantized_kv_b200/csrc/nvkv_common.cuh",
                 "include/nvkv.h"],
-    "sha256": "ff1d0ce95f87c7ae6ba420ea1b189f0cb41e54b715274f76871d411ec66ee6e6",
-    "dram_bytes_read": 207593216,
-    "dram_bytes_write": 4328192,
+    "sha256": "cc497b3949b877049093e0c373fdab8f332cd7d4eeca000e7c4e2d88e85a02cb",
+    "dram_bytes_read": 207595776,
+    "dram_bytes_write": 3718912,
     "kv_bytes": 207363456,
 }
 
